@@ -1,0 +1,339 @@
+"""Plain fp64 CPU oracle of the sparse Mixture-of-Experts FFN layer forward.
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+benchmark's CPU legs may use this module; the product path never does.  It
+shares no code with the CUDA library.
+
+Inputs are the exact (bf16- or fp32-rounded) values the GPU sees, widened to
+fp64; every step below runs in fp64 with NumPy.  Each function follows one
+passage of the source pages, cited by page title and section/equation:
+
+  [GLaM]     "GLaM" architecture note, section "Sparse MoE Layer"
+             (eq. FFN, eq. r_t, eq. S_t, eq. MoE).
+  [GLM45-SE] "Shared Expert" study note for GLM-4.5, section "How it works"
+             (E_sh, the sigmoid router with correction bias, eq. g-bar,
+             w_i = alpha g-bar_i, eq. y).
+  [GLM5-SE]  "GLM-5 - Shared expert" (OpenModelAtlas), sections "All 5 steps",
+             "Exact per-instance accounting" and the quoted
+             GlmMoeDsaExperts / GlmMoeDsaMoE / GlmMoeDsaMLP forward excerpts.
+
+Readings taken where the pages leave a step open (each is also listed in the
+design notes):
+  * GLaM's "normalized gate weight": the softmax probabilities of the k
+    selected experts renormalised to sum to one; because the full softmax
+    denominator cancels, alpha_j = exp(l_j - l_max) / sum_S exp(l - l_max).
+  * GLaM's sigma: GELU with the tanh approximation.
+  * The correction bias enters the selection only; weights use the unbiased
+    sigmoid scores g_i.
+  * Selection order: descending score, exact ties to the lower expert index;
+    slot j of a token is its j-th largest score.
+  * Dispatch order inside an expert's segment: by (slot j, then token t),
+    the order the quoted GlmMoeDsaExperts.forward enumerates with
+    ``torch.where`` over the [k, T] expert mask.
+  * The routed weight multiplies b2 too: w * (W2 h + b2).
+
+Pins: every function here is checked, independently of its own code, by
+tests/test_oracle_pins.py (library routines, closed forms, invariants, brute
+force over all experts on tiny inputs, and the parameter counts the GLM-5 page
+prints).  The pages print no worked example of a layer output, so full-size
+outputs rest on this definition plus those pins.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "gelu_tanh", "silu", "sigmoid", "router_logits", "selection_scores",
+    "topk_select", "topk_weights", "route", "permute", "expert_ffn",
+    "shared_expert", "moe_tokens", "moe_forward", "adopt_topk",
+    "param_count", "error_metrics",
+]
+
+
+def _f64(a):
+    return np.asarray(a, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Activations
+# ---------------------------------------------------------------------------
+
+def gelu_tanh(v):
+    """sigma of [GLaM] eq. FFN, read as GELU with the tanh approximation:
+    0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3)))."""
+    v = _f64(v)
+    return 0.5 * v * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (v + 0.044715 * v ** 3)))
+
+
+def sigmoid(v):
+    v = _f64(v)
+    return 1.0 / (1.0 + np.exp(-v))
+
+
+def silu(v):
+    """[GLM5-SE] "All 5 steps": a = g * sigmoid(g)."""
+    v = _f64(v)
+    return v * sigmoid(v)
+
+
+# ---------------------------------------------------------------------------
+# Router
+# ---------------------------------------------------------------------------
+
+def router_logits(x, w_r):
+    """Raw router scores W_r x_t for every token ([GLaM] eq. r_t before the
+    softmax; [GLM45-SE] "a sigmoid router scores the routed experts").
+    x is [T, D]; w_r is stored [D, M], so the scores are x @ w_r."""
+    return _f64(x) @ _f64(w_r)
+
+
+def selection_scores(logits, gate, e_bias=None):
+    """Scores the top-k is taken over, and the gate values the weights use.
+
+    softmax ([GLaM] eq. r_t, eq. S_t): the top-k of softmax(l) is the top-k
+    of l (softmax is monotone), so the selection score is the logit itself.
+    sigmoid_bias ([GLM45-SE]): g = sigmoid(l); selection score g + e_bias.
+    Returns (selection score [T, M], gate value [T, M])."""
+    logits = _f64(logits)
+    if gate == "softmax":
+        return logits, logits
+    if gate == "sigmoid_bias":
+        g = sigmoid(logits)
+        b = np.zeros(logits.shape[1]) if e_bias is None else _f64(e_bias)
+        return g + b[None, :], g
+    raise ValueError(gate)
+
+
+def topk_select(sel, k):
+    """S_t = TopK(score, k) ([GLaM] eq. S_t; [GLM45-SE] "keeps the top 8"):
+    indices of the k largest scores per token, largest first, exact ties to
+    the lower expert index.  A stable sort of -score keeps equal scores in
+    index order."""
+    sel = _f64(sel)
+    order = np.argsort(-sel, axis=1, kind="stable")
+    return order[:, :k].astype(np.int64)
+
+
+def topk_weights(idx, logits, g, gate, norm_topk_prob, alpha, eps):
+    """Gate weights of the selected experts.
+
+    softmax, normalised ([GLaM] eq. MoE, "normalized gate weight"):
+        alpha_j = exp(l_j - l_top) / sum_{i in S} exp(l_i - l_top)
+    softmax, not normalised: the full softmax probability of expert j.
+    sigmoid_bias ([GLM45-SE] eq. g-bar, then w_i = alpha g-bar_i):
+        w_j = alpha * g_j / (sum_{i in S} g_i + eps)   if norm_topk_prob
+        w_j = alpha * g_j                              otherwise
+    routed_scaling_factor (alpha) multiplies every routed weight."""
+    idx = np.asarray(idx)
+    if gate == "softmax":
+        l = _f64(logits)
+        ls = np.take_along_axis(l, idx, axis=1)
+        if norm_topk_prob:
+            e = np.exp(ls - ls.max(axis=1, keepdims=True))
+            w = e / e.sum(axis=1, keepdims=True)
+        else:
+            full = np.exp(l - l.max(axis=1, keepdims=True))
+            full = full / full.sum(axis=1, keepdims=True)
+            w = np.take_along_axis(full, idx, axis=1)
+        return alpha * w
+    if gate == "sigmoid_bias":
+        gs = np.take_along_axis(_f64(g), idx, axis=1)
+        if norm_topk_prob:
+            gs = gs / (gs.sum(axis=1, keepdims=True) + eps)
+        return alpha * gs
+    raise ValueError(gate)
+
+
+def route(x, w_r, e_bias, k, gate, norm_topk_prob, alpha, eps):
+    """The whole router: logits, selection, weights."""
+    logits = router_logits(x, w_r)
+    sel, g = selection_scores(logits, gate, e_bias)
+    idx = topk_select(sel, k)
+    w = topk_weights(idx, logits, g, gate, norm_topk_prob, alpha, eps)
+    return {"logits": logits, "sel": sel, "g": g, "idx": idx, "w": w}
+
+
+def adopt_topk(gpu_idx, sel, rel=1e-5):
+    """Accept a GPU top-k that differs from the oracle's only at near-ties.
+
+    The GPU's choice stands if, for every slot j, the oracle's score of the
+    expert the GPU put in slot j lies within ``rel`` (relative) of the j-th
+    largest oracle score, and its k indices are distinct and in range.
+    Returns (ok, number of tokens whose choice differs, first bad token)."""
+    gpu_idx = np.asarray(gpu_idx, dtype=np.int64)
+    sel = _f64(sel)
+    T, k = gpu_idx.shape
+    M = sel.shape[1]
+    ref = topk_select(sel, k)
+    differ = np.nonzero((gpu_idx != ref).any(axis=1))[0]
+    for t in differ:
+        g = gpu_idx[t]
+        if (g < 0).any() or (g >= M).any() or len(set(g.tolist())) != k:
+            return False, len(differ), int(t)
+        sg = sel[t, g]
+        sr = sel[t, ref[t]]
+        band = rel * np.maximum(np.abs(sg), np.abs(sr))
+        if (np.abs(sg - sr) > band).any():
+            return False, len(differ), int(t)
+    return True, len(differ), -1
+
+
+# ---------------------------------------------------------------------------
+# Dispatch
+# ---------------------------------------------------------------------------
+
+def permute(idx, w, M):
+    """Dispatch order of the (token, slot) pairs.
+
+    [GLM5-SE] GlmMoeDsaExperts.forward: the expert mask one_hot(idx)
+    permuted to [M, k, T]; ``torch.where(expert_mask[e])`` lists expert e's
+    pairs as (slot j, token t) in row-major order.  Laying the experts'
+    lists end to end gives a stable sort by expert of the pairs taken in
+    (j, t) order.  Returns
+      counts[e]       pairs routed to expert e
+      offsets[e]      exclusive prefix sum of counts (offsets[M] = T k)
+      slot_of[t, j]   position of pair (t, j) in the dispatch order
+      row_token[s]    token of the pair at position s
+      row_w[s]        its gate weight w[t, j]
+    """
+    idx = np.asarray(idx, dtype=np.int64)
+    T, k = idx.shape
+    counts = np.bincount(idx.reshape(-1), minlength=M).astype(np.int64)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    jmajor = idx.T.reshape(-1)                      # position p = j*T + t
+    order = np.argsort(jmajor, kind="stable")       # dispatch position -> p
+    slot_jmajor = np.empty(T * k, dtype=np.int64)
+    slot_jmajor[order] = np.arange(T * k)
+    slot_of = slot_jmajor.reshape(k, T).T.copy()
+    row_token = (order % T).astype(np.int64) if T > 0 else order.astype(np.int64)
+    row_w = None
+    if w is not None:
+        row_w = _f64(w).T.reshape(-1)[order]
+    return {"counts": counts, "offsets": offsets, "slot_of": slot_of,
+            "row_token": row_token, "row_w": row_w}
+
+
+# ---------------------------------------------------------------------------
+# Experts
+# ---------------------------------------------------------------------------
+
+def expert_ffn(xe, act, w1e, w2e, b1e=None, b2e=None):
+    """One expert on a batch of rows xe [n, D].
+
+    gelu_tanh ([GLaM] eq. FFN): W2 sigma(W1 x + b1) + b2, with W1 [H, D],
+      W2 [D, H] in the nn.Linear [out, in] layout.
+    swiglu ([GLM45-SE] E_sh; [GLM5-SE] GlmMoeDsaExperts.forward): the
+      fused stack W1 = gate_up [2I, D]; ``linear(x, gate_up).chunk(2)``
+      makes rows 0..I-1 the gate and rows I..2I-1 the up projection;
+      E(x) = W_down (SiLU(W_gate x) * W_up x) with W_down = W2 [D, I]."""
+    xe = _f64(xe)
+    w1e = _f64(w1e)
+    w2e = _f64(w2e)
+    if act == "gelu_tanh":
+        a = xe @ w1e.T
+        if b1e is not None:
+            a = a + _f64(b1e)[None, :]
+        out = gelu_tanh(a) @ w2e.T
+        if b2e is not None:
+            out = out + _f64(b2e)[None, :]
+        return out
+    if act == "swiglu":
+        I = w1e.shape[0] // 2
+        gu = xe @ w1e.T
+        h = silu(gu[:, :I]) * gu[:, I:]
+        return h @ w2e.T
+    raise ValueError(act)
+
+
+def shared_expert(x, sh_w1, sh_w2):
+    """Always-on shared SwiGLU ([GLM45-SE] E_sh; [GLM5-SE] GlmMoeDsaMLP):
+    down(SiLU(gate x) * up x) on every token of the pre-routing x, with
+    gate/up stored as one [2 I_sh, D] stack (gate rows first)."""
+    return expert_ffn(x, "swiglu", sh_w1, sh_w2)
+
+
+def moe_tokens(x_rows, idx_rows, w_rows, act, get_expert, shared=None):
+    """y_t = sum_{j} w_{t,j} E_{idx[t,j]}(x_t) (+ E_sh(x_t)) for given tokens.
+
+    [GLaM] eq. MoE; [GLM45-SE] eq. y (a sum, no residual inside the layer).
+    ``get_expert(e)`` returns (w1e, w2e, b1e, b2e); ``shared`` is
+    (sh_w1, sh_w2) or None.  Rows that chose expert e are batched into one
+    matmul; each row's value is that of its own matrix-vector product."""
+    x_rows = _f64(x_rows)
+    idx_rows = np.asarray(idx_rows, dtype=np.int64)
+    w_rows = _f64(w_rows)
+    n, k = idx_rows.shape
+    y = np.zeros((n, x_rows.shape[1]), dtype=np.float64)
+    for e in np.unique(idx_rows):
+        rr, jj = np.nonzero(idx_rows == e)
+        w1e, w2e, b1e, b2e = get_expert(int(e))
+        out = expert_ffn(x_rows[rr], act, w1e, w2e, b1e, b2e)
+        np.add.at(y, rr, w_rows[rr, jj][:, None] * out)
+    if shared is not None:
+        y = y + shared_expert(x_rows, shared[0], shared[1])
+    return y
+
+
+def moe_forward(cfg, inp, idx=None):
+    """Whole layer: route, dispatch order, experts, combine, shared add.
+
+    ``cfg`` holds T, D, M, k, gate, act, norm_topk_prob, alpha, eps, I_sh;
+    ``inp`` holds numpy arrays x, w_r, e_bias, w1, b1, w2, b2, sh_w1, sh_w2
+    (w1/w2/b1/b2 indexable by expert).  ``idx`` overrides the selection
+    (used when the oracle adopts the GPU's choice at a near-tie)."""
+    r = route(inp["x"], inp["w_r"], inp.get("e_bias"), cfg["k"], cfg["gate"],
+              cfg["norm_topk_prob"], cfg["alpha"], cfg["eps"])
+    if idx is not None:
+        r["idx"] = np.asarray(idx, dtype=np.int64)
+        r["w"] = topk_weights(r["idx"], r["logits"], r["g"], cfg["gate"],
+                              cfg["norm_topk_prob"], cfg["alpha"], cfg["eps"])
+    p = permute(r["idx"], r["w"], cfg["M"])
+
+    def get_expert(e):
+        b1 = inp.get("b1")
+        b2 = inp.get("b2")
+        return (inp["w1"][e], inp["w2"][e],
+                None if b1 is None else b1[e], None if b2 is None else b2[e])
+
+    shared = None
+    if cfg.get("I_sh"):
+        shared = (inp["sh_w1"], inp["sh_w2"])
+    y = moe_tokens(inp["x"], r["idx"], r["w"], cfg["act"], get_expert, shared)
+    out = dict(r)
+    out.update(p)
+    out["y"] = y
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Accounting and comparison
+# ---------------------------------------------------------------------------
+
+def param_count(D, M, I, act, I_sh=0, has_bias=False, router=True, e_bias=False):
+    """Parameters of one MoE layer ([GLM5-SE] "Exact per-instance
+    accounting": gate D*I_sh, up D*I_sh, down I_sh*D for the shared expert;
+    the same per routed SwiGLU expert; GELU experts 2*D*H (+ H + D biases);
+    the router D*M, plus M correction-bias buffer values)."""
+    if act == "swiglu":
+        per = 3 * D * I
+    else:
+        per = 2 * D * I + ((I + D) if has_bias else 0)
+    total = M * per + 3 * D * I_sh
+    if router:
+        total += D * M
+    if e_bias:
+        total += M
+    return total
+
+
+def error_metrics(y, y_ref):
+    """max |y - y_ref| / rms(y_ref) and sum|y - y_ref| / sum|y_ref|."""
+    y = _f64(y)
+    y_ref = _f64(y_ref)
+    d = np.abs(y - y_ref)
+    rms = float(np.sqrt(np.mean(y_ref ** 2))) if y_ref.size else 0.0
+    den = float(np.sum(np.abs(y_ref)))
+    return {
+        "max_over_rms": float(d.max() / rms) if y_ref.size and rms > 0 else 0.0,
+        "mean_rel": float(d.sum() / den) if den > 0 else float(d.sum()),
+    }

@@ -1,0 +1,115 @@
+"""Plant plausible mistakes in a patched copy of the oracle (on the CPU) and
+check that at least one pin fails for each: the pins have teeth."""
+import importlib.util
+import os
+
+import numpy as np
+import pytest
+
+from oracle_pins import ALL_PINS
+
+ORACLE_SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                          "oracle", "moe_oracle.py")
+
+
+def fresh_oracle():
+    spec = importlib.util.spec_from_file_location("oracle_mutant", ORACLE_SRC)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def caught(mod):
+    for pin in ALL_PINS:
+        try:
+            pin(mod)
+        except AssertionError:
+            return pin.__name__
+    return None
+
+
+def m_swap_gate_up(O):
+    orig = O.expert_ffn
+
+    def ffn(xe, act, w1e, w2e, b1e=None, b2e=None):
+        if act == "swiglu":
+            w1e = np.asarray(w1e)
+            I = w1e.shape[0] // 2
+            w1e = np.concatenate([w1e[I:], w1e[:I]])
+        return orig(xe, act, w1e, w2e, b1e, b2e)
+    O.expert_ffn = ffn
+
+
+def m_drop_b2(O):
+    orig = O.expert_ffn
+    O.expert_ffn = lambda xe, act, w1e, w2e, b1e=None, b2e=None: orig(xe, act, w1e, w2e, b1e, None)
+
+
+def m_bias_in_weights(O):
+    orig = O.selection_scores
+    O.selection_scores = lambda logits, gate, e_bias=None: (
+        orig(logits, gate, e_bias)[0], orig(logits, gate, e_bias)[0])
+
+
+def m_tie_to_higher_index(O):
+    def topk(sel, k):
+        sel = np.asarray(sel, np.float64)
+        M = sel.shape[1]
+        rev = np.argsort(-sel[:, ::-1], axis=1, kind="stable")
+        return (M - 1 - rev)[:, :k].astype(np.int64)
+    O.topk_select = topk
+
+
+def m_no_renorm(O):
+    orig = O.topk_weights
+    O.topk_weights = lambda idx, l, g, gate, norm, a, eps: orig(idx, l, g, gate, 0, a, eps)
+
+
+def m_no_alpha(O):
+    orig = O.topk_weights
+    O.topk_weights = lambda idx, l, g, gate, norm, a, eps: orig(idx, l, g, gate, norm, 1.0, eps)
+
+
+def m_token_major_dispatch(O):
+    def permute(idx, w, M):
+        idx = np.asarray(idx, np.int64)
+        T, k = idx.shape
+        order = np.argsort(idx.reshape(-1), kind="stable")  # (t, j) order: wrong
+        slot = np.empty(T * k, np.int64)
+        slot[order] = np.arange(T * k)
+        counts = np.bincount(idx.reshape(-1), minlength=M)
+        return {"counts": counts, "offsets": np.concatenate([[0], np.cumsum(counts)]),
+                "slot_of": slot.reshape(T, k), "row_token": order // k,
+                "row_w": np.asarray(w, np.float64).reshape(-1)[order]}
+    O.permute = permute
+
+
+def m_gelu_erf(O):
+    from math import erf
+    O.gelu_tanh = lambda v: np.vectorize(lambda a: 0.5 * a * (1 + erf(a / np.sqrt(2))))(np.asarray(v, np.float64))
+
+
+def m_shared_missing(O):
+    O.shared_expert = lambda x, a, b: np.zeros((np.asarray(x).shape[0], np.asarray(b).shape[0]))
+
+
+def m_transposed_router(O):
+    O.router_logits = lambda x, w_r: np.asarray(x, np.float64) @ np.asarray(w_r, np.float64)[::-1, :]
+
+
+def m_wrong_param_count(O):
+    orig = O.param_count
+    O.param_count = lambda D, M, I, act, I_sh=0, **kw: orig(D, M, I, act, I_sh=I_sh, **kw) - (2 * D * I_sh)
+
+
+MUTANTS = [m_swap_gate_up, m_drop_b2, m_bias_in_weights, m_tie_to_higher_index,
+           m_no_renorm, m_no_alpha, m_token_major_dispatch, m_gelu_erf,
+           m_shared_missing, m_transposed_router, m_wrong_param_count]
+
+
+@pytest.mark.parametrize("mutant", MUTANTS, ids=lambda f: f.__name__)
+def test_mutant_is_caught(mutant):
+    O = fresh_oracle()
+    assert caught(O) is None, "unpatched oracle must pass every pin"
+    mutant(O)
+    assert caught(O) is not None, f"no pin caught {mutant.__name__}"

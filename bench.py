@@ -1,0 +1,495 @@
+#!/usr/bin/env python
+"""Benchmark of the sparse MoE FFN layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one moe_forward call (router, dispatch, routed experts, shared
+expert, combine) over one batch of T synthetic tokens already resident in
+HBM.  With N > 1 (torchrun, one process per GPU) every rank runs its own
+batch of T tokens against replicated weights: the layer has no data-path
+exchange, so there is no collective besides the timing reduction (weak
+scaling).  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (fp64 NumPy) on the host cores on
+bounded samples of the same workload; it is the slow reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import moe_synth as ms  # noqa: E402
+
+METRIC = "MoE-layer fwd tokens/s at 1 B200; % of bf16 tensor peak or HBM roofline"
+DEFAULT_CONFIG = "glam_prefill_bf16"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Files whose content defines the GEMM kernel measured by the recorded ncu
+# counters (a change voids the recorded traffic figure).
+GEMM_SOURCES = ["sparse_mixture_experts_logits_b200/csrc/gemm_sm100.cuh",
+                "sparse_mixture_experts_logits_b200/csrc/gemm_sm100.cu",
+                "sparse_mixture_experts_logits_b200/csrc/common.cuh"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU-baseline run time")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing
+# --------------------------------------------------------------------------
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def dist_init(world, local_rank, backend="nccl"):
+    if world <= 1:
+        return None
+    import torch.distributed as dist
+    if backend == "nccl":
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    else:
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return dist
+
+
+def token_rows(rank: int, T: int) -> tuple[int, int]:
+    """Rows of the global synthetic token stream that rank `rank` processes."""
+    return rank * T, (rank + 1) * T
+
+
+def max_over_ranks(dist, value: float, device) -> float:
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------
+# measurement helpers
+# --------------------------------------------------------------------------
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(parts)
+            except ValueError:
+                pass
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        power = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(power) if power else None}
+
+
+def source_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_stage: str, workload: str, units_scale: float = 1.0):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, or None when absent or taken on a different kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    e = rec.get(workload, {}).get(kernel_stage)
+    if not e or e.get("source_hash") != source_hash(GEMM_SOURCES):
+        return None
+    return e["dram_bytes_per_launch"] * units_scale
+
+
+def stage_work(cfg, counts):
+    """Algorithmic FLOPs and bytes of each stage (active experts only;
+    intermediates and padding rows are not credited)."""
+    T, D, M, k, I = cfg["T"], cfg["D"], cfg["M"], cfg["k"], cfg["I"]
+    es = 2 if cfg["dtype"] == "bf16" else 4
+    swiglu = cfg["act"] == "swiglu"
+    n1 = 2 * I if swiglu else I
+    touched = int((counts > 0).sum())
+    pairs = T * k
+    bias = (not swiglu) and cfg.get("has_bias")
+    Ish = cfg.get("I_sh") or 0
+    w = {
+        "route": (2.0 * T * D * M, (T * D + D * M) * es + T * k * 8),
+        "dispatch": (0.0, T * k * 4 * 5),
+        "gather": (0.0, 2.0 * pairs * D * es),
+        "expert_up": (2.0 * pairs * D * n1, touched * (n1 * D + (I if bias else 0)) * es),
+        "expert_down": (2.0 * pairs * I * D, touched * (D * I + (D if bias else 0)) * es),
+        "shared_up": (2.0 * T * D * 2 * Ish, 2.0 * Ish * D * es),
+        "combine": (2.0 * T * Ish * D, (D * Ish * es if Ish else 0) + 2.0 * T * D * es),
+    }
+    return w
+
+
+# --------------------------------------------------------------------------
+# the GPU arm
+# --------------------------------------------------------------------------
+
+def run_ours(args):
+    import sparse_mixture_experts_logits_b200 as B
+
+    rank, local_rank, world = dist_env()
+    if world != args.gpus and world > 1:
+        print(f"warning: WORLD_SIZE={world} but --gpus {args.gpus}", file=sys.stderr)
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = dist_init(world, local_rank)
+
+    cfg = ms.get_config(args.config)
+    T, D = cfg["T"], cfg["D"]
+    inp = ms.layer_inputs(dict(cfg, T=1), dev)  # weights; x below
+    r0, r1 = token_rows(rank, T)
+    x = ms.normal_rows(torch.arange(r0, r1, device=dev), D, 1.0, ms._key(cfg, "x"),
+                       ms.act_dtype(cfg))
+    inp["x"] = x
+    layer = B.MoELayer(cfg, inp)
+    y = torch.empty_like(x)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def fwd():
+        B.moe_forward(layer.desc, layer.weights, x.data_ptr(), y.data_ptr(), layer.ws_ptr,
+                      layer.ws_bytes, sh)
+
+    for _ in range(max(3, args.warmup)):
+        fwd()
+    torch.cuda.synchronize()
+    if layer.device_status() != 0:
+        raise RuntimeError("device status flag set during warm-up")
+    counts = layer.view("counts").cpu().numpy()
+
+    K = args.steps
+    n_ev = B.NUM_STAGE_EVENTS
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(K)]
+    for evs in [starts, ends] + stage_ev:  # torch creates the CUDA event on first record
+        for e in evs:
+            e.record(stream)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    for i in range(K):
+        flush.zero_()  # L2 flush between steps, outside the timed events
+        starts[i].record(stream)
+        B.moe_forward_profiled(layer.desc, layer.weights, x.data_ptr(), y.data_ptr(), layer.ws_ptr,
+                               layer.ws_bytes, sh, [e.cuda_event for e in stage_ev[i]])
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    if dist is not None:
+        dist.barrier()
+    step_ms = [starts[i].elapsed_time(ends[i]) for i in range(K)]
+    ms_local = sum(step_ms) / K
+    stage_ms = {}
+    for s, name in enumerate(B.STAGE_NAMES):
+        stage_ms[name] = sum(stage_ev[i][s].elapsed_time(stage_ev[i][s + 1]) for i in range(K)) / K
+    ms_step = max_over_ranks(dist, ms_local, dev)
+    if layer.device_status() != 0:
+        raise RuntimeError("device status flag set during the timed steps")
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        x_host = x.cpu().pin_memory()
+        y_host = torch.empty_like(x_host).pin_memory()
+        x_dev = torch.empty_like(x)
+        e_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        e_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        for _ in range(2):
+            x_dev.copy_(x_host, non_blocking=True)
+            B.moe_forward(layer.desc, layer.weights, x_dev.data_ptr(), y.data_ptr(), layer.ws_ptr,
+                          layer.ws_bytes, sh)
+            y_host.copy_(y, non_blocking=True)
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for i in range(K):
+            flush.zero_()
+            e_s[i].record(stream)
+            x_dev.copy_(x_host, non_blocking=True)
+            B.moe_forward(layer.desc, layer.weights, x_dev.data_ptr(), y.data_ptr(), layer.ws_ptr,
+                          layer.ws_bytes, sh)
+            y_host.copy_(y, non_blocking=True)
+            e_e[i].record(stream)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        e2e_ms = max_over_ranks(dist, sum(e_s[i].elapsed_time(e_e[i]) for i in range(K)) / K, dev)
+        nbytes = x.numel() * x.element_size()
+        e2e = {"value": world * T / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes}
+
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+
+    peaks, peak_src = load_peaks()
+    work = stage_work(cfg, counts)
+    flops_total, bytes_total = B.moe_algorithmic_work(layer.desc, counts)
+    gemm_stages = [s for s in ("expert_up", "expert_down", "shared_up", "combine") if stage_ms[s] > 0.002]
+    dom = max(gemm_stages, key=lambda s: stage_ms[s])
+    f, b = work[dom]
+    t_s = stage_ms[dom] / 1e3
+    peak_tf = peaks["bf16_tflops"]
+    peak_bw = peaks["hbm_gbs"]
+    t_f, t_b = f / (peak_tf * 1e12), b / (peak_bw * 1e9)
+    if t_f >= t_b:
+        roof = {"bound": "tensor", "achieved": f / t_s / 1e12, "peak": peak_tf, "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": b / t_s / 1e9, "peak": peak_bw, "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = recorded_traffic(dom, args.config)
+    roof["kernel"] = f"moe_gemm_sm100_kernel ({dom})"
+    roof["peak_source"] = f"{peak_src} ({'burst' if peak_src == 'measured' else 'fallback'} figure)"
+    roof["algorithmic"] = {"flops": f, "bytes": b}
+    t_layer_ideal = max(flops_total / (peak_tf * 1e12), bytes_total / (peak_bw * 1e9))
+
+    out = {
+        "metric": METRIC,
+        "value": world * T / (ms_step / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": cfg["dtype"],
+        "data": "synthetic (seeded counter-based generator; random-init weights)",
+        "config": {"workload": args.config, "T_per_gpu": T, "D": D, "M": cfg["M"], "k": cfg["k"],
+                   "I": cfg["I"], "I_sh": cfg.get("I_sh", 0), "gate": cfg["gate"], "act": cfg["act"],
+                   "l2": "flushed between steps (256 MiB write outside the timed events)",
+                   "parallelism": f"replicas x{world} (token batches, no data-path collective)"},
+        "roofline": roof,
+        "layer": {"tflops": flops_total / (ms_step / 1e3) / 1e12,
+                  "algorithmic_flops": flops_total, "algorithmic_bytes": bytes_total,
+                  "ideal_ms": t_layer_ideal * 1e3, "frac_of_ideal": t_layer_ideal / (ms_step / 1e3)},
+        "stages_ms": stage_ms,
+        "e2e": e2e,
+        "gpu_launches": B.moe_forward_launch_count(layer.desc) * K,
+        "clocks": clocks,
+        "routing": {"touched_experts": int((counts > 0).sum()), "max_over_mean":
+                    float(counts.max() / max(1e-9, counts.mean()))},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(cfg, inp, args.cpu_seconds)
+    print(json.dumps(out), flush=True)
+    del layer
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------
+# the oracle on the host cores
+# --------------------------------------------------------------------------
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = [i for i in threadpool_info() if i.get("user_api") == "blas"]
+        if info:
+            return int(max(i.get("num_threads", 1) for i in info)), info[0].get("internal_api", "blas")
+    except Exception:
+        pass
+    return os.cpu_count() or 1, "unknown"
+
+
+class OracleRunner:
+    """Runs the CPU oracle on token blocks of one workload.  Weights live on
+    the host as bf16 and are widened to fp64 per expert when used, as the
+    oracle does at full size."""
+
+    def __init__(self, cfg, inp):
+        import oracle
+        self.oracle = oracle
+        self.cfg = cfg
+        self.x = inp["x"]
+        host = {k: (None if v is None else v.cpu()) for k, v in inp.items() if k != "x"}
+        self.w_r = host["w_r"].double().numpy()
+        self.e_bias = None if host["e_bias"] is None else host["e_bias"].double().numpy()
+        self.host = host
+        self.shared = None
+        if cfg.get("I_sh"):
+            self.shared = (host["sh_w1"].double().numpy(), host["sh_w2"].double().numpy())
+
+    def get_expert(self, e):
+        h = self.host
+        return (h["w1"][e].double().numpy(), h["w2"][e].double().numpy(),
+                None if h["b1"] is None else h["b1"][e].double().numpy(),
+                None if h["b2"] is None else h["b2"][e].double().numpy())
+
+    def x_block(self, t0, n):
+        T = self.x.shape[0]
+        rows = torch.arange(t0, t0 + n) % T
+        return self.x[rows.to(self.x.device)].double().cpu().numpy()
+
+    def run(self, xs):
+        c = self.cfg
+        r = self.oracle.route(xs, self.w_r, self.e_bias, c["k"], c["gate"], c["norm_topk_prob"],
+                              c["alpha"], c["eps"])
+        return self.oracle.moe_tokens(xs, r["idx"], r["w"], c["act"], self.get_expert, self.shared)
+
+
+def cpu_baseline(cfg, inp, target_s):
+    runner = OracleRunner(cfg, inp)
+    n = 16
+    while True:
+        xs = runner.x_block(0, n)
+        t0 = time.perf_counter()
+        runner.run(xs)
+        dt = time.perf_counter() - t0
+        if dt >= target_s * 0.5 or n >= cfg["T"]:
+            break
+        n = int(min(cfg["T"], max(2 * n, n * target_s / max(dt, 1e-3))))
+    cores, api = _blas_threads()
+    return {"value": n / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {n} of the workload's {cfg['T']} tokens through the fp64 NumPy oracle "
+                      f"({api} BLAS); weights widened from bf16 per expert inside the timed run",
+            "seconds": dt}
+
+
+def run_reference(args):
+    rank, local_rank, world = dist_env()
+    if rank != 0:
+        return
+    cfg = ms.get_config(args.config)
+    dev = torch.device("cuda", local_rank) if torch.cuda.is_available() else torch.device("cpu")
+    inp = ms.layer_inputs(cfg, dev)
+    runner = OracleRunner(cfg, inp)
+    # size one step's token sample from a probe so that the whole run stays short
+    probe_n = 8
+    t0 = time.perf_counter()
+    runner.run(runner.x_block(0, probe_n))
+    per_step_budget = max(0.5, 150.0 / max(1, args.steps + args.warmup))
+    dt = time.perf_counter() - t0
+    n = int(max(4, min(cfg["T"], probe_n * per_step_budget / max(dt, 1e-3))))
+    cursor = 0
+    for _ in range(args.warmup):
+        runner.run(runner.x_block(cursor, n))
+        cursor += n
+    times = []
+    for _ in range(args.steps):
+        xs = runner.x_block(cursor, n)
+        cursor += n
+        t0 = time.perf_counter()
+        runner.run(xs)
+        times.append(time.perf_counter() - t0)
+    mean_s = sum(times) / len(times)
+    value = n / mean_s
+    cores, api = _blas_threads()
+    sample = (f"{n} consecutive tokens per step of the {cfg['T']}-token workload, fp64 NumPy oracle "
+              f"({api} BLAS)")
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_s * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded counter-based generator; random-init weights)",
+        "config": {"workload": args.config, "T_per_gpu": cfg["T"], "D": cfg["D"], "M": cfg["M"],
+                   "k": cfg["k"], "I": cfg["I"], "I_sh": cfg.get("I_sh", 0)},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

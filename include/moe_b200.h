@@ -1,0 +1,244 @@
+/*
+ * moe_b200.h - C ABI of the sparse Mixture-of-Experts FFN layer forward on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (sources: the "GLaM" architecture note, section "Sparse MoE
+ * Layer"; the GLM-4.5 "Shared Expert" study note, section "How it works";
+ * the "GLM-5 - Shared expert" page of OpenModelAtlas, its quoted
+ * GlmMoeDsaMoE / GlmMoeDsaExperts / GlmMoeDsaMLP forward excerpts):
+ *
+ *   route     s[t,e] = sum_d x[t,d] W_r[d,e]                     (fp32)
+ *             softmax gate: S_t = TopK(s_t, k); w = renormalised softmax
+ *             sigmoid gate: g = sigmoid(s); S_t = TopK(g + e_bias, k);
+ *                           w = alpha * g / (sum_S g + eps)
+ *   dispatch  pairs (t, j) grouped by expert, inside an expert by (j, t)
+ *   experts   GELU:   E(x) = W2 GELU_tanh(W1 x + b1) + b2
+ *             SwiGLU: E(x) = W_down(SiLU(W_gate x) * W_up x)
+ *   combine   y_t = sum_j w[t,j] E_{idx[t,j]}(x_t)  (+ E_sh(x_t))
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensors are dense row-major.  Weights use the nn.Linear [out, in]
+ *    layout, except W_r, which is [D, M].
+ *  - Every pointer argument is a DEVICE pointer to caller-owned memory on
+ *    the current device, except the descriptor and weight structs, which are
+ *    host structs (the pointers inside them are device pointers).  The
+ *    library never allocates, frees or synchronises; every call only
+ *    enqueues kernels on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and returns.
+ *  - Scratch memory ("workspace") is caller-provided; each entry point has a
+ *    *_workspace_size query.  Workspaces must be 256-byte aligned.  Calls
+ *    that share a workspace must be ordered on one stream.
+ *  - dtype MOE_DTYPE_BF16: x, W_r, expert/shared weights, biases, y are
+ *    bf16; all accumulation is fp32.  MOE_DTYPE_F32: all of them are fp32.
+ *    e_bias, topk_w and row_w are always fp32; indices are int32.
+ *  - Errors: every call validates its arguments on the host and returns a
+ *    status without launching anything when they are invalid.  Device-side
+ *    faults are never raised: kernels that find an out-of-range expert index
+ *    or whose bounded waits time out set a flag in the workspace, read back
+ *    with moe_device_status().
+ *  - T = 0 is valid and launches nothing.
+ */
+#ifndef MOE_B200_H_
+#define MOE_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null pointer, bad size, k > M, workspace too small */
+  MOE_ERR_UNSUPPORTED = 2, /* shape/dtype outside what the kernels implement */
+  MOE_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+  MOE_ERR_DEVICE = 4       /* a kernel reported an error through the workspace flag */
+} moe_status_t;
+
+typedef enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 } moe_dtype_t;
+
+/* Router kinds.  SOFTMAX: "GLaM" eq. r_t and S_t.  SIGMOID_BIAS: the GLM-4.5
+ * note's sigmoid scores plus loss-free correction bias. */
+typedef enum { MOE_GATE_SOFTMAX = 0, MOE_GATE_SIGMOID_BIAS = 1 } moe_gate_t;
+
+/* Expert kinds.  GELU_TANH: "GLaM" eq. FFN with sigma = GELU (tanh form).
+ * SWIGLU: W_down(SiLU(W_gate x) * W_up x). */
+typedef enum { MOE_ACT_GELU_TANH = 0, MOE_ACT_SWIGLU = 1 } moe_act_t;
+
+/* Device-side error codes written to the workspace flag. */
+#define MOE_DEVERR_NONE 0
+#define MOE_DEVERR_BAD_EXPERT_INDEX 1 /* topk_idx entry outside [0, M) */
+#define MOE_DEVERR_TIMEOUT 2          /* a bounded wait inside a kernel gave up */
+
+/* One MoE layer's shape and options (HF config names in brackets). */
+typedef struct {
+  int dtype;                   /* moe_dtype_t */
+  int T;                       /* tokens (batch x sequence flattened) */
+  int D;                       /* model width [hidden_size] */
+  int M;                       /* routed experts [n_routed_experts] */
+  int k;                       /* experts per token [num_experts_per_tok] */
+  int gate;                    /* moe_gate_t */
+  int act;                     /* moe_act_t */
+  int I;                       /* expert hidden width [moe_intermediate_size] */
+  int has_bias;                /* GELU experts: b1, b2 present */
+  int norm_topk_prob;          /* renormalise the k selected gate values */
+  float routed_scaling_factor; /* alpha, multiplies every routed weight */
+  float eps;                   /* sigmoid renormalisation epsilon (1e-20) */
+  int I_sh;                    /* shared expert width, 0 = no shared expert
+                                  [moe_intermediate_size * n_shared_experts] */
+} moe_layer_desc_t;
+
+/* Device pointers to one layer's weights.  Unused fields may be NULL. */
+typedef struct {
+  const void* w_r;     /* [D, M] router weight */
+  const float* e_bias; /* [M] correction bias (SIGMOID_BIAS; NULL = zeros) */
+  const void* w1;      /* GELU: [M, I, D] W1.  SWIGLU: [M, 2I, D] fused
+                          gate_up stack, rows 0..I-1 gate, I..2I-1 up */
+  const void* b1;      /* GELU with bias: [M, I] */
+  const void* w2;      /* [M, D, I] W2 / down projection */
+  const void* b2;      /* GELU with bias: [M, D] */
+  const void* sh_w1;   /* [2 I_sh, D] shared gate_up (gate rows first) */
+  const void* sh_w2;   /* [D, I_sh] shared down projection */
+} moe_weights_t;
+
+/* Byte offsets, inside a moe_forward workspace, of the intermediates the
+ * forward pass leaves there (valid after the stream reaches the end of a
+ * moe_forward call).  Exposed so that tests can check every stage. */
+typedef struct {
+  size_t status;    /* int32 device status flag */
+  size_t topk_idx;  /* int32 [T, k] */
+  size_t topk_w;    /* fp32  [T, k] */
+  size_t counts;    /* int32 [M] */
+  size_t offsets;   /* int32 [M + 1] */
+  size_t slot_of;   /* int32 [T, k] */
+  size_t row_token; /* int32 [T k] */
+  size_t row_w;     /* fp32  [T k] */
+  size_t out_perm;  /* fp32  [T k, D] weighted expert outputs, dispatch order */
+  size_t total;     /* bytes needed */
+} moe_ws_layout_t;
+
+/* ------------------------------------------------------------------------ */
+
+/* Status string ("MOE_OK", ...); never NULL. */
+const char* moe_status_string(moe_status_t s);
+
+/* Library version string. */
+const char* moe_version(void);
+
+/* Reads the device status flag at the start of workspace `ws` (any entry
+ * point's workspace) into *out (MOE_DEVERR_*) and clears it.  This call
+ * synchronises `stream`.  Returns MOE_ERR_CUDA if the copy fails. */
+moe_status_t moe_device_status(void* ws, void* stream, int* out);
+
+/* ---- router: "GLaM" eq. r_t, S_t and MoE; GLM-4.5 note eq. g-bar ------- */
+
+size_t moe_route_workspace_size(int T, int D, int M, int dtype);
+
+/* Router scores, top-k and gate weights for T tokens.
+ *   x [T, D], w_r [D, M] (dtype), e_bias [M] fp32 or NULL.
+ *   Outputs topk_idx [T, k] int32 (slot j = j-th largest selection score,
+ *   exact ties to the lower expert index) and topk_w [T, k] fp32.
+ *   SOFTMAX: selection on the logits; w = alpha * softmax renormalised over
+ *   the k selected (norm_topk_prob) or the full softmax probability.
+ *   SIGMOID_BIAS: selection on sigmoid(s) + e_bias; w = alpha * g /
+ *   (sum_S g + eps) (norm_topk_prob) or alpha * g; the bias never enters w.
+ * Limits: 1 <= k <= min(M, 32), M <= 1024; bf16 needs D % 16 == 0. */
+moe_status_t moe_route_topk(const void* x, const void* w_r, const float* e_bias,
+                            int T, int D, int M, int k, int dtype, int gate,
+                            int norm_topk_prob, float routed_scaling_factor, float eps,
+                            int32_t* topk_idx, float* topk_w,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* ---- dispatch: the GLM-5 page's GlmMoeDsaExperts.forward expert mask --- */
+
+size_t moe_permute_workspace_size(int T, int k, int M);
+
+/* Deterministic dispatch order of the T*k (token, slot) pairs: a stable
+ * counting sort by expert of the pairs taken in (slot j, token t) order.
+ *   counts[M], offsets[M+1] (exclusive prefix sum, offsets[M] = T k),
+ *   slot_of[T, k] (dispatch position of pair (t, j)), row_token[T k],
+ *   row_w[T k] = topk_w[t, j] of the pair at each position.
+ * Bit-exact and independent of scheduling (no atomics decide an order).
+ * An out-of-range entry of topk_idx sets MOE_DEVERR_BAD_EXPERT_INDEX and
+ * is skipped (its outputs are then unspecified). */
+moe_status_t moe_permute(const int32_t* topk_idx, const float* topk_w, int T, int k, int M,
+                         int32_t* counts, int32_t* offsets, int32_t* slot_of,
+                         int32_t* row_token, float* row_w,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* ---- experts: "GLaM" eq. FFN; GLM-5 GlmMoeDsaExperts.forward ----------- */
+
+size_t moe_expert_ffn_workspace_size(const moe_layer_desc_t* d);
+
+/* Routed experts over the dispatch order:
+ *   out_perm[s, :] = row_w[s] * E_e(x[row_token[s], :]) for every position s
+ *   in expert e's segment [offsets[e], offsets[e+1]).
+ * out_perm is fp32 [T k, D] (the accumulator, unrounded, so that the
+ * combine rounds only once). */
+moe_status_t moe_expert_ffn(const moe_layer_desc_t* d, const moe_weights_t* w,
+                            const void* x, const int32_t* offsets,
+                            const int32_t* row_token, const float* row_w,
+                            void* out_perm, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- shared expert: GLM-4.5 note E_sh; GLM-5 GlmMoeDsaMLP.forward ------ */
+
+size_t moe_shared_expert_workspace_size(const moe_layer_desc_t* d);
+
+/* y_sh[T, D] = W_down(SiLU(W_gate x) * W_up x) over the pre-routing x. */
+moe_status_t moe_shared_expert(const moe_layer_desc_t* d, const moe_weights_t* w,
+                               const void* x, void* y_sh,
+                               void* ws, size_t ws_bytes, void* stream);
+
+/* ---- combine: "GLaM" eq. MoE; GLM-4.5 note eq. y ----------------------- */
+
+/* y[t, :] = sum_{j=0}^{k-1} out_perm[slot_of[t, j], :] (+ shared_out[t, :]),
+ * out_perm fp32 [T k, D], shared_out and y [T, D] in dtype,
+ * summed in fp32 in slot order and rounded once.  shared_out may be NULL. */
+moe_status_t moe_combine(const moe_layer_desc_t* d, const void* out_perm,
+                         const int32_t* slot_of, const void* shared_out, void* y,
+                         void* stream);
+
+/* ---- the whole layer --------------------------------------------------- */
+
+size_t moe_workspace_size(const moe_layer_desc_t* d);
+moe_status_t moe_workspace_layout(const moe_layer_desc_t* d, moe_ws_layout_t* out);
+
+/* y[T, D] = MoE-FFN(x): route, dispatch, routed experts, and the combine
+ * fused with the shared expert's down projection (when I_sh > 0).  All
+ * stages run back to back on `stream` with no host synchronisation. */
+moe_status_t moe_forward(const moe_layer_desc_t* d, const moe_weights_t* w,
+                         const void* x, void* y, void* ws, size_t ws_bytes, void* stream);
+
+/* Stage boundaries recorded by moe_forward_profiled (the "routing overhead"
+ * breakdown of the GLaM note's reporting table: gate, dispatch, expert
+ * batching, combination cost). */
+#define MOE_NUM_STAGE_EVENTS 8
+/* event 0: start; 1: route done (scores, top-k, weights); 2: dispatch order
+ * done; 3: rows gathered into dispatch order; 4: routed experts' first GEMM
+ * done; 5: routed experts' second GEMM done; 6: shared expert's first GEMM
+ * done; 7: combine (fused with the shared down projection) done.  Stages a
+ * layer does not have record their event right after the previous one. */
+
+/* moe_forward, recording `events[i]` (cudaEvent_t handles created by the
+ * caller, n_events == MOE_NUM_STAGE_EVENTS) on `stream` at each boundary. */
+moe_status_t moe_forward_profiled(const moe_layer_desc_t* d, const moe_weights_t* w,
+                                  const void* x, void* y, void* ws, size_t ws_bytes, void* stream,
+                                  void* const* events, int n_events);
+
+/* Number of kernels one moe_forward call with this descriptor launches. */
+int moe_forward_launch_count(const moe_layer_desc_t* d);
+
+/* Algorithmic work of one moe_forward call given the routing counts
+ * (host array counts[M], as produced by moe_permute): FLOPs of the router
+ * and of the routed and shared experts, and bytes of the weights of the
+ * experts that received at least one token plus x and y.  Padding and
+ * intermediate buffers are not counted. */
+void moe_algorithmic_work(const moe_layer_desc_t* d, const int32_t* counts_host,
+                          double* flops, double* bytes);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H_ */

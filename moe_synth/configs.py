@@ -91,6 +91,8 @@ def get_config(name: str, **overrides) -> dict:
     cfg["name"] = name
     cfg.setdefault("seed", 0)
     cfg.update(overrides)
+    # one of the five named workloads, unchanged
+    cfg["named"] = name in CONFIGS and not overrides
     return cfg
 
 

@@ -1,0 +1,74 @@
+// Host-side launchers of the library's kernels (internal interface between
+// the C ABI in moe_api.cu and the kernel files).
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// router.cu
+cudaError_t launch_transpose_bf16(const void* src, void* dst, int rows, int cols, cudaStream_t s);
+cudaError_t launch_logits_f32(const float* x, const float* w_r, float* logits, int T, int D, int M,
+                              cudaStream_t s);
+cudaError_t launch_topk(const float* logits, const float* e_bias, int T, int M, int k, int gate,
+                        int norm, float alpha, float eps, int32_t* idx, float* w, cudaStream_t s);
+
+// permute.cu
+constexpr int kPermChunk = 512;  // (slot, token) pairs per chunk of the counting sort
+inline int perm_num_chunks(long long pairs) {
+  return static_cast<int>((pairs + kPermChunk - 1) / kPermChunk);
+}
+cudaError_t launch_permute(const int32_t* topk_idx, const float* topk_w, int T, int k, int M,
+                           int32_t* counts, int32_t* offsets, int32_t* slot_of, int32_t* row_token,
+                           float* row_w, int32_t* chunk_counts, int32_t* chunk_base, int* status,
+                           cudaStream_t s);
+
+// misc.cu
+cudaError_t launch_gather_rows(const void* x, const int32_t* row_token, void* x_perm, int rows,
+                               int D, int elem_bytes, cudaStream_t s);
+cudaError_t launch_combine(int dtype, const void* out_perm, const int32_t* slot_of,
+                           const void* shared_out, void* y, int T, int D, int k, cudaStream_t s);
+
+// gemm_sm100.cu: grouped bf16 GEMM on tcgen05.  `epi` is a GemmEpilogue.
+struct GemmLaunch {
+  int epi;
+  const void* A; long long a_rows; // bf16 [a_rows, K]
+  const void* B; long long b_rows; // bf16 [b_rows, K]
+  int K;
+  int num_groups;
+  const int* offsets;  // device [G+1] or nullptr (single group of a_rows rows)
+  long long rows_upper;  // host upper bound of the rows covered by the segments
+  int bn, n_tiles, b_rows_per_group, b_row_step, b_hi_offset;
+  int out_cols, out_col_step, ldo;
+  void* out;
+  const float* row_scale;
+  const void* bias;
+  const void* comb_src;
+  const int32_t* slot_of;
+  int k;
+  int* status;
+};
+cudaError_t launch_gemm_sm100(const GemmLaunch& L, cudaStream_t s);
+int num_sms();
+
+// simt.cu: fp32 grouped GEMM with the same epilogues (fp32 dtype path).
+struct SimtLaunch {
+  int epi;
+  const float* A; const int32_t* a_row_index; int K; // A row of output row r: a_row_index[r] or r
+  const float* B;                                     // [G * b_rows_per_group, K]
+  int num_groups;
+  const int* offsets;  // device [G+1] or nullptr
+  long long rows;      // rows when offsets == nullptr; upper bound otherwise
+  int b_rows_per_group;
+  int swiglu_hi;       // SwiGLU: row offset of the up half (I); 0 otherwise
+  int out_cols, ldo;
+  float* out;
+  const float* row_scale;
+  const float* bias;
+  const float* comb_src;
+  const int32_t* slot_of;
+  int k;
+};
+cudaError_t launch_simt_gemm(const SimtLaunch& L, cudaStream_t s);
+
+}  // namespace moe

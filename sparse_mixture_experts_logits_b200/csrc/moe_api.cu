@@ -1,0 +1,583 @@
+// C ABI of the MoE layer forward: argument checks, workspace layouts and
+// the sequence of kernel launches of every entry point (see moe_b200.h).
+#include <algorithm>
+#include <atomic>
+#include <cstring>
+
+#include "gemm_sm100.cuh"
+#include "kernels.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
+
+struct Carve {
+  size_t off = 0;
+  size_t take(size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes);
+    return o;
+  }
+};
+
+inline size_t esize(int dtype) { return dtype == MOE_DTYPE_BF16 ? 2 : 4; }
+
+// Every entry point runs only on compute capability 10.0 (sm_100a code).
+moe_status_t check_device() {
+  static std::atomic<int> verdict[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
+  int v = verdict[dev].load();
+  if (v == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    v = (major == 10 && minor == 0) ? 1 : 2;
+    verdict[dev].store(v);
+  }
+  return v == 1 ? MOE_OK : MOE_ERR_UNSUPPORTED;
+}
+
+inline moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+#define MOE_TRY(expr)                          \
+  do {                                         \
+    moe_status_t st_ = (expr);                 \
+    if (st_ != MOE_OK) return st_;             \
+  } while (0)
+#define MOE_CUDA(expr) MOE_TRY(cuda_status(expr))
+
+bool aligned_ws(const void* ws) { return (reinterpret_cast<uintptr_t>(ws) % kAlign) == 0; }
+
+moe_status_t check_router_args(int T, int D, int M, int k, int dtype, int gate) {
+  if (T < 0 || D < 1 || M < 1 || k < 1) return MOE_ERR_INVALID_ARG;
+  if (k > M) return MOE_ERR_INVALID_ARG;
+  if (dtype != MOE_DTYPE_F32 && dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (gate != MOE_GATE_SOFTMAX && gate != MOE_GATE_SIGMOID_BIAS) return MOE_ERR_INVALID_ARG;
+  if (k > kMaxTopK || M > kMaxExperts) return MOE_ERR_UNSUPPORTED;
+  if (dtype == MOE_DTYPE_BF16 && D % 16 != 0) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(T) * std::max(D, M) >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status_t check_desc(const moe_layer_desc_t* d) {
+  if (d == nullptr) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_router_args(d->T, d->D, d->M, d->k, d->dtype, d->gate));
+  if (d->act != MOE_ACT_GELU_TANH && d->act != MOE_ACT_SWIGLU) return MOE_ERR_INVALID_ARG;
+  if (d->I < 1 || d->I_sh < 0 || !(d->eps >= 0.0f)) return MOE_ERR_INVALID_ARG;
+  if (d->dtype == MOE_DTYPE_BF16 && (d->I % 16 != 0 || d->I_sh % 16 != 0)) return MOE_ERR_UNSUPPORTED;
+  const long long pairs = static_cast<long long>(d->T) * d->k;
+  const long long wide = std::max<long long>({d->D, 2ll * d->I, 2ll * d->I_sh});
+  if (pairs * wide >= (1ll << 40) || pairs >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(d->M) * 2 * d->I * std::max(d->D, d->I) >= (1ll << 40))
+    return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status_t check_weights(const moe_layer_desc_t* d, const moe_weights_t* w, bool routed, bool shared) {
+  if (w == nullptr) return MOE_ERR_INVALID_ARG;
+  if (routed) {
+    if (w->w1 == nullptr || w->w2 == nullptr) return MOE_ERR_INVALID_ARG;
+    if (d->act == MOE_ACT_GELU_TANH && d->has_bias && (w->b1 == nullptr || w->b2 == nullptr))
+      return MOE_ERR_INVALID_ARG;
+  }
+  if (shared && d->I_sh > 0 && (w->sh_w1 == nullptr || w->sh_w2 == nullptr)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------- layouts
+struct RouteWs { size_t status, logits, wrT, total; };
+RouteWs route_layout(int T, int D, int M, int dtype) {
+  Carve c;
+  RouteWs L;
+  L.status = c.take(4);
+  L.logits = c.take(static_cast<size_t>(T) * M * 4);
+  L.wrT = c.take(dtype == MOE_DTYPE_BF16 ? static_cast<size_t>(M) * D * 2 : 0);
+  L.total = c.off;
+  return L;
+}
+
+struct PermWs { size_t status, chunk_counts, chunk_base, total; };
+PermWs perm_layout(int T, int k, int M) {
+  Carve c;
+  PermWs L;
+  const size_t n = static_cast<size_t>(M) * perm_num_chunks(static_cast<long long>(T) * k);
+  L.status = c.take(4);
+  L.chunk_counts = c.take(n * 4);
+  L.chunk_base = c.take(n * 4);
+  L.total = c.off;
+  return L;
+}
+
+struct FfnWs { size_t status, x_perm, h, total; };
+FfnWs ffn_layout(const moe_layer_desc_t* d) {
+  Carve c;
+  FfnWs L;
+  const size_t pairs = static_cast<size_t>(d->T) * d->k;
+  L.status = c.take(4);
+  L.x_perm = c.take(d->dtype == MOE_DTYPE_BF16 ? pairs * d->D * 2 : 0);
+  L.h = c.take(pairs * d->I * esize(d->dtype));
+  L.total = c.off;
+  return L;
+}
+
+struct SharedWs { size_t status, h_sh, total; };
+SharedWs shared_layout(const moe_layer_desc_t* d) {
+  Carve c;
+  SharedWs L;
+  L.status = c.take(4);
+  L.h_sh = c.take(static_cast<size_t>(d->T) * d->I_sh * esize(d->dtype));
+  L.total = c.off;
+  return L;
+}
+
+struct FwdWs {
+  moe_ws_layout_t pub;
+  size_t logits, wrT, chunk_counts, chunk_base, x_perm, h, h_sh;
+};
+FwdWs forward_layout(const moe_layer_desc_t* d) {
+  Carve c;
+  FwdWs L;
+  const size_t pairs = static_cast<size_t>(d->T) * d->k;
+  const size_t es = esize(d->dtype);
+  L.pub.status = c.take(4);
+  L.pub.topk_idx = c.take(pairs * 4);
+  L.pub.topk_w = c.take(pairs * 4);
+  L.pub.counts = c.take(static_cast<size_t>(d->M) * 4);
+  L.pub.offsets = c.take(static_cast<size_t>(d->M + 1) * 4);
+  L.pub.slot_of = c.take(pairs * 4);
+  L.pub.row_token = c.take(pairs * 4);
+  L.pub.row_w = c.take(pairs * 4);
+  L.pub.out_perm = c.take(pairs * d->D * 4);
+  L.logits = c.take(static_cast<size_t>(d->T) * d->M * 4);
+  L.wrT = c.take(d->dtype == MOE_DTYPE_BF16 ? static_cast<size_t>(d->M) * d->D * 2 : 0);
+  const size_t nch = static_cast<size_t>(d->M) * perm_num_chunks(static_cast<long long>(pairs));
+  L.chunk_counts = c.take(nch * 4);
+  L.chunk_base = c.take(nch * 4);
+  L.x_perm = c.take(d->dtype == MOE_DTYPE_BF16 ? pairs * d->D * 2 : 0);
+  L.h = c.take(pairs * d->I * es);
+  L.h_sh = c.take(static_cast<size_t>(d->T) * d->I_sh * es);
+  L.pub.total = c.off;
+  return L;
+}
+
+template <typename P> inline P at(void* ws, size_t off) {
+  return reinterpret_cast<P>(static_cast<char*>(ws) + off);
+}
+
+// ------------------------------------------------------------ the stages
+// Records caller-provided CUDA events at stage boundaries (profiled forward).
+struct Marks {
+  void* const* ev = nullptr;
+  cudaStream_t s = nullptr;
+  moe_status_t at(int i) const {
+    if (ev == nullptr) return MOE_OK;
+    return cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s));
+  }
+};
+
+moe_status_t run_route(const void* x, const void* w_r, const float* e_bias, int T, int D, int M, int k,
+                       int dtype, int gate, int norm, float alpha, float eps, int32_t* idx, float* w,
+                       float* logits, void* wrT, int* status, cudaStream_t s) {
+  if (dtype == MOE_DTYPE_BF16) {
+    MOE_CUDA(launch_transpose_bf16(w_r, wrT, D, M, s));
+    GemmLaunch L{};
+    L.epi = EPI_STORE_F32;
+    L.A = x; L.a_rows = T;
+    L.B = wrT; L.b_rows = M;
+    L.K = D;
+    L.num_groups = 1; L.offsets = nullptr; L.rows_upper = T;
+    L.bn = std::min(256, round_up(M, 16));
+    L.n_tiles = (M + L.bn - 1) / L.bn;
+    L.b_rows_per_group = M; L.b_row_step = L.bn; L.b_hi_offset = L.bn / 2;
+    L.out_cols = M; L.out_col_step = L.bn; L.ldo = M;
+    L.out = logits;
+    L.status = status;
+    MOE_CUDA(launch_gemm_sm100(L, s));
+  } else {
+    MOE_CUDA(launch_logits_f32(static_cast<const float*>(x), static_cast<const float*>(w_r), logits, T,
+                               D, M, s));
+  }
+  MOE_CUDA(launch_topk(logits, gate == MOE_GATE_SIGMOID_BIAS ? e_bias : nullptr, T, M, k, gate, norm,
+                       alpha, eps, idx, w, s));
+  return MOE_OK;
+}
+
+moe_status_t run_experts(const moe_layer_desc_t* d, const moe_weights_t* w, const void* x,
+                         const int32_t* offsets, const int32_t* row_token, const float* row_w,
+                         void* out_perm, void* x_perm, void* h, int* status, cudaStream_t s,
+                         const Marks& mk = Marks()) {
+  const int pairs = d->T * d->k;
+  const bool swiglu = d->act == MOE_ACT_SWIGLU;
+  const int n1 = swiglu ? 2 * d->I : d->I;
+  const void* b1 = (!swiglu && d->has_bias) ? w->b1 : nullptr;
+  const void* b2 = (!swiglu && d->has_bias) ? w->b2 : nullptr;
+  if (d->dtype == MOE_DTYPE_BF16) {
+    MOE_CUDA(launch_gather_rows(x, row_token, x_perm, pairs, d->D, 2, s));
+    MOE_TRY(mk.at(3));
+    GemmLaunch g1{};
+    g1.A = x_perm; g1.a_rows = pairs;
+    g1.B = w->w1; g1.b_rows = static_cast<long long>(d->M) * n1;
+    g1.K = d->D;
+    g1.num_groups = d->M; g1.offsets = offsets; g1.rows_upper = pairs;
+    if (swiglu) {
+      const int half = std::min(128, round_up(d->I, 16));
+      g1.epi = EPI_SWIGLU;
+      g1.bn = 2 * half;
+      g1.n_tiles = (d->I + half - 1) / half;
+      g1.b_rows_per_group = n1; g1.b_row_step = half; g1.b_hi_offset = d->I;
+      g1.out_col_step = half;
+    } else {
+      g1.epi = EPI_GELU_BIAS;
+      g1.bn = std::min(256, round_up(d->I, 16));
+      g1.n_tiles = (d->I + g1.bn - 1) / g1.bn;
+      g1.b_rows_per_group = n1; g1.b_row_step = g1.bn; g1.b_hi_offset = g1.bn / 2;
+      g1.out_col_step = g1.bn;
+      g1.bias = b1;
+    }
+    g1.out_cols = d->I; g1.ldo = d->I; g1.out = h;
+    g1.status = status;
+    MOE_CUDA(launch_gemm_sm100(g1, s));
+    MOE_TRY(mk.at(4));
+
+    GemmLaunch g2{};
+    g2.epi = EPI_SCALE_BIAS;
+    g2.A = h; g2.a_rows = pairs;
+    g2.B = w->w2; g2.b_rows = static_cast<long long>(d->M) * d->D;
+    g2.K = d->I;
+    g2.num_groups = d->M; g2.offsets = offsets; g2.rows_upper = pairs;
+    g2.bn = std::min(256, round_up(d->D, 16));
+    g2.n_tiles = (d->D + g2.bn - 1) / g2.bn;
+    g2.b_rows_per_group = d->D; g2.b_row_step = g2.bn; g2.b_hi_offset = g2.bn / 2;
+    g2.out_cols = d->D; g2.out_col_step = g2.bn; g2.ldo = d->D;
+    g2.out = out_perm; g2.row_scale = row_w; g2.bias = b2;
+    g2.status = status;
+    MOE_CUDA(launch_gemm_sm100(g2, s));
+    MOE_TRY(mk.at(5));
+  } else {
+    MOE_TRY(mk.at(3));
+    SimtLaunch g1{};
+    g1.epi = swiglu ? EPI_SWIGLU : EPI_GELU_BIAS;
+    g1.A = static_cast<const float*>(x); g1.a_row_index = row_token; g1.K = d->D;
+    g1.B = static_cast<const float*>(w->w1);
+    g1.num_groups = d->M; g1.offsets = offsets; g1.rows = pairs;
+    g1.b_rows_per_group = n1; g1.swiglu_hi = swiglu ? d->I : 0;
+    g1.out_cols = d->I; g1.ldo = d->I; g1.out = static_cast<float*>(h);
+    g1.bias = static_cast<const float*>(b1);
+    MOE_CUDA(launch_simt_gemm(g1, s));
+    MOE_TRY(mk.at(4));
+    SimtLaunch g2{};
+    g2.epi = EPI_SCALE_BIAS;
+    g2.A = static_cast<const float*>(h); g2.a_row_index = nullptr; g2.K = d->I;
+    g2.B = static_cast<const float*>(w->w2);
+    g2.num_groups = d->M; g2.offsets = offsets; g2.rows = pairs;
+    g2.b_rows_per_group = d->D;
+    g2.out_cols = d->D; g2.ldo = d->D; g2.out = static_cast<float*>(out_perm);
+    g2.row_scale = row_w; g2.bias = static_cast<const float*>(b2);
+    MOE_CUDA(launch_simt_gemm(g2, s));
+    MOE_TRY(mk.at(5));
+  }
+  return MOE_OK;
+}
+
+// Shared SwiGLU on all T tokens.  The down projection's epilogue adds
+// sum_j comb_src[slot_of[t, j]] (k_comb slots; 0 = none) to the accumulator.
+moe_status_t run_shared(const moe_layer_desc_t* d, const moe_weights_t* w, const void* x, void* out,
+                        void* h_sh, const void* comb_src, const int32_t* slot_of, int k_comb,
+                        int* status, cudaStream_t s, const Marks& mk = Marks()) {
+  if (d->dtype == MOE_DTYPE_BF16) {
+    const int half = std::min(128, round_up(d->I_sh, 16));
+    GemmLaunch g1{};
+    g1.epi = EPI_SWIGLU;
+    g1.A = x; g1.a_rows = d->T;
+    g1.B = w->sh_w1; g1.b_rows = 2ll * d->I_sh;
+    g1.K = d->D;
+    g1.num_groups = 1; g1.offsets = nullptr; g1.rows_upper = d->T;
+    g1.bn = 2 * half; g1.n_tiles = (d->I_sh + half - 1) / half;
+    g1.b_rows_per_group = 2 * d->I_sh; g1.b_row_step = half; g1.b_hi_offset = d->I_sh;
+    g1.out_cols = d->I_sh; g1.out_col_step = half; g1.ldo = d->I_sh; g1.out = h_sh;
+    g1.status = status;
+    MOE_CUDA(launch_gemm_sm100(g1, s));
+    MOE_TRY(mk.at(6));
+    GemmLaunch g2{};
+    g2.epi = EPI_COMBINE;
+    g2.A = h_sh; g2.a_rows = d->T;
+    g2.B = w->sh_w2; g2.b_rows = d->D;
+    g2.K = d->I_sh;
+    g2.num_groups = 1; g2.offsets = nullptr; g2.rows_upper = d->T;
+    g2.bn = std::min(256, round_up(d->D, 16)); g2.n_tiles = (d->D + g2.bn - 1) / g2.bn;
+    g2.b_rows_per_group = d->D; g2.b_row_step = g2.bn; g2.b_hi_offset = g2.bn / 2;
+    g2.out_cols = d->D; g2.out_col_step = g2.bn; g2.ldo = d->D; g2.out = out;
+    g2.comb_src = comb_src; g2.slot_of = slot_of; g2.k = k_comb;
+    g2.status = status;
+    MOE_CUDA(launch_gemm_sm100(g2, s));
+  } else {
+    SimtLaunch g1{};
+    g1.epi = EPI_SWIGLU;
+    g1.A = static_cast<const float*>(x); g1.K = d->D;
+    g1.B = static_cast<const float*>(w->sh_w1);
+    g1.num_groups = 1; g1.offsets = nullptr; g1.rows = d->T;
+    g1.b_rows_per_group = 2 * d->I_sh; g1.swiglu_hi = d->I_sh;
+    g1.out_cols = d->I_sh; g1.ldo = d->I_sh; g1.out = static_cast<float*>(h_sh);
+    MOE_CUDA(launch_simt_gemm(g1, s));
+    MOE_TRY(mk.at(6));
+    SimtLaunch g2{};
+    g2.epi = EPI_COMBINE;
+    g2.A = static_cast<const float*>(h_sh); g2.K = d->I_sh;
+    g2.B = static_cast<const float*>(w->sh_w2);
+    g2.num_groups = 1; g2.offsets = nullptr; g2.rows = d->T;
+    g2.b_rows_per_group = d->D;
+    g2.out_cols = d->D; g2.ldo = d->D; g2.out = static_cast<float*>(out);
+    g2.comb_src = static_cast<const float*>(comb_src); g2.slot_of = slot_of; g2.k = k_comb;
+    MOE_CUDA(launch_simt_gemm(g2, s));
+  }
+  return MOE_OK;
+}
+
+}  // namespace
+
+// =========================================================== public ABI
+extern "C" {
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+const char* moe_version(void) { return "moe_b200 0.1 (sm_100a)"; }
+
+moe_status_t moe_device_status(void* ws, void* stream, int* out) {
+  if (ws == nullptr || out == nullptr) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  MOE_CUDA(cudaMemcpyAsync(&v, ws, sizeof(int), cudaMemcpyDeviceToHost, s));
+  MOE_CUDA(cudaStreamSynchronize(s));
+  MOE_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), s));
+  *out = v;
+  return MOE_OK;
+}
+
+size_t moe_route_workspace_size(int T, int D, int M, int dtype) {
+  return route_layout(std::max(T, 0), std::max(D, 0), std::max(M, 0), dtype).total;
+}
+
+moe_status_t moe_route_topk(const void* x, const void* w_r, const float* e_bias, int T, int D, int M,
+                            int k, int dtype, int gate, int norm_topk_prob,
+                            float routed_scaling_factor, float eps, int32_t* topk_idx, float* topk_w,
+                            void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_router_args(T, D, M, k, dtype, gate));
+  if (!(eps >= 0.0f)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !w_r || !topk_idx || !topk_w || !ws || !aligned_ws(ws)) return MOE_ERR_INVALID_ARG;
+  const RouteWs L = route_layout(T, D, M, dtype);
+  if (ws_bytes < L.total) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_device());
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = at<int*>(ws, L.status);
+  MOE_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
+  return run_route(x, w_r, e_bias, T, D, M, k, dtype, gate, norm_topk_prob, routed_scaling_factor, eps,
+                   topk_idx, topk_w, at<float*>(ws, L.logits), at<void*>(ws, L.wrT), status, s);
+}
+
+size_t moe_permute_workspace_size(int T, int k, int M) {
+  return perm_layout(std::max(T, 0), std::max(k, 0), std::max(M, 0)).total;
+}
+
+moe_status_t moe_permute(const int32_t* topk_idx, const float* topk_w, int T, int k, int M,
+                         int32_t* counts, int32_t* offsets, int32_t* slot_of, int32_t* row_token,
+                         float* row_w, void* ws, size_t ws_bytes, void* stream) {
+  if (T < 0 || k < 1 || M < 1 || k > M) return MOE_ERR_INVALID_ARG;
+  if (M > kMaxExperts || k > kMaxTopK) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(T) * k >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+  if (!counts || !offsets || !ws || !aligned_ws(ws)) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!topk_idx || !topk_w || !slot_of || !row_token || !row_w)) return MOE_ERR_INVALID_ARG;
+  const PermWs L = perm_layout(T, k, M);
+  if (ws_bytes < L.total) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_device());
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = at<int*>(ws, L.status);
+  MOE_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
+  if (T == 0) {
+    MOE_CUDA(cudaMemsetAsync(counts, 0, static_cast<size_t>(M) * 4, s));
+    MOE_CUDA(cudaMemsetAsync(offsets, 0, static_cast<size_t>(M + 1) * 4, s));
+    return MOE_OK;
+  }
+  MOE_CUDA(launch_permute(topk_idx, topk_w, T, k, M, counts, offsets, slot_of, row_token, row_w,
+                          at<int32_t*>(ws, L.chunk_counts), at<int32_t*>(ws, L.chunk_base), status, s));
+  return MOE_OK;
+}
+
+size_t moe_expert_ffn_workspace_size(const moe_layer_desc_t* d) {
+  if (check_desc(d) != MOE_OK) return 0;
+  return ffn_layout(d).total;
+}
+
+moe_status_t moe_expert_ffn(const moe_layer_desc_t* d, const moe_weights_t* w, const void* x,
+                            const int32_t* offsets, const int32_t* row_token, const float* row_w,
+                            void* out_perm, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_desc(d));
+  MOE_TRY(check_weights(d, w, true, false));
+  if (d->T == 0) return MOE_OK;
+  if (!x || !offsets || !row_token || !row_w || !out_perm || !ws || !aligned_ws(ws))
+    return MOE_ERR_INVALID_ARG;
+  const FfnWs L = ffn_layout(d);
+  if (ws_bytes < L.total) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_device());
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = at<int*>(ws, L.status);
+  MOE_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
+  return run_experts(d, w, x, offsets, row_token, row_w, out_perm, at<void*>(ws, L.x_perm),
+                     at<void*>(ws, L.h), status, s);
+}
+
+size_t moe_shared_expert_workspace_size(const moe_layer_desc_t* d) {
+  if (check_desc(d) != MOE_OK) return 0;
+  return shared_layout(d).total;
+}
+
+moe_status_t moe_shared_expert(const moe_layer_desc_t* d, const moe_weights_t* w, const void* x,
+                               void* y_sh, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_desc(d));
+  if (d->I_sh == 0) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_weights(d, w, false, true));
+  if (d->T == 0) return MOE_OK;
+  if (!x || !y_sh || !ws || !aligned_ws(ws)) return MOE_ERR_INVALID_ARG;
+  const SharedWs L = shared_layout(d);
+  if (ws_bytes < L.total) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_device());
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = at<int*>(ws, L.status);
+  MOE_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
+  return run_shared(d, w, x, y_sh, at<void*>(ws, L.h_sh), nullptr, nullptr, 0, status, s);
+}
+
+moe_status_t moe_combine(const moe_layer_desc_t* d, const void* out_perm, const int32_t* slot_of,
+                         const void* shared_out, void* y, void* stream) {
+  MOE_TRY(check_desc(d));
+  if (d->T == 0) return MOE_OK;
+  if (!out_perm || !slot_of || !y) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_device());
+  MOE_CUDA(launch_combine(d->dtype, out_perm, slot_of, shared_out, y, d->T, d->D, d->k,
+                          static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+size_t moe_workspace_size(const moe_layer_desc_t* d) {
+  if (check_desc(d) != MOE_OK) return 0;
+  return forward_layout(d).pub.total;
+}
+
+moe_status_t moe_workspace_layout(const moe_layer_desc_t* d, moe_ws_layout_t* out) {
+  MOE_TRY(check_desc(d));
+  if (out == nullptr) return MOE_ERR_INVALID_ARG;
+  *out = forward_layout(d).pub;
+  return MOE_OK;
+}
+
+static moe_status_t forward_impl(const moe_layer_desc_t* d, const moe_weights_t* w, const void* x,
+                                 void* y, void* ws, size_t ws_bytes, cudaStream_t s,
+                                 void* const* events) {
+  MOE_TRY(check_desc(d));
+  MOE_TRY(check_weights(d, w, true, true));
+  if (w->w_r == nullptr) return MOE_ERR_INVALID_ARG;
+  if (d->T == 0) return MOE_OK;
+  if (!x || !y || !ws || !aligned_ws(ws)) return MOE_ERR_INVALID_ARG;
+  const FwdWs L = forward_layout(d);
+  if (ws_bytes < L.pub.total) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_device());
+  Marks mk;
+  mk.ev = events;
+  mk.s = s;
+  int* status = at<int*>(ws, L.pub.status);
+  int32_t* idx = at<int32_t*>(ws, L.pub.topk_idx);
+  float* tw = at<float*>(ws, L.pub.topk_w);
+  int32_t* counts = at<int32_t*>(ws, L.pub.counts);
+  int32_t* offsets = at<int32_t*>(ws, L.pub.offsets);
+  int32_t* slot_of = at<int32_t*>(ws, L.pub.slot_of);
+  int32_t* row_token = at<int32_t*>(ws, L.pub.row_token);
+  float* row_w = at<float*>(ws, L.pub.row_w);
+  void* out_perm = at<void*>(ws, L.pub.out_perm);
+  MOE_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
+  MOE_TRY(mk.at(0));
+  MOE_TRY(run_route(x, w->w_r, w->e_bias, d->T, d->D, d->M, d->k, d->dtype, d->gate, d->norm_topk_prob,
+                    d->routed_scaling_factor, d->eps, idx, tw, at<float*>(ws, L.logits),
+                    at<void*>(ws, L.wrT), status, s));
+  MOE_TRY(mk.at(1));
+  MOE_CUDA(launch_permute(idx, tw, d->T, d->k, d->M, counts, offsets, slot_of, row_token, row_w,
+                          at<int32_t*>(ws, L.chunk_counts), at<int32_t*>(ws, L.chunk_base), status, s));
+  MOE_TRY(mk.at(2));
+  MOE_TRY(run_experts(d, w, x, offsets, row_token, row_w, out_perm, at<void*>(ws, L.x_perm),
+                      at<void*>(ws, L.h), status, s, mk));
+  if (d->I_sh > 0) {
+    MOE_TRY(run_shared(d, w, x, y, at<void*>(ws, L.h_sh), out_perm, slot_of, d->k, status, s, mk));
+  } else {
+    MOE_TRY(mk.at(6));
+    MOE_CUDA(launch_combine(d->dtype, out_perm, slot_of, nullptr, y, d->T, d->D, d->k, s));
+  }
+  MOE_TRY(mk.at(7));
+  return MOE_OK;
+}
+
+moe_status_t moe_forward(const moe_layer_desc_t* d, const moe_weights_t* w, const void* x, void* y,
+                         void* ws, size_t ws_bytes, void* stream) {
+  return forward_impl(d, w, x, y, ws, ws_bytes, static_cast<cudaStream_t>(stream), nullptr);
+}
+
+moe_status_t moe_forward_profiled(const moe_layer_desc_t* d, const moe_weights_t* w, const void* x,
+                                  void* y, void* ws, size_t ws_bytes, void* stream,
+                                  void* const* events, int n_events) {
+  if (events == nullptr || n_events != MOE_NUM_STAGE_EVENTS) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < n_events; ++i)
+    if (events[i] == nullptr) return MOE_ERR_INVALID_ARG;
+  return forward_impl(d, w, x, y, ws, ws_bytes, static_cast<cudaStream_t>(stream), events);
+}
+
+int moe_forward_launch_count(const moe_layer_desc_t* d) {
+  if (check_desc(d) != MOE_OK || d->T == 0) return 0;
+  const bool bf16 = d->dtype == MOE_DTYPE_BF16;
+  int n = bf16 ? 3 : 2;   // [transpose,] logits, top-k
+  n += 3;                 // histogram, scan, scatter
+  n += bf16 ? 3 : 2;      // [gather,] first GEMM, second GEMM
+  n += d->I_sh > 0 ? 2 : 1;  // shared first GEMM + fused combine, or combine
+  return n;
+}
+
+void moe_algorithmic_work(const moe_layer_desc_t* d, const int32_t* counts_host, double* flops,
+                          double* bytes) {
+  double f = 0.0, b = 0.0;
+  if (d != nullptr && check_desc(d) == MOE_OK) {
+    const double es = static_cast<double>(esize(d->dtype));
+    const double D = d->D, I = d->I, T = d->T, Ish = d->I_sh;
+    const bool swiglu = d->act == MOE_ACT_SWIGLU;
+    const double n1 = swiglu ? 2.0 * I : I;
+    const double bias_params = (!swiglu && d->has_bias) ? (I + D) : 0.0;
+    f += 2.0 * T * D * d->M;           // router
+    b += D * d->M * es + T * D * es * 2.0;  // W_r, x in, y out
+    if (d->gate == MOE_GATE_SIGMOID_BIAS) b += 4.0 * d->M;
+    for (int e = 0; e < d->M; ++e) {
+      const double c = counts_host ? counts_host[e] : 0.0;
+      if (c <= 0) continue;
+      f += c * (2.0 * D * n1 + 2.0 * I * D);
+      b += (n1 * D + D * I + bias_params) * es;
+    }
+    if (Ish > 0) {
+      f += T * (2.0 * D * 2.0 * Ish + 2.0 * Ish * D);
+      b += 3.0 * D * Ish * es;
+    }
+  }
+  if (flops) *flops = f;
+  if (bytes) *bytes = b;
+}
+
+}  // extern "C"

@@ -1,0 +1,98 @@
+"""Torch-side convenience around the C ABI: descriptor and weight structs
+from tensors, a workspace buffer, and views of the intermediates that
+moe_forward leaves in it.  No computation happens here."""
+from __future__ import annotations
+
+import torch
+
+from . import abi
+
+_GATES = {"softmax": abi.GATE_SOFTMAX, "sigmoid_bias": abi.GATE_SIGMOID_BIAS}
+_ACTS = {"gelu_tanh": abi.ACT_GELU_TANH, "swiglu": abi.ACT_SWIGLU}
+_DTYPES = {"f32": abi.DTYPE_F32, "bf16": abi.DTYPE_BF16}
+
+
+def desc_from_config(cfg: dict, T: int | None = None) -> abi.LayerDesc:
+    d = abi.LayerDesc()
+    d.dtype = _DTYPES[cfg["dtype"]]
+    d.T = cfg["T"] if T is None else T
+    d.D, d.M, d.k, d.I = cfg["D"], cfg["M"], cfg["k"], cfg["I"]
+    d.gate = _GATES[cfg["gate"]]
+    d.act = _ACTS[cfg["act"]]
+    d.has_bias = int(bool(cfg.get("has_bias", 0)))
+    d.norm_topk_prob = int(bool(cfg.get("norm_topk_prob", 1)))
+    d.routed_scaling_factor = float(cfg.get("alpha", 1.0))
+    d.eps = float(cfg.get("eps", 1e-20))
+    d.I_sh = int(cfg.get("I_sh", 0) or 0)
+    return d
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def weights_from_tensors(t: dict) -> abi.Weights:
+    w = abi.Weights()
+    for name in ("w_r", "e_bias", "w1", "b1", "w2", "b2", "sh_w1", "sh_w2"):
+        v = t.get(name)
+        if v is not None and not v.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        setattr(w, name, _ptr(v))
+    return w
+
+
+def _stream_handle(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+class MoELayer:
+    """One MoE layer bound to device weight tensors (kept alive here)."""
+
+    def __init__(self, cfg: dict, tensors: dict, T: int | None = None):
+        self.cfg = cfg
+        self.tensors = tensors
+        self.desc = desc_from_config(cfg, T)
+        self.weights = weights_from_tensors(tensors)
+        self.device = tensors["w_r"].device
+        self.ws_bytes = abi.moe_workspace_size(self.desc)
+        if self.ws_bytes == 0:
+            raise abi.MoEError("moe_workspace_size", abi.MOE_ERR_INVALID_ARG)
+        self.ws = torch.zeros(self.ws_bytes + 256, dtype=torch.uint8, device=self.device)
+        base = self.ws.data_ptr()
+        self._ws_off = (-base) % 256
+        self.layout = abi.moe_workspace_layout(self.desc)
+
+    @property
+    def ws_ptr(self) -> int:
+        return self.ws.data_ptr() + self._ws_off
+
+    def forward(self, x: torch.Tensor, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        if y is None:
+            y = torch.empty_like(x)
+        abi.moe_forward(self.desc, self.weights, x.data_ptr(), y.data_ptr(), self.ws_ptr, self.ws_bytes,
+                        _stream_handle(stream))
+        return y
+
+    def device_status(self, stream=None) -> int:
+        return abi.moe_device_status(self.ws_ptr, _stream_handle(stream))
+
+    def view(self, name: str, dtype=None) -> torch.Tensor:
+        """The intermediate ``name`` of the last forward, as a tensor view."""
+        d = self.desc
+        pairs = d.T * d.k
+        shapes = {
+            "status": ((1,), torch.int32), "topk_idx": ((d.T, d.k), torch.int32),
+            "topk_w": ((d.T, d.k), torch.float32), "counts": ((d.M,), torch.int32),
+            "offsets": ((d.M + 1,), torch.int32), "slot_of": ((d.T, d.k), torch.int32),
+            "row_token": ((pairs,), torch.int32), "row_w": ((pairs,), torch.float32),
+            "out_perm": ((pairs, d.D), torch.float32),
+        }
+        shape, dt = shapes[name]
+        off = self._ws_off + getattr(self.layout, name)
+        n = 1
+        for s in shape:
+            n *= s
+        nbytes = n * torch.empty((), dtype=dt).element_size()
+        return self.ws[off:off + nbytes].view(dt).view(*shape)

@@ -1,0 +1,134 @@
+"""The C-ABI library loads and exports every symbol the header declares; the
+host-side argument checks answer without touching a GPU."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import moe_synth as ms
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_b200.h")
+
+
+@pytest.fixture(scope="module")
+def B():
+    from sparse_mixture_experts_logits_b200 import build
+    build.build()
+    import sparse_mixture_experts_logits_b200 as B
+    return B
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("moe_route_topk", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(B):
+    lib = ctypes.CDLL(B.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert sorted(B.EXPORTED_SYMBOLS) == declared_functions()
+
+
+def test_version_and_status_strings(B):
+    assert "sm_100a" in B.moe_version()
+    assert B.moe_status_string(0) == "MOE_OK"
+    assert B.moe_status_string(4) == "MOE_ERR_DEVICE"
+    assert B.moe_status_string(99) == "MOE_ERR_UNKNOWN"
+
+
+def test_struct_layout_matches_header(B):
+    assert ctypes.sizeof(B.LayerDesc) == 13 * 4
+    assert ctypes.sizeof(B.Weights) == 8 * 8
+    assert ctypes.sizeof(B.WsLayout) == 10 * 8
+
+
+def _desc(B, name, **kw):
+    return B.desc_from_config(ms.get_config(name, **kw))
+
+
+def test_invalid_arguments_are_rejected_on_the_host(B):
+    d = _desc(B, "glm_small_bf16")
+    w = B.Weights()
+    # k > M, k < 1, bad dtype, bf16 width not a multiple of 16
+    for field, value, code in [("k", 17, 1), ("k", 0, 1), ("dtype", 7, 2), ("D", 250, 2),
+                               ("I", 100, 2), ("M", 2000, 2), ("act", 5, 1), ("T", -1, 1)]:
+        dd = _desc(B, "glm_small_bf16")
+        setattr(dd, field, value)
+        with pytest.raises(B.MoEError) as e:
+            B.moe_forward(dd, w, 1, 1, 256, 1 << 30)
+        assert e.value.status == code, (field, value)
+        assert B.moe_workspace_size(dd) == 0
+    # null weights
+    with pytest.raises(B.MoEError) as e:
+        B.moe_forward(d, w, 1, 1, 256, 1 << 30)
+    assert e.value.status == 1
+    # workspace too small / misaligned
+    w.w_r, w.w1, w.w2, w.sh_w1, w.sh_w2 = 256, 256, 256, 256, 256
+    need = B.moe_workspace_size(d)
+    with pytest.raises(B.MoEError) as e:
+        B.moe_forward(d, w, 256, 256, 256, need - 1)
+    assert e.value.status == 1
+    with pytest.raises(B.MoEError) as e:
+        B.moe_forward(d, w, 256, 256, 255, need)
+    assert e.value.status == 1
+    with pytest.raises(B.MoEError):
+        B.moe_route_topk(256, 256, None, 10, 64, 8, 9, 1, 0, 1, 1.0, 1e-20, 256, 256, 256, 1 << 20)
+    with pytest.raises(B.MoEError):
+        B.moe_permute(256, 256, 10, 2, 8, 256, 256, 256, 256, 256, 256, 0)
+
+
+def test_zero_tokens_launch_nothing(B):
+    d = _desc(B, "glm_small_bf16", T=0)
+    w = B.Weights()
+    w.w_r, w.w1, w.w2, w.sh_w1, w.sh_w2 = 256, 256, 256, 256, 256
+    B.moe_forward(d, w, None, None, None, 0)
+    B.moe_route_topk(None, None, None, 0, 64, 8, 2, 1, 0, 1, 1.0, 1e-20, None, None, None, 0)
+    B.moe_expert_ffn(d, w, None, None, None, None, None, None, 0)
+    B.moe_combine(d, None, None, None, None)
+
+
+def test_workspace_layout_is_aligned_and_ordered(B):
+    for name in ms.all_config_names():
+        d = _desc(B, name)
+        L = B.moe_workspace_layout(d)
+        offs = [L.status, L.topk_idx, L.topk_w, L.counts, L.offsets, L.slot_of, L.row_token,
+                L.row_w, L.out_perm]
+        assert all(o % 256 == 0 for o in offs)
+        assert offs == sorted(offs) and L.total >= offs[-1] + d.T * d.k * d.D * (2 if d.dtype else 4)
+        assert B.moe_workspace_size(d) == L.total
+        assert B.moe_expert_ffn_workspace_size(d) > 0
+
+
+def test_algorithmic_work_closed_form(B):
+    """FLOPs and bytes of the GLaM prefill layer from the shapes alone:
+    every token runs 2 experts of 2*D*H*2 FLOPs; the router D*M*2 per token."""
+    cfg = ms.get_config("glam_prefill_bf16")
+    d = B.desc_from_config(cfg)
+    T, D, M, H = cfg["T"], cfg["D"], cfg["M"], cfg["I"]
+    counts = np.full(M, T * 2 // M, dtype=np.int32)
+    f, b = B.moe_algorithmic_work(d, counts)
+    assert f == 2 * T * D * M + T * 2 * (2 * D * H * 2)
+    weights = M * (2 * D * H + H + D) * 2
+    assert b == weights + D * M * 2 + 2 * T * D * 2
+    assert abs(f / 1e12 - 1.1017) < 1e-3
+    # untouched experts cost no bytes
+    counts[1:] = 0
+    counts[0] = T * 2
+    f2, b2 = B.moe_algorithmic_work(d, counts)
+    assert f2 == f and b2 == (2 * D * H + H + D) * 2 + D * M * 2 + 2 * T * D * 2
+    # GLM-5 shared expert bytes: 3 * 6144 * 2048 parameters at 2 bytes
+    cfg5 = ms.get_config("glm5_skewed_prefill_bf16")
+    d5 = B.desc_from_config(cfg5)
+    f5, b5 = B.moe_algorithmic_work(d5, np.zeros(cfg5["M"], np.int32))
+    assert b5 == 37748736 * 2 + 6144 * 256 * 2 + 4 * 256 + 2 * cfg5["T"] * 6144 * 2

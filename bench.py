@@ -54,6 +54,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU-baseline run time")
+    ap.add_argument("--T", type=int, default=None, help="override tokens per GPU (profiling runs)")
+    ap.add_argument("--M", type=int, default=None, help="override routed experts (profiling runs)")
     return ap.parse_args()
 
 
@@ -203,6 +205,15 @@ def stage_work(cfg, counts):
     return w
 
 
+def workload_config(args):
+    over = {}
+    if args.T is not None:
+        over["T"] = args.T
+    if args.M is not None:
+        over["M"] = args.M
+    return ms.get_config(args.config, **over)
+
+
 # --------------------------------------------------------------------------
 # the GPU arm
 # --------------------------------------------------------------------------
@@ -217,7 +228,7 @@ def run_ours(args):
     torch.cuda.set_device(dev)
     dist = dist_init(world, local_rank)
 
-    cfg = ms.get_config(args.config)
+    cfg = workload_config(args)
     T, D = cfg["T"], cfg["D"]
     inp = ms.layer_inputs(dict(cfg, T=1), dev)  # weights; x below
     r0, r1 = token_rows(rank, T)
@@ -346,7 +357,8 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": cfg["dtype"],
         "data": "synthetic (seeded counter-based generator; random-init weights)",
-        "config": {"workload": args.config, "T_per_gpu": T, "D": D, "M": cfg["M"], "k": cfg["k"],
+        "config": {"workload": args.config + ("" if cfg["named"] else " (overridden: T=%d, M=%d)" % (T, cfg["M"])),
+                   "T_per_gpu": T, "D": D, "M": cfg["M"], "k": cfg["k"],
                    "I": cfg["I"], "I_sh": cfg.get("I_sh", 0), "gate": cfg["gate"], "act": cfg["act"],
                    "l2": "flushed between steps (256 MiB write outside the timed events)",
                    "parallelism": f"replicas x{world} (token batches, no data-path collective)"},
@@ -442,7 +454,7 @@ def run_reference(args):
     rank, local_rank, world = dist_env()
     if rank != 0:
         return
-    cfg = ms.get_config(args.config)
+    cfg = workload_config(args)
     dev = torch.device("cuda", local_rank) if torch.cuda.is_available() else torch.device("cpu")
     inp = ms.layer_inputs(cfg, dev)
     runner = OracleRunner(cfg, inp)

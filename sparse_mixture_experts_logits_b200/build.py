@@ -1,6 +1,6 @@
 """Build the sm_100a CUDA library ``libmoe_b200.so`` in place.
 
-    python -m sparse_mixture_experts_logits_b200.build [--verbose-ptxas]
+    python sparse_mixture_experts_logits_b200/build.py [--force] [--verbose-ptxas]
 
 Every ``csrc/*.cu`` file is compiled by nvcc for sm_100a only and linked,
 with the CUDA runtime linked statically, into one shared library next to

@@ -15,8 +15,8 @@ HEADER = os.path.join(ROOT, "include", "moe_b200.h")
 
 @pytest.fixture(scope="module")
 def B():
-    from sparse_mixture_experts_logits_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__._build_module().build()
     import sparse_mixture_experts_logits_b200 as B
     return B
 

@@ -168,6 +168,27 @@ moe_status_t moe_permute(const int32_t* topk_idx, const float* topk_w, int T, in
                          int32_t* row_token, float* row_w,
                          void* ws, size_t ws_bytes, void* stream);
 
+/* The same dispatch as moe_permute, for callers that cannot allocate device
+ * memory where they route tokens (a process whose device memory is owned by
+ * a pool, a latency-critical loop that cannot take cudaMalloc's implicit
+ * synchronisation, a plug-in host without an allocator).  The source pages
+ * have no counterpart for this entry point: it exists for those callers.
+ *   Scratch: a 4 MiB array compiled into the library, reserved on every GPU
+ *   that loads the library until the process exits.  Supported sizes:
+ *   M * ceil(T*k / 512) <= 524288; larger requests return
+ *   MOE_ERR_UNSUPPORTED without launching.  No cudaMalloc/cudaFree.
+ *   device_status: optional int32 device word, cleared by the call, set to
+ *   MOE_DEVERR_BAD_EXPERT_INDEX if topk_idx holds an index outside [0, M).
+ *   All calls on a device share the scratch array; calls whose kernels
+ *   overlap on the GPU (unordered streams) race and may give wrong results.
+ *   The first call on each device looks up the array's address with that
+ *   device current; make it before any stream capture begins.
+ * Other arguments and outputs: as moe_permute (bit-identical results). */
+moe_status_t moe_permute_static_scratch(const int32_t* topk_idx, const float* topk_w, int T, int k,
+                                        int M, int32_t* counts, int32_t* offsets, int32_t* slot_of,
+                                        int32_t* row_token, float* row_w, int32_t* device_status,
+                                        void* stream);
+
 /* ---- experts: "GLaM" eq. FFN; GLM-5 GlmMoeDsaExperts.forward ----------- */
 
 size_t moe_expert_ffn_workspace_size(const moe_layer_desc_t* d);

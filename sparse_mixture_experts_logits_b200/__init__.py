@@ -11,7 +11,7 @@ from .abi import (  # noqa: F401
     LIB_PATH, MoEError, LayerDesc, Weights, WsLayout, lib,
     moe_status_string, moe_version, moe_device_status,
     moe_route_workspace_size, moe_route_topk,
-    moe_permute_workspace_size, moe_permute,
+    moe_permute_workspace_size, moe_permute, moe_permute_static_scratch,
     moe_expert_ffn_workspace_size, moe_expert_ffn,
     moe_shared_expert_workspace_size, moe_shared_expert,
     moe_combine, moe_workspace_size, moe_workspace_layout, moe_forward,

@@ -21,7 +21,7 @@ DEVERR_NONE, DEVERR_BAD_EXPERT_INDEX, DEVERR_TIMEOUT = 0, 1, 2
 EXPORTED_SYMBOLS = [
     "moe_status_string", "moe_version", "moe_device_status",
     "moe_route_workspace_size", "moe_route_topk",
-    "moe_permute_workspace_size", "moe_permute",
+    "moe_permute_workspace_size", "moe_permute", "moe_permute_static_scratch",
     "moe_expert_ffn_workspace_size", "moe_expert_ffn",
     "moe_shared_expert_workspace_size", "moe_shared_expert",
     "moe_combine", "moe_workspace_size", "moe_workspace_layout", "moe_forward",
@@ -60,7 +60,7 @@ class WsLayout(ctypes.Structure):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m sparse_mixture_experts_logits_b200.build` "
+            f"{LIB_PATH} is missing: build it with `python sparse_mixture_experts_logits_b200/build.py` "
             "(there is no fallback path)")
     return ctypes.CDLL(LIB_PATH)
 
@@ -85,6 +85,7 @@ _decl("moe_route_workspace_size", _sz, [_i, _i, _i, _i])
 _decl("moe_route_topk", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _f, _vp, _vp, _vp, _sz, _vp])
 _decl("moe_permute_workspace_size", _sz, [_i, _i, _i])
 _decl("moe_permute", _i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
+_decl("moe_permute_static_scratch", _i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp])
 _decl("moe_expert_ffn_workspace_size", _sz, [_P(LayerDesc)])
 _decl("moe_expert_ffn", _i, [_P(LayerDesc), _P(Weights), _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
 _decl("moe_shared_expert_workspace_size", _sz, [_P(LayerDesc)])
@@ -140,6 +141,13 @@ def moe_permute(topk_idx, topk_w, T, k, M, counts, offsets, slot_of, row_token, 
                 stream=None):
     _check("moe_permute", lib.moe_permute(topk_idx, topk_w, T, k, M, counts, offsets, slot_of,
                                           row_token, row_w, ws, ws_bytes, stream))
+
+
+def moe_permute_static_scratch(topk_idx, topk_w, T, k, M, counts, offsets, slot_of, row_token, row_w,
+                               device_status=None, stream=None):
+    """moe_permute without a workspace (scratch compiled into the library)."""
+    _check("moe_permute_static_scratch", lib.moe_permute_static_scratch(
+        topk_idx, topk_w, T, k, M, counts, offsets, slot_of, row_token, row_w, device_status, stream))
 
 
 def moe_expert_ffn_workspace_size(desc: LayerDesc) -> int:

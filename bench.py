@@ -200,7 +200,8 @@ def stage_work(cfg, counts):
         "expert_up": (2.0 * pairs * D * n1, touched * (n1 * D + (I if bias else 0)) * es),
         "expert_down": (2.0 * pairs * I * D, touched * (D * I + (D if bias else 0)) * es),
         "shared_up": (2.0 * T * D * 2 * Ish, 2.0 * Ish * D * es),
-        "combine": (2.0 * T * Ish * D, (D * Ish * es if Ish else 0) + 2.0 * T * D * es),
+        "shared_down": (2.0 * T * Ish * D, D * Ish * es),
+        "combine": (0.0, T * D * es),
     }
     return w
 
@@ -326,7 +327,7 @@ def run_ours(args):
     peaks, peak_src = load_peaks()
     work = stage_work(cfg, counts)
     flops_total, bytes_total = B.moe_algorithmic_work(layer.desc, counts)
-    gemm_stages = [s for s in ("expert_up", "expert_down", "shared_up", "combine") if stage_ms[s] > 0.002]
+    gemm_stages = [s for s in ("expert_up", "expert_down", "shared_up", "shared_down") if stage_ms[s] > 0.002]
     dom = max(gemm_stages, key=lambda s: stage_ms[s])
     f, b = work[dom]
     t_s = stage_ms[dom] / 1e3

@@ -226,20 +226,23 @@ moe_status_t moe_combine(const moe_layer_desc_t* d, const void* out_perm,
 size_t moe_workspace_size(const moe_layer_desc_t* d);
 moe_status_t moe_workspace_layout(const moe_layer_desc_t* d, moe_ws_layout_t* out);
 
-/* y[T, D] = MoE-FFN(x): route, dispatch, routed experts, and the combine
- * fused with the shared expert's down projection (when I_sh > 0).  All
- * stages run back to back on `stream` with no host synchronisation. */
+/* y[T, D] = MoE-FFN(x): route, dispatch, routed experts, shared expert (when
+ * I_sh > 0, its output kept in fp32) and the combine, which adds each
+ * token's k weighted expert rows and its shared-expert row in fp32 and
+ * rounds once.  All stages run back to back on `stream` with no host
+ * synchronisation. */
 moe_status_t moe_forward(const moe_layer_desc_t* d, const moe_weights_t* w,
                          const void* x, void* y, void* ws, size_t ws_bytes, void* stream);
 
 /* Stage boundaries recorded by moe_forward_profiled (the "routing overhead"
  * breakdown of the GLaM note's reporting table: gate, dispatch, expert
  * batching, combination cost). */
-#define MOE_NUM_STAGE_EVENTS 8
+#define MOE_NUM_STAGE_EVENTS 9
 /* event 0: start; 1: route done (scores, top-k, weights); 2: dispatch order
  * done; 3: rows gathered into dispatch order; 4: routed experts' first GEMM
  * done; 5: routed experts' second GEMM done; 6: shared expert's first GEMM
- * done; 7: combine (fused with the shared down projection) done.  Stages a
+ * done; 7: shared expert's second GEMM done; 8: combine (the k routed rows
+ * of every token plus its shared-expert row) done.  Stages a
  * layer does not have record their event right after the previous one. */
 
 /* moe_forward, recording `events[i]` (cudaEvent_t handles created by the

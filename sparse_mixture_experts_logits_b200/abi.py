@@ -27,8 +27,9 @@ EXPORTED_SYMBOLS = [
     "moe_combine", "moe_workspace_size", "moe_workspace_layout", "moe_forward",
     "moe_forward_profiled", "moe_forward_launch_count", "moe_algorithmic_work",
 ]
-NUM_STAGE_EVENTS = 8
-STAGE_NAMES = ["route", "dispatch", "gather", "expert_up", "expert_down", "shared_up", "combine"]
+NUM_STAGE_EVENTS = 9
+STAGE_NAMES = ["route", "dispatch", "gather", "expert_up", "expert_down", "shared_up", "shared_down",
+               "combine"]
 
 
 class MoEError(RuntimeError):

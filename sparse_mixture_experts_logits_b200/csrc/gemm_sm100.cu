@@ -2,6 +2,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "gemm_sm100.cuh"
@@ -39,20 +40,56 @@ bool make_tmap(CUtensorMap* map, const void* base, long long rows, int K, int bo
   return r == CUDA_SUCCESS;
 }
 
-template <int EPI>
-cudaError_t launch_epi(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args, int grid,
-                       cudaStream_t s) {
-  static int configured_mask = 0;  // one bit per device
+template <int EPI, int NCTA>
+cudaError_t launch_epi(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args,
+                       long long tiles_ub, cudaStream_t s) {
+  static std::atomic<unsigned> configured{0};  // one bit per device
+  static std::atomic<int> max_units[32];       // CTAs (NCTA = 1) or clusters (NCTA = 2) per device
   int dev = 0;
   cudaGetDevice(&dev);
-  if (!(configured_mask & (1 << (dev & 31)))) {
-    cudaError_t e = cudaFuncSetAttribute(moe_gemm_sm100_kernel<EPI>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmDynSmem);
+  auto kernel = moe_gemm_sm100_kernel<EPI, NCTA>;
+  constexpr int smem = gemm_dyn_smem<NCTA>();
+  const unsigned bit = 1u << (dev & 31);
+  if (!(configured.load() & bit)) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    configured_mask |= 1 << (dev & 31);
+    int units = num_sms();
+    if (NCTA == 2) {
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+      (void)e;
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3(2 * (units / 2), 1, 1);
+      q.blockDim = dim3(kGemmThreads, 1, 1);
+      q.dynamicSmemBytes = smem;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = 2;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      q.attrs = at;
+      q.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &q) != cudaSuccess || clusters <= 0)
+        clusters = units / 2;
+      units = clusters;
+    }
+    max_units[dev & 31].store(units);
+    configured.fetch_or(bit);
   }
-  moe_gemm_sm100_kernel<EPI><<<grid, kGemmThreads, kGemmDynSmem, s>>>(ta, tb, args);
-  return cudaGetLastError();
+  const long long units = std::min<long long>(max_units[dev & 31].load(), std::max<long long>(1, tiles_ub));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(units * NCTA), 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = NCTA;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, ta, tb, args);
 }
 
 }  // namespace
@@ -71,8 +108,10 @@ int num_sms() {
 }
 
 cudaError_t launch_gemm_sm100(const GemmLaunch& L, cudaStream_t s) {
+  const int ncta = L.ncta == 1 ? 1 : 2;
+  const int tile_rows = 128 * ncta;
   CUtensorMap ta, tb;
-  if (!make_tmap(&ta, L.A, L.a_rows, L.K, kBM)) return cudaErrorInvalidValue;
+  if (!make_tmap(&ta, L.A, L.a_rows, L.K, 128)) return cudaErrorInvalidValue;
   if (!make_tmap(&tb, L.B, L.b_rows, L.K, L.bn / 2)) return cudaErrorInvalidValue;
   GemmArgs a;
   a.num_groups = L.num_groups;
@@ -93,20 +132,23 @@ cudaError_t launch_gemm_sm100(const GemmLaunch& L, cudaStream_t s) {
   a.comb_src = static_cast<const float*>(L.comb_src);
   a.slot_of = L.slot_of;
   a.k = L.k;
-  a.idesc = umma_idesc_bf16(kBM, L.bn);
+  a.idesc = umma_idesc_bf16(tile_rows, L.bn);
   a.status = L.status;
-  // upper bound of the tile count: sum_g ceil(rows_g / 128) <= rows/128 + (#non-empty groups)
-  long long mt_ub = L.offsets ? L.rows_upper / kBM + std::min<long long>(L.num_groups, L.rows_upper)
-                              : (L.a_rows + kBM - 1) / kBM;
-  long long tiles_ub = mt_ub * L.n_tiles;
-  int grid = static_cast<int>(std::min<long long>(num_sms(), std::max<long long>(1, tiles_ub)));
+  // upper bound of the tile count: sum_g ceil(rows_g / tile_rows) <= rows/tile_rows + (#non-empty groups)
+  const long long mt_ub = L.offsets ? L.rows_upper / tile_rows + std::min<long long>(L.num_groups, L.rows_upper)
+                                    : (L.a_rows + tile_rows - 1) / tile_rows;
+  const long long tiles_ub = mt_ub * L.n_tiles;
+#define MOE_GEMM_CASE(E)                                                              \
+  case E:                                                                             \
+    return ncta == 2 ? launch_epi<E, 2>(ta, tb, a, tiles_ub, s) : launch_epi<E, 1>(ta, tb, a, tiles_ub, s);
   switch (L.epi) {
-    case EPI_STORE_F32: return launch_epi<EPI_STORE_F32>(ta, tb, a, grid, s);
-    case EPI_GELU_BIAS: return launch_epi<EPI_GELU_BIAS>(ta, tb, a, grid, s);
-    case EPI_SWIGLU: return launch_epi<EPI_SWIGLU>(ta, tb, a, grid, s);
-    case EPI_SCALE_BIAS: return launch_epi<EPI_SCALE_BIAS>(ta, tb, a, grid, s);
-    case EPI_COMBINE: return launch_epi<EPI_COMBINE>(ta, tb, a, grid, s);
+    MOE_GEMM_CASE(EPI_STORE_F32)
+    MOE_GEMM_CASE(EPI_GELU_BIAS)
+    MOE_GEMM_CASE(EPI_SWIGLU)
+    MOE_GEMM_CASE(EPI_SCALE_BIAS)
+    MOE_GEMM_CASE(EPI_COMBINE)
   }
+#undef MOE_GEMM_CASE
   return cudaErrorInvalidValue;
 }
 

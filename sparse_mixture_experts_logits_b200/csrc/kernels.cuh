@@ -27,11 +27,13 @@ cudaError_t launch_permute(const int32_t* topk_idx, const float* topk_w, int T, 
 cudaError_t launch_gather_rows(const void* x, const int32_t* row_token, void* x_perm, int rows,
                                int D, int elem_bytes, cudaStream_t s);
 cudaError_t launch_combine(int dtype, const void* out_perm, const int32_t* slot_of,
-                           const void* shared_out, void* y, int T, int D, int k, cudaStream_t s);
+                           const void* shared_out, bool shared_f32, void* y, int T, int D, int k,
+                           cudaStream_t s);
 
 // gemm_sm100.cu: grouped bf16 GEMM on tcgen05.  `epi` is a GemmEpilogue.
 struct GemmLaunch {
   int epi;
+  int ncta;  // 1: one CTA per 128-row tile; 2 (default, 0): 2-SM MMA on CTA pairs, 256-row tiles
   const void* A; long long a_rows; // bf16 [a_rows, K]
   const void* B; long long b_rows; // bf16 [b_rows, K]
   int K;

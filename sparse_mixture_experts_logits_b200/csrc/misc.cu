@@ -40,11 +40,47 @@ cudaError_t launch_gather_rows(const void* x, const int32_t* row_token, void* x_
 }
 
 // y[t, :] = sum_j out_perm[slot_of[t, j], :] (+ shared[t, :]) in fp32, in
-// slot order, rounded once.  out_perm is fp32; shared and y have the layer's
-// type.  One block per token.
-template <typename T>
+// slot order, rounded once.  out_perm is fp32; shared is fp32 or the layer's
+// type; y has the layer's type.  One block per token; every row read is
+// contiguous, and the k rows of a token are loaded together.
+template <typename TY, typename TS>
+__global__ void __launch_bounds__(128) combine_vec4_kernel(const float4* __restrict__ out_perm,
+                                                           const int32_t* __restrict__ slot_of,
+                                                           const TS* __restrict__ shared, TY* __restrict__ y,
+                                                           int D4, int k) {
+  __shared__ int s_slot[kMaxTopK];
+  const int t = blockIdx.x;
+  if (threadIdx.x < k) s_slot[threadIdx.x] = slot_of[static_cast<size_t>(t) * k + threadIdx.x];
+  __syncthreads();
+  for (int v = threadIdx.x; v < D4; v += blockDim.x) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+    for (int j = 0; j < k; ++j) {
+      const float4 a = out_perm[static_cast<size_t>(s_slot[j]) * D4 + v];
+      acc.x += a.x; acc.y += a.y; acc.z += a.z; acc.w += a.w;
+    }
+    if (shared != nullptr) {
+      const size_t e = (static_cast<size_t>(t) * D4 + v) * 4;
+      acc.x += to_f32(shared[e]); acc.y += to_f32(shared[e + 1]);
+      acc.z += to_f32(shared[e + 2]); acc.w += to_f32(shared[e + 3]);
+    }
+    const size_t o = (static_cast<size_t>(t) * D4 + v) * 4;
+    if constexpr (sizeof(TY) == 2) {
+      __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+      uint2 u;
+      u.x = *reinterpret_cast<uint32_t*>(&lo);
+      u.y = *reinterpret_cast<uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(y + o) = u;
+    } else {
+      *reinterpret_cast<float4*>(y + o) = acc;
+    }
+  }
+}
+
+// Any D: one element per thread step.
+template <typename TY, typename TS>
 __global__ void combine_kernel(const float* __restrict__ out_perm, const int32_t* __restrict__ slot_of,
-                               const T* __restrict__ shared, T* __restrict__ y, int D, int k) {
+                               const TS* __restrict__ shared, TY* __restrict__ y, int D, int k) {
   const int t = blockIdx.x;
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
     float acc = 0.f;
@@ -53,52 +89,32 @@ __global__ void combine_kernel(const float* __restrict__ out_perm, const int32_t
       acc += out_perm[static_cast<size_t>(slot) * D + d];
     }
     if (shared != nullptr) acc += to_f32(shared[static_cast<size_t>(t) * D + d]);
-    y[static_cast<size_t>(t) * D + d] = from_f32<T>(acc);
+    y[static_cast<size_t>(t) * D + d] = from_f32<TY>(acc);
   }
 }
 
-// bf16 output, 8 columns per thread.
-__global__ void combine_bf16x8_kernel(const float4* __restrict__ out_perm,
-                                      const int32_t* __restrict__ slot_of,
-                                      const uint4* __restrict__ shared, uint4* __restrict__ y,
-                                      int vecs, int k) {
-  const int t = blockIdx.x;
-  for (int v = threadIdx.x; v < vecs; v += blockDim.x) {
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j < k; ++j) {
-      const int slot = slot_of[static_cast<size_t>(t) * k + j];
-      const float4 a = out_perm[(static_cast<size_t>(slot) * vecs + v) * 2];
-      const float4 b = out_perm[(static_cast<size_t>(slot) * vecs + v) * 2 + 1];
-      acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-      acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
-    }
-    if (shared != nullptr) {
-      float f[8];
-      bf16x8_to_f32(shared[static_cast<size_t>(t) * vecs + v], f);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] += f[i];
-    }
-    y[static_cast<size_t>(t) * vecs + v] = f32_to_bf16x8(acc);
+template <typename TY, typename TS>
+static cudaError_t combine_typed(const float* op, const int32_t* slot_of, const void* shared, void* y,
+                                 int T, int D, int k, cudaStream_t s) {
+  if (D % 4 == 0) {
+    combine_vec4_kernel<TY, TS><<<T, 128, 0, s>>>(reinterpret_cast<const float4*>(op), slot_of,
+                                                  static_cast<const TS*>(shared), static_cast<TY*>(y), D / 4, k);
+  } else {
+    combine_kernel<TY, TS><<<T, 128, 0, s>>>(op, slot_of, static_cast<const TS*>(shared),
+                                             static_cast<TY*>(y), D, k);
   }
+  return cudaGetLastError();
 }
 
 cudaError_t launch_combine(int dtype, const void* out_perm, const int32_t* slot_of,
-                           const void* shared_out, void* y, int T, int D, int k, cudaStream_t s) {
+                           const void* shared_out, bool shared_f32, void* y, int T, int D, int k,
+                           cudaStream_t s) {
   const float* op = static_cast<const float*>(out_perm);
-  if (dtype == MOE_DTYPE_BF16 && D % 8 == 0) {
-    const int vecs = D / 8;
-    combine_bf16x8_kernel<<<T, min(256, ((vecs + 31) / 32) * 32), 0, s>>>(
-        reinterpret_cast<const float4*>(op), slot_of, static_cast<const uint4*>(shared_out),
-        static_cast<uint4*>(y), vecs, k);
-  } else if (dtype == MOE_DTYPE_BF16) {
-    combine_kernel<__nv_bfloat16><<<T, 256, 0, s>>>(op, slot_of,
-                                                    static_cast<const __nv_bfloat16*>(shared_out),
-                                                    static_cast<__nv_bfloat16*>(y), D, k);
-  } else {
-    combine_kernel<float><<<T, 256, 0, s>>>(op, slot_of, static_cast<const float*>(shared_out),
-                                            static_cast<float*>(y), D, k);
+  if (dtype == MOE_DTYPE_BF16) {
+    return shared_f32 ? combine_typed<__nv_bfloat16, float>(op, slot_of, shared_out, y, T, D, k, s)
+                      : combine_typed<__nv_bfloat16, __nv_bfloat16>(op, slot_of, shared_out, y, T, D, k, s);
   }
-  return cudaGetLastError();
+  return combine_typed<float, float>(op, slot_of, shared_out, y, T, D, k, s);
 }
 
 }  // namespace moe

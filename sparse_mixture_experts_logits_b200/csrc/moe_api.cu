@@ -138,7 +138,7 @@ SharedWs shared_layout(const moe_layer_desc_t* d) {
 
 struct FwdWs {
   moe_ws_layout_t pub;
-  size_t logits, wrT, chunk_counts, chunk_base, x_perm, h, h_sh;
+  size_t logits, wrT, chunk_counts, chunk_base, x_perm, h, h_sh, y_sh;
 };
 FwdWs forward_layout(const moe_layer_desc_t* d) {
   Carve c;
@@ -162,6 +162,7 @@ FwdWs forward_layout(const moe_layer_desc_t* d) {
   L.x_perm = c.take(d->dtype == MOE_DTYPE_BF16 ? pairs * d->D * 2 : 0);
   L.h = c.take(pairs * d->I * es);
   L.h_sh = c.take(static_cast<size_t>(d->T) * d->I_sh * es);
+  L.y_sh = c.take(d->I_sh > 0 ? static_cast<size_t>(d->T) * d->D * 4 : 0);
   L.pub.total = c.off;
   return L;
 }
@@ -285,11 +286,12 @@ moe_status_t run_experts(const moe_layer_desc_t* d, const moe_weights_t* w, cons
   return MOE_OK;
 }
 
-// Shared SwiGLU on all T tokens.  The down projection's epilogue adds
-// sum_j comb_src[slot_of[t, j]] (k_comb slots; 0 = none) to the accumulator.
+// Shared SwiGLU on all T tokens ([GLM45-SE] E_sh).  The down projection
+// writes `out` in fp32 when out_f32 (the forward pass adds it in the
+// combine), else in the layer's dtype.
 moe_status_t run_shared(const moe_layer_desc_t* d, const moe_weights_t* w, const void* x, void* out,
-                        void* h_sh, const void* comb_src, const int32_t* slot_of, int k_comb,
-                        int* status, cudaStream_t s, const Marks& mk = Marks()) {
+                        void* h_sh, bool out_f32, int* status, cudaStream_t s,
+                        const Marks& mk = Marks()) {
   if (d->dtype == MOE_DTYPE_BF16) {
     const int half = std::min(128, round_up(d->I_sh, 16));
     GemmLaunch g1{};
@@ -305,7 +307,7 @@ moe_status_t run_shared(const moe_layer_desc_t* d, const moe_weights_t* w, const
     MOE_CUDA(launch_gemm_sm100(g1, s));
     MOE_TRY(mk.at(6));
     GemmLaunch g2{};
-    g2.epi = EPI_COMBINE;
+    g2.epi = out_f32 ? EPI_STORE_F32 : EPI_COMBINE;  // EPI_COMBINE with k = 0: a plain bf16 store
     g2.A = h_sh; g2.a_rows = d->T;
     g2.B = w->sh_w2; g2.b_rows = d->D;
     g2.K = d->I_sh;
@@ -313,7 +315,7 @@ moe_status_t run_shared(const moe_layer_desc_t* d, const moe_weights_t* w, const
     g2.bn = std::min(256, round_up(d->D, 16)); g2.n_tiles = (d->D + g2.bn - 1) / g2.bn;
     g2.b_rows_per_group = d->D; g2.b_row_step = g2.bn; g2.b_hi_offset = g2.bn / 2;
     g2.out_cols = d->D; g2.out_col_step = g2.bn; g2.ldo = d->D; g2.out = out;
-    g2.comb_src = comb_src; g2.slot_of = slot_of; g2.k = k_comb;
+    g2.k = 0;
     g2.status = status;
     MOE_CUDA(launch_gemm_sm100(g2, s));
   } else {
@@ -327,15 +329,15 @@ moe_status_t run_shared(const moe_layer_desc_t* d, const moe_weights_t* w, const
     MOE_CUDA(launch_simt_gemm(g1, s));
     MOE_TRY(mk.at(6));
     SimtLaunch g2{};
-    g2.epi = EPI_COMBINE;
+    g2.epi = EPI_STORE_F32;
     g2.A = static_cast<const float*>(h_sh); g2.K = d->I_sh;
     g2.B = static_cast<const float*>(w->sh_w2);
     g2.num_groups = 1; g2.offsets = nullptr; g2.rows = d->T;
     g2.b_rows_per_group = d->D;
     g2.out_cols = d->D; g2.ldo = d->D; g2.out = static_cast<float*>(out);
-    g2.comb_src = static_cast<const float*>(comb_src); g2.slot_of = slot_of; g2.k = k_comb;
     MOE_CUDA(launch_simt_gemm(g2, s));
   }
+  MOE_TRY(mk.at(7));
   return MOE_OK;
 }
 
@@ -459,7 +461,7 @@ moe_status_t moe_shared_expert(const moe_layer_desc_t* d, const moe_weights_t* w
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* status = at<int*>(ws, L.status);
   MOE_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
-  return run_shared(d, w, x, y_sh, at<void*>(ws, L.h_sh), nullptr, nullptr, 0, status, s);
+  return run_shared(d, w, x, y_sh, at<void*>(ws, L.h_sh), false, status, s);
 }
 
 moe_status_t moe_combine(const moe_layer_desc_t* d, const void* out_perm, const int32_t* slot_of,
@@ -468,7 +470,7 @@ moe_status_t moe_combine(const moe_layer_desc_t* d, const void* out_perm, const 
   if (d->T == 0) return MOE_OK;
   if (!out_perm || !slot_of || !y) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_device());
-  MOE_CUDA(launch_combine(d->dtype, out_perm, slot_of, shared_out, y, d->T, d->D, d->k,
+  MOE_CUDA(launch_combine(d->dtype, out_perm, slot_of, shared_out, false, y, d->T, d->D, d->k,
                           static_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }
@@ -519,13 +521,16 @@ static moe_status_t forward_impl(const moe_layer_desc_t* d, const moe_weights_t*
   MOE_TRY(mk.at(2));
   MOE_TRY(run_experts(d, w, x, offsets, row_token, row_w, out_perm, at<void*>(ws, L.x_perm),
                       at<void*>(ws, L.h), status, s, mk));
+  void* y_sh = nullptr;
   if (d->I_sh > 0) {
-    MOE_TRY(run_shared(d, w, x, y, at<void*>(ws, L.h_sh), out_perm, slot_of, d->k, status, s, mk));
+    y_sh = at<void*>(ws, L.y_sh);
+    MOE_TRY(run_shared(d, w, x, y_sh, at<void*>(ws, L.h_sh), true, status, s, mk));
   } else {
     MOE_TRY(mk.at(6));
-    MOE_CUDA(launch_combine(d->dtype, out_perm, slot_of, nullptr, y, d->T, d->D, d->k, s));
+    MOE_TRY(mk.at(7));
   }
-  MOE_TRY(mk.at(7));
+  MOE_CUDA(launch_combine(d->dtype, out_perm, slot_of, y_sh, true, y, d->T, d->D, d->k, s));
+  MOE_TRY(mk.at(8));
   return MOE_OK;
 }
 
@@ -549,7 +554,7 @@ int moe_forward_launch_count(const moe_layer_desc_t* d) {
   int n = bf16 ? 3 : 2;   // [transpose,] logits, top-k
   n += 3;                 // histogram, scan, scatter
   n += bf16 ? 3 : 2;      // [gather,] first GEMM, second GEMM
-  n += d->I_sh > 0 ? 2 : 1;  // shared first GEMM + fused combine, or combine
+  n += d->I_sh > 0 ? 3 : 1;  // [shared first GEMM, shared second GEMM,] combine
   return n;
 }
 

@@ -43,6 +43,7 @@ enum GemmEpilogue : int {
   EPI_SCALE_BIAS = 3,  // out fp32 = (acc + b2[g, n]) * row_scale[r]   (second GEMM)
   EPI_COMBINE = 4,     // out bf16 = acc + sum_j src[slot_of[r, j], n] (shared down + combine,
                        //            src fp32)
+  EPI_STORE_BF16 = 5,  // out bf16 = acc                         (standalone shared down projection)
 };
 
 constexpr int kBK = 64;

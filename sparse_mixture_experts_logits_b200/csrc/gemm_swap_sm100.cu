@@ -1,0 +1,123 @@
+// Host side of the token-on-N grouped GEMM: tensor maps, grid, cluster launch.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <mutex>
+
+#include "gemm_swap_sm100.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// bf16 [rows, K] row-major, box = box_rows x 64, 128-byte swizzle; rows past the end read as zero.
+bool tmap_bf16(CUtensorMap* map, const void* base, long long rows, int K, int box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EPI>
+cudaError_t launch_swap_epi(const CUtensorMap& tw, const CUtensorMap& tx, const SwapArgs& args,
+                            long long tiles_ub, cudaStream_t s) {
+  static std::atomic<unsigned> configured{0};
+  static std::atomic<int> max_clusters[32];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  auto kernel = moe_gemm_swap_kernel<EPI>;
+  const unsigned bit = 1u << (dev & 31);
+  if (!(configured.load() & bit)) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSwDynSmem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t q = {};
+    q.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
+    q.blockDim = dim3(kGemmThreads, 1, 1);
+    q.dynamicSmemBytes = kSwDynSmem;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    q.attrs = at;
+    q.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &q) != cudaSuccess || clusters <= 0)
+      clusters = num_sms() / 2;
+    max_clusters[dev & 31].store(clusters);
+    configured.fetch_or(bit);
+  }
+  const long long units = std::min<long long>(max_clusters[dev & 31].load(), std::max<long long>(1, tiles_ub));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * units), 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSwDynSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, tw, tx, args);
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_swap(const SwapLaunch& L, cudaStream_t s) {
+  CUtensorMap tw, tx;
+  if (!tmap_bf16(&tw, L.W, L.w_rows, L.K, 64)) return cudaErrorInvalidValue;
+  if (!tmap_bf16(&tx, L.X, L.x_rows, L.K, 128)) return cudaErrorInvalidValue;
+  SwapArgs a;
+  a.num_groups = L.num_groups;
+  a.offsets = L.offsets;
+  a.rows = static_cast<int>(L.rows);
+  a.K = L.K;
+  a.w_rows_per_group = L.w_rows_per_group;
+  a.w_tiles = L.w_tiles;
+  a.w_tile_step = L.w_tile_step;
+  a.w_hi_offset = L.w_hi_offset;
+  a.w_cta_step = L.w_cta_step;
+  a.cols_per_tile = L.cols_per_tile;
+  a.out_cols = L.out_cols;
+  a.ldo = L.ldo;
+  a.out = L.out;
+  a.row_scale = L.row_scale;
+  a.bias = static_cast<const __nv_bfloat16*>(L.bias);
+  a.status = L.status;
+  // token tiles of a segment: ceil(rows_g / 256) at most, so the total is at most rows/256 + #groups
+  const long long tt_ub = L.offsets ? L.rows / kSwMaxTile + std::min<long long>(L.num_groups, L.rows)
+                                    : (L.rows + kSwMaxTile - 1) / kSwMaxTile;
+  const long long tiles_ub = tt_ub * L.w_tiles;
+  switch (L.epi) {
+    case EPI_GELU_BIAS: return launch_swap_epi<EPI_GELU_BIAS>(tw, tx, a, tiles_ub, s);
+    case EPI_SWIGLU: return launch_swap_epi<EPI_SWIGLU>(tw, tx, a, tiles_ub, s);
+    case EPI_SCALE_BIAS: return launch_swap_epi<EPI_SCALE_BIAS>(tw, tx, a, tiles_ub, s);
+    case EPI_STORE_F32: return launch_swap_epi<EPI_STORE_F32>(tw, tx, a, tiles_ub, s);
+    case EPI_STORE_BF16: return launch_swap_epi<EPI_STORE_BF16>(tw, tx, a, tiles_ub, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

@@ -1,0 +1,344 @@
+// Grouped GEMM with the tokens on the MMA's N side ("swap-AB"), on CTA pairs
+// (tcgen05.mma.cta_group::2, M = 256 weight rows, N = 16..256 tokens).
+//
+//   out[r, n] = epilogue( sum_k W[g*w_rows + n', k] * X[r, k] )
+//
+// for every dispatch row r of group g's segment offsets[g] .. offsets[g+1]
+// and every output column n.  W is a bf16 stack of per-group [rows, K]
+// weight blocks (nn.Linear layout, K-major) and is the MMA's A operand;
+// the token rows X[r] (dispatch order: x gathered per expert, or h) are the
+// B operand.  Each CTA loads one 128-row TMA box of token rows per stage and
+// the MMA reads the first N/2 of them.  (Loading the rows by index with
+// tile::gather4 instead, 4 rows per TMA instruction, measured 2-3x slower:
+// the TMA instruction rate, not the bytes, became the limit.)
+//
+// Why tokens on N: an expert's segment is cut into token tiles of at most
+// 256 rows whose width N is rounded up only to a multiple of 16, so the
+// padding per segment is at most 15 rows (instead of up to 255 with 256-row
+// M tiles); and in the accumulator a TMEM lane is an output column, so each
+// token's 32 (or 64) output columns leave a warp as one contiguous store.
+//
+// Per CTA pair and tile: 256 weight rows (128 staged by each CTA: two 64-row
+// TMA boxes) x N tokens (N/2 staged by each CTA).  SwiGLU tiles stage 64 gate
+// and the matching 64 up rows in each CTA, so gate and up of one output
+// column sit in TMEM lanes m and m + 64 of the same CTA; the epilogue warps
+// of the up lanes hand their values to the gate lanes through shared memory.
+//
+// Warp roles (320 threads per CTA): warp 0 TMA producer, warp 1 TMEM
+// allocator and (first CTA) MMA issuer, warps 2..9 epilogue.  Every wait is bounded (kWaitTimeoutNs) and reports
+// MOE_DEVERR_TIMEOUT through the status word instead of hanging.
+#pragma once
+
+#include "gemm_sm100.cuh"
+
+namespace moe {
+
+constexpr int kSwStages = 6;
+constexpr int kSwATileBytes = 128 * kBK * 2;  // 128 weight rows per CTA
+constexpr int kSwBTileBytes = 128 * kBK * 2;  // up to 128 token rows per CTA
+constexpr int kSwStageBytes = kSwATileBytes + kSwBTileBytes;
+constexpr int kSwXPitch = 33;                 // floats per row of the gate/up hand-off buffer
+constexpr int kSwXBytes = 4 * 32 * kSwXPitch * 4;
+constexpr int kSwDynSmem = kSwStages * kSwStageBytes + kSwXBytes + 1024;
+constexpr int kSwMaxTile = 256;               // tokens per tile
+
+struct SwapArgs {
+  int num_groups;
+  const int* offsets;      // [G + 1] or nullptr: one group [0, rows)
+  int rows;
+  int K;
+  int w_rows_per_group;    // weight rows of one group
+  int w_tiles;             // weight tiles per group
+  int w_tile_step;         // weight-row advance per weight tile (256; SwiGLU 128)
+  int w_hi_offset;         // row offset of a CTA's second 64-row box (64; SwiGLU: I, the up block)
+  int w_cta_step;          // row offset of the second CTA's boxes (128; SwiGLU 64)
+  int cols_per_tile;       // output columns of one weight tile (256; SwiGLU 128)
+  int out_cols;            // valid output columns
+  int ldo;
+  void* out;
+  const float* row_scale;      // EPI_SCALE_BIAS: [rows]
+  const __nv_bfloat16* bias;   // EPI_GELU_BIAS / EPI_SCALE_BIAS: [G, out_cols] or nullptr
+  int* status;
+};
+
+// Token tiles of a segment of `cnt` rows: ceil(cnt / 256) tiles of equal
+// width rounded up to 16, then as many as that width needs.
+__device__ __forceinline__ void token_tiling(int cnt, int& width, int& ntiles) {
+  if (cnt <= 0) { width = 16; ntiles = 0; return; }
+  const int n0 = (cnt + kSwMaxTile - 1) / kSwMaxTile;
+  width = (((cnt + n0 - 1) / n0) + 15) & ~15;
+  ntiles = (cnt + width - 1) / width;
+}
+
+struct SwapTile {
+  int g, wt, tok0, nrows, n;  // group, weight tile, first token, rows, MMA N
+};
+
+__device__ __forceinline__ SwapTile swap_decode(int tile, int G, const int* s_tstart, const int* s_off,
+                                                int w_tiles) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_tstart[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  SwapTile t;
+  t.g = lo;
+  const int cnt = s_off[lo + 1] - s_off[lo];
+  int width, ntt;
+  token_tiling(cnt, width, ntt);
+  const int local = tile - s_tstart[lo];
+  const int band = local / (kBandM * w_tiles);
+  const int rem = local - band * kBandM * w_tiles;
+  const int bt = min(kBandM, ntt - band * kBandM);
+  t.wt = rem / bt;
+  const int tt = band * kBandM + (rem - t.wt * bt);
+  t.tok0 = tt * width;
+  t.nrows = min(width, cnt - t.tok0);
+  t.n = (t.nrows + 15) & ~15;
+  return t;
+}
+
+// Stores of one token's value for this lane's output column: the warp's 32
+// lanes cover 32 consecutive columns, i.e. one contiguous row segment.
+template <int EPI>
+__device__ __forceinline__ void swap_store(const SwapArgs& a, size_t row, int col, float v) {
+  if constexpr (EPI == EPI_SCALE_BIAS || EPI == EPI_STORE_F32)
+    static_cast<float*>(a.out)[row * a.ldo + col] = v;
+  else
+    static_cast<__nv_bfloat16*>(a.out)[row * a.ldo + col] = __float2bfloat16_rn(v);
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    moe_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmap_w,
+                         const __grid_constant__ CUtensorMap tmap_x, const SwapArgs args) {
+  constexpr int S = kSwStages;
+  constexpr bool kSwiglu = EPI == EPI_SWIGLU;
+  extern __shared__ uint8_t dyn_smem[];
+  __shared__ int s_off[kMaxExperts + 1];
+  __shared__ int s_tstart[kMaxExperts + 1];
+  __shared__ __align__(8) uint64_t s_full[S];
+  __shared__ __align__(8) uint64_t s_empty[S];
+  __shared__ __align__(8) uint64_t s_tfull[2];
+  __shared__ __align__(8) uint64_t s_tempty[2];
+  __shared__ __align__(8) uint64_t s_xfull[4];
+  __shared__ __align__(8) uint64_t s_xempty[4];
+  __shared__ __align__(8) uint64_t s_drain;
+  __shared__ uint32_t s_tmem_base;
+  __shared__ int s_abort;
+  __shared__ int s_total;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int unit = static_cast<int>(blockIdx.x >> 1);
+  const int units = static_cast<int>(gridDim.x >> 1);
+  const uint32_t smem_base = (smem_addr(dyn_smem) + 1023u) & ~1023u;
+  float* xbuf = reinterpret_cast<float*>(dyn_smem + (smem_base - smem_addr(dyn_smem)) + S * kSwStageBytes);
+  const int G = args.num_groups;
+
+  for (int i = threadIdx.x; i <= G; i += blockDim.x)
+    s_off[i] = args.offsets != nullptr ? args.offsets[i] : (i == 0 ? 0 : args.rows);
+  __syncthreads();
+  if (warp == 0) {
+    int carry = 0;
+    for (int base = 0; base < G; base += 32) {
+      const int g = base + lane;
+      int v = 0;
+      if (g < G) {
+        int width, ntt;
+        token_tiling(s_off[g + 1] - s_off[g], width, ntt);
+        v = ntt * args.w_tiles;
+      }
+      int incl = v;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += t;
+      }
+      if (g < G) s_tstart[g] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      s_tstart[G] = carry;
+      s_total = carry;
+      s_abort = 0;
+      for (int s = 0; s < S; ++s) {
+        mbar_init(smem_addr(&s_full[s]), 1);
+        mbar_init(smem_addr(&s_empty[s]), 1);
+      }
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(smem_addr(&s_tfull[b]), 1);
+        mbar_init(smem_addr(&s_tempty[b]), kEpiWarps * 32 * 2);
+      }
+      for (int x = 0; x < 4; ++x) {
+        mbar_init(smem_addr(&s_xfull[x]), 32);
+        mbar_init(smem_addr(&s_xempty[x]), 32);
+      }
+      mbar_init(smem_addr(&s_drain), 1);
+      fence_mbar_init();
+      tma_prefetch_desc(&tmap_w);
+      tma_prefetch_desc(&tmap_x);
+    }
+  } else if (warp == 1) {
+    tmem_alloc_pair(smem_addr(&s_tmem_base), 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  tc_fence_after();
+
+  const uint32_t tmem_base = s_tmem_base;
+  const int total = s_total;
+  const int num_kb = (args.K + kBK - 1) / kBK;
+  volatile int* abort_flag = &s_abort;
+
+  if (warp == 0) {
+    // -------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      uint32_t kiter = 0;
+      bool ok = true;
+      constexpr uint32_t tx_bytes = 2u * kSwStageBytes;  // both CTAs: weight rows + 128 token rows
+      for (int tile = unit; ok && tile < total; tile += units) {
+        const SwapTile t = swap_decode(tile, G, s_tstart, s_off, args.w_tiles);
+        const int x_row = s_off[t.g] + t.tok0 + static_cast<int>(rank) * (t.n >> 1);
+        const int w_base = t.g * args.w_rows_per_group + t.wt * args.w_tile_step +
+                           static_cast<int>(rank) * args.w_cta_step;
+        for (int kb = 0; kb < num_kb; ++kb, ++kiter) {
+          const int s = kiter % S;
+          const uint32_t ph = (kiter / S) & 1u;
+          if (!mbar_wait(smem_addr(&s_empty[s]), ph ^ 1u, abort_flag, args.status)) { ok = false; break; }
+          const uint32_t sa = smem_base + s * kSwStageBytes;
+          const uint32_t sb = sa + kSwATileBytes;
+          const uint32_t full_leader = mapa_shared(smem_addr(&s_full[s]), 0);
+          if (leader) mbar_arrive_expect_tx(smem_addr(&s_full[s]), tx_bytes);
+          tma_load_2d_pair(sa, &tmap_w, full_leader, kb * kBK, w_base);
+          tma_load_2d_pair(sa + 64 * kBK * 2, &tmap_w, full_leader, kb * kBK, w_base + args.w_hi_offset);
+          tma_load_2d_pair(sb, &tmap_x, full_leader, kb * kBK, x_row);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // -------------------------------------------------------- MMA issuer
+      uint32_t kiter = 0, it = 0;
+      bool ok = true;
+      for (int tile = unit; ok && tile < total; tile += units, ++it) {
+        const SwapTile t = swap_decode(tile, G, s_tstart, s_off, args.w_tiles);
+        const uint32_t idesc = umma_idesc_bf16(256, t.n);
+        const uint32_t buf = it & 1u;
+        const uint32_t tph = (it >> 1) & 1u;
+        if (!mbar_wait(smem_addr(&s_tempty[buf]), tph ^ 1u, abort_flag, args.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * 256u;
+        for (int kb = 0; kb < num_kb; ++kb, ++kiter) {
+          const int s = kiter % S;
+          const uint32_t ph = (kiter / S) & 1u;
+          if (!mbar_wait(smem_addr(&s_full[s]), ph, abort_flag, args.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_base + s * kSwStageBytes;
+          const uint32_t sb = sa + kSwATileBytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            umma_bf16_pair(d_tmem, sw128_kmajor_desc(sa + kk * 32), sw128_kmajor_desc(sb + kk * 32), idesc,
+                           (kb | kk) != 0 ? 1u : 0u);
+          umma_commit_pair(smem_addr(&s_empty[s]), 0x3);
+        }
+        if (!ok) break;
+        umma_commit_pair(smem_addr(&s_tfull[buf]), 0x3);
+      }
+      umma_commit_pair(smem_addr(&s_drain), 0x1);
+      mbar_wait_drain(smem_addr(&s_drain), 0, kWaitTimeoutNs);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;           // TMEM lane quarter
+    const int part = (warp - 2) >> 2; // token chunks part, part + 2, ...
+    const int m = q * 32 + lane;      // accumulator lane = weight row inside this CTA
+    const uint32_t tempty0 = mapa_shared(smem_addr(&s_tempty[0]), 0);
+    const uint32_t tempty1 = mapa_shared(smem_addr(&s_tempty[1]), 0);
+    const int pair = part * 2 + (q & 1);          // SwiGLU hand-off pair (gate q, up q + 2)
+    float* xs = xbuf + pair * 32 * kSwXPitch;
+    const bool up_warp = kSwiglu && q >= 2;
+    uint32_t it = 0, xc = 0;
+    bool ok = true;
+    for (int tile = unit; ok && tile < total; tile += units, ++it) {
+      const SwapTile t = swap_decode(tile, G, s_tstart, s_off, args.w_tiles);
+      const uint32_t buf = it & 1u;
+      const uint32_t tph = (it >> 1) & 1u;
+      if (!mbar_wait(smem_addr(&s_tfull[buf]), tph, abort_flag, args.status)) break;
+      tc_fence_after();
+      const int col = kSwiglu ? t.wt * args.cols_per_tile + static_cast<int>(rank) * 64 + (m & 63)
+                              : t.wt * args.cols_per_tile + static_cast<int>(rank) * 128 + m;
+      const bool col_ok = col < args.out_cols;
+      float bias = 0.f;
+      if constexpr (EPI == EPI_GELU_BIAS || EPI == EPI_SCALE_BIAS) {
+        if (args.bias != nullptr && col_ok)
+          bias = __bfloat162float(args.bias[static_cast<size_t>(t.g) * args.out_cols + col]);
+      }
+      const size_t row0 = static_cast<size_t>(s_off[t.g]) + t.tok0;
+      const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * 256u;
+      for (int c = 32 * part; c < t.n; c += 64) {
+        uint32_t r[32];
+        MOE_TMEM_LD32(tacc + c, r);
+        tmem_ld_wait();
+        const int nv = min(32, t.nrows - c);  // tokens of this chunk that exist
+        if constexpr (kSwiglu) {
+          if (up_warp) {
+            if (!mbar_wait(smem_addr(&s_xempty[pair]), (xc & 1u) ^ 1u, abort_flag, args.status)) { ok = false; break; }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) xs[lane * kSwXPitch + i] = __uint_as_float(r[i]);
+            mbar_arrive(smem_addr(&s_xfull[pair]));
+          } else {
+            if (!mbar_wait(smem_addr(&s_xfull[pair]), xc & 1u, abort_flag, args.status)) { ok = false; break; }
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = silu_fast(__uint_as_float(r[i])) * xs[lane * kSwXPitch + i];
+            mbar_arrive(smem_addr(&s_xempty[pair]));
+            if (col_ok) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (i < nv) swap_store<EPI>(args, row0 + c + i, col, v[i]);
+            }
+          }
+          ++xc;
+        } else {
+          float rs = 1.f;
+          if constexpr (EPI == EPI_SCALE_BIAS) {
+            if (lane < nv) rs = args.row_scale[row0 + c + lane];
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            float v = __uint_as_float(r[i]) + bias;
+            if constexpr (EPI == EPI_GELU_BIAS) v = gelu_tanh_fast(v);
+            if constexpr (EPI == EPI_SCALE_BIAS) v *= __shfl_sync(0xffffffffu, rs, i);
+            if (col_ok && i < nv) swap_store<EPI>(args, row0 + c + i, col, v);
+          }
+        }
+      }
+      if (!ok) break;
+      tc_fence_before();
+      mbar_arrive_remote(buf ? tempty1 : tempty0);
+    }
+  }
+
+  __syncthreads();
+  if (s_abort && warp == 0 && lane == 0) {
+    // let TMA loads still in flight land before shared memory is released
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 200000ull) {
+    }
+  }
+  __syncthreads();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, 512);
+  }
+}
+
+}  // namespace moe

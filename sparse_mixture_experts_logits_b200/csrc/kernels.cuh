@@ -53,6 +53,25 @@ struct GemmLaunch {
 cudaError_t launch_gemm_sm100(const GemmLaunch& L, cudaStream_t s);
 int num_sms();
 
+// gemm_swap_sm100.cu: grouped bf16 GEMM with the token rows on the MMA's N
+// side (see gemm_swap_sm100.cuh).  `epi` is a GemmEpilogue.
+struct SwapLaunch {
+  int epi;
+  const void* W; long long w_rows;  // bf16 [w_rows, K] weight stack
+  const void* X; long long x_rows;  // bf16 [x_rows, K] token rows in dispatch order
+  int K;
+  int num_groups;
+  const int* offsets;        // device [G+1] or nullptr (single group of `rows` rows)
+  long long rows;            // dispatch rows (upper bound when grouped)
+  int w_rows_per_group, w_tiles, w_tile_step, w_hi_offset, w_cta_step, cols_per_tile;
+  int out_cols, ldo;
+  void* out;
+  const float* row_scale;
+  const void* bias;
+  int* status;
+};
+cudaError_t launch_gemm_swap(const SwapLaunch& L, cudaStream_t s);
+
 // simt.cu: fp32 grouped GEMM with the same epilogues (fp32 dtype path).
 struct SimtLaunch {
   int epi;

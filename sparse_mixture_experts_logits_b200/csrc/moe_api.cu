@@ -221,44 +221,39 @@ moe_status_t run_experts(const moe_layer_desc_t* d, const moe_weights_t* w, cons
   if (d->dtype == MOE_DTYPE_BF16) {
     MOE_CUDA(launch_gather_rows(x, row_token, x_perm, pairs, d->D, 2, s));
     MOE_TRY(mk.at(3));
-    GemmLaunch g1{};
-    g1.A = x_perm; g1.a_rows = pairs;
-    g1.B = w->w1; g1.b_rows = static_cast<long long>(d->M) * n1;
+    SwapLaunch g1{};
+    g1.W = w->w1; g1.w_rows = static_cast<long long>(d->M) * n1;
+    g1.X = x_perm; g1.x_rows = pairs;
     g1.K = d->D;
-    g1.num_groups = d->M; g1.offsets = offsets; g1.rows_upper = pairs;
+    g1.num_groups = d->M; g1.offsets = offsets; g1.rows = pairs;
     if (swiglu) {
-      const int half = std::min(128, round_up(d->I, 16));
       g1.epi = EPI_SWIGLU;
-      g1.bn = 2 * half;
-      g1.n_tiles = (d->I + half - 1) / half;
-      g1.b_rows_per_group = n1; g1.b_row_step = half; g1.b_hi_offset = d->I;
-      g1.out_col_step = half;
+      g1.w_rows_per_group = n1; g1.w_tile_step = 128; g1.w_hi_offset = d->I; g1.w_cta_step = 64;
+      g1.cols_per_tile = 128;
     } else {
       g1.epi = EPI_GELU_BIAS;
-      g1.bn = std::min(256, round_up(d->I, 16));
-      g1.n_tiles = (d->I + g1.bn - 1) / g1.bn;
-      g1.b_rows_per_group = n1; g1.b_row_step = g1.bn; g1.b_hi_offset = g1.bn / 2;
-      g1.out_col_step = g1.bn;
+      g1.w_rows_per_group = n1; g1.w_tile_step = 256; g1.w_hi_offset = 64; g1.w_cta_step = 128;
+      g1.cols_per_tile = 256;
       g1.bias = b1;
     }
+    g1.w_tiles = (d->I + g1.cols_per_tile - 1) / g1.cols_per_tile;
     g1.out_cols = d->I; g1.ldo = d->I; g1.out = h;
     g1.status = status;
-    MOE_CUDA(launch_gemm_sm100(g1, s));
+    MOE_CUDA(launch_gemm_swap(g1, s));
     MOE_TRY(mk.at(4));
 
-    GemmLaunch g2{};
+    SwapLaunch g2{};
     g2.epi = EPI_SCALE_BIAS;
-    g2.A = h; g2.a_rows = pairs;
-    g2.B = w->w2; g2.b_rows = static_cast<long long>(d->M) * d->D;
+    g2.W = w->w2; g2.w_rows = static_cast<long long>(d->M) * d->D;
+    g2.X = h; g2.x_rows = pairs;
     g2.K = d->I;
-    g2.num_groups = d->M; g2.offsets = offsets; g2.rows_upper = pairs;
-    g2.bn = std::min(256, round_up(d->D, 16));
-    g2.n_tiles = (d->D + g2.bn - 1) / g2.bn;
-    g2.b_rows_per_group = d->D; g2.b_row_step = g2.bn; g2.b_hi_offset = g2.bn / 2;
-    g2.out_cols = d->D; g2.out_col_step = g2.bn; g2.ldo = d->D;
-    g2.out = out_perm; g2.row_scale = row_w; g2.bias = b2;
+    g2.num_groups = d->M; g2.offsets = offsets; g2.rows = pairs;
+    g2.w_rows_per_group = d->D; g2.w_tile_step = 256; g2.w_hi_offset = 64; g2.w_cta_step = 128;
+    g2.cols_per_tile = 256; g2.w_tiles = (d->D + 255) / 256;
+    g2.out_cols = d->D; g2.ldo = d->D; g2.out = out_perm;
+    g2.row_scale = row_w; g2.bias = b2;
     g2.status = status;
-    MOE_CUDA(launch_gemm_sm100(g2, s));
+    MOE_CUDA(launch_gemm_swap(g2, s));
     MOE_TRY(mk.at(5));
   } else {
     MOE_TRY(mk.at(3));
@@ -293,31 +288,29 @@ moe_status_t run_shared(const moe_layer_desc_t* d, const moe_weights_t* w, const
                         void* h_sh, bool out_f32, int* status, cudaStream_t s,
                         const Marks& mk = Marks()) {
   if (d->dtype == MOE_DTYPE_BF16) {
-    const int half = std::min(128, round_up(d->I_sh, 16));
-    GemmLaunch g1{};
+    SwapLaunch g1{};
     g1.epi = EPI_SWIGLU;
-    g1.A = x; g1.a_rows = d->T;
-    g1.B = w->sh_w1; g1.b_rows = 2ll * d->I_sh;
+    g1.W = w->sh_w1; g1.w_rows = 2ll * d->I_sh;
+    g1.X = x; g1.x_rows = d->T;
     g1.K = d->D;
-    g1.num_groups = 1; g1.offsets = nullptr; g1.rows_upper = d->T;
-    g1.bn = 2 * half; g1.n_tiles = (d->I_sh + half - 1) / half;
-    g1.b_rows_per_group = 2 * d->I_sh; g1.b_row_step = half; g1.b_hi_offset = d->I_sh;
-    g1.out_cols = d->I_sh; g1.out_col_step = half; g1.ldo = d->I_sh; g1.out = h_sh;
+    g1.num_groups = 1; g1.offsets = nullptr; g1.rows = d->T;
+    g1.w_rows_per_group = 2 * d->I_sh; g1.w_tile_step = 128; g1.w_hi_offset = d->I_sh; g1.w_cta_step = 64;
+    g1.cols_per_tile = 128; g1.w_tiles = (d->I_sh + 127) / 128;
+    g1.out_cols = d->I_sh; g1.ldo = d->I_sh; g1.out = h_sh;
     g1.status = status;
-    MOE_CUDA(launch_gemm_sm100(g1, s));
+    MOE_CUDA(launch_gemm_swap(g1, s));
     MOE_TRY(mk.at(6));
-    GemmLaunch g2{};
-    g2.epi = out_f32 ? EPI_STORE_F32 : EPI_COMBINE;  // EPI_COMBINE with k = 0: a plain bf16 store
-    g2.A = h_sh; g2.a_rows = d->T;
-    g2.B = w->sh_w2; g2.b_rows = d->D;
+    SwapLaunch g2{};
+    g2.epi = out_f32 ? EPI_STORE_F32 : EPI_STORE_BF16;
+    g2.W = w->sh_w2; g2.w_rows = d->D;
+    g2.X = h_sh; g2.x_rows = d->T;
     g2.K = d->I_sh;
-    g2.num_groups = 1; g2.offsets = nullptr; g2.rows_upper = d->T;
-    g2.bn = std::min(256, round_up(d->D, 16)); g2.n_tiles = (d->D + g2.bn - 1) / g2.bn;
-    g2.b_rows_per_group = d->D; g2.b_row_step = g2.bn; g2.b_hi_offset = g2.bn / 2;
-    g2.out_cols = d->D; g2.out_col_step = g2.bn; g2.ldo = d->D; g2.out = out;
-    g2.k = 0;
+    g2.num_groups = 1; g2.offsets = nullptr; g2.rows = d->T;
+    g2.w_rows_per_group = d->D; g2.w_tile_step = 256; g2.w_hi_offset = 64; g2.w_cta_step = 128;
+    g2.cols_per_tile = 256; g2.w_tiles = (d->D + 255) / 256;
+    g2.out_cols = d->D; g2.ldo = d->D; g2.out = out;
     g2.status = status;
-    MOE_CUDA(launch_gemm_sm100(g2, s));
+    MOE_CUDA(launch_gemm_swap(g2, s));
   } else {
     SimtLaunch g1{};
     g1.epi = EPI_SWIGLU;

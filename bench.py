@@ -331,19 +331,26 @@ def run_ours(args):
     dom = max(gemm_stages, key=lambda s: stage_ms[s])
     f, b = work[dom]
     t_s = stage_ms[dom] / 1e3
-    peak_tf = peaks["bf16_tflops"]
+    # The GEMMs are timed inside a long run of back-to-back steps, which settles
+    # at the board power cap: the sustained tensor figure is the denominator
+    # (the burst figure is reported beside it).
+    peak_tf = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    peak_tf_burst = peaks["bf16_tflops"]
     peak_bw = peaks["hbm_gbs"]
     t_f, t_b = f / (peak_tf * 1e12), b / (peak_bw * 1e9)
     if t_f >= t_b:
         roof = {"bound": "tensor", "achieved": f / t_s / 1e12, "peak": peak_tf, "unit": "TFLOP/s"}
+        roof["frac_of_burst_peak"] = roof["achieved"] / peak_tf_burst
     else:
         roof = {"bound": "hbm", "achieved": b / t_s / 1e9, "peak": peak_bw, "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = recorded_traffic(dom, args.config)
-    roof["kernel"] = f"moe_gemm_sm100_kernel ({dom})"
-    roof["peak_source"] = f"{peak_src} ({'burst' if peak_src == 'measured' else 'fallback'} figure)"
+    roof["kernel"] = f"moe_gemm_swap_kernel ({dom})"
+    roof["peak_source"] = (f"{peak_src}: " + ("bf16_tflops_sustained (kernel timed inside a long loop)"
+                                             if roof["bound"] == "tensor" else "hbm_gbs"))
     roof["algorithmic"] = {"flops": f, "bytes": b}
     t_layer_ideal = max(flops_total / (peak_tf * 1e12), bytes_total / (peak_bw * 1e9))
+    t_layer_ideal_burst = max(flops_total / (peak_tf_burst * 1e12), bytes_total / (peak_bw * 1e9))
 
     out = {
         "metric": METRIC,
@@ -366,7 +373,8 @@ def run_ours(args):
         "roofline": roof,
         "layer": {"tflops": flops_total / (ms_step / 1e3) / 1e12,
                   "algorithmic_flops": flops_total, "algorithmic_bytes": bytes_total,
-                  "ideal_ms": t_layer_ideal * 1e3, "frac_of_ideal": t_layer_ideal / (ms_step / 1e3)},
+                  "ideal_ms": t_layer_ideal * 1e3, "frac_of_ideal": t_layer_ideal / (ms_step / 1e3),
+                  "frac_of_ideal_burst": t_layer_ideal_burst / (ms_step / 1e3)},
         "stages_ms": stage_ms,
         "e2e": e2e,
         "gpu_launches": B.moe_forward_launch_count(layer.desc) * K,

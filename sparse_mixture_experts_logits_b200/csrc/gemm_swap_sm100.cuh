@@ -238,7 +238,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int s = kiter % S;
           const uint32_t ph = (kiter / S) & 1u;
           if (!mbar_wait(smem_addr(&s_full[s]), ph, abort_flag, args.status)) { ok = false; break; }
-          tc_fence_after();
           const uint32_t sa = smem_base + s * kSwStageBytes;
           const uint32_t sb = sa + kSwATileBytes;
 #pragma unroll

@@ -10,6 +10,11 @@ namespace moe {
 cudaError_t launch_transpose_bf16(const void* src, void* dst, int rows, int cols, cudaStream_t s);
 cudaError_t launch_logits_f32(const float* x, const float* w_r, float* logits, int T, int D, int M,
                               cudaStream_t s);
+// Small-T bf16 router: route_splits(T, D, dtype) partial logit sums
+// [nsplit][T][M] (written to `partial`), added in order into `logits`.
+int route_splits(int T, int D, int dtype);
+cudaError_t launch_logits_splitk_bf16(const void* x, const void* w_r, float* partial, float* logits, int T,
+                                      int D, int M, cudaStream_t s);
 cudaError_t launch_topk(const float* logits, const float* e_bias, int T, int M, int k, int gate,
                         int norm, float alpha, float eps, int32_t* idx, float* w, cudaStream_t s);
 

@@ -41,8 +41,8 @@ cudaError_t launch_gather_rows(const void* x, const int32_t* row_token, void* x_
 
 // y[t, :] = sum_j out_perm[slot_of[t, j], :] (+ shared[t, :]) in fp32, in
 // slot order, rounded once.  out_perm is fp32; shared is fp32 or the layer's
-// type; y has the layer's type.  One block per token; every row read is
-// contiguous, and the k rows of a token are loaded together.
+// type; y has the layer's type.  Block (token, 128 four-column groups); every
+// row read is contiguous, and the k rows of a token are loaded together.
 template <typename TY, typename TS>
 __global__ void __launch_bounds__(128) combine_vec4_kernel(const float4* __restrict__ out_perm,
                                                            const int32_t* __restrict__ slot_of,
@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(128) combine_vec4_kernel(const float4* __restr
   const int t = blockIdx.x;
   if (threadIdx.x < k) s_slot[threadIdx.x] = slot_of[static_cast<size_t>(t) * k + threadIdx.x];
   __syncthreads();
-  for (int v = threadIdx.x; v < D4; v += blockDim.x) {
+  for (int v = blockIdx.y * blockDim.x + threadIdx.x; v < D4; v += blockDim.x * gridDim.y) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 8
     for (int j = 0; j < k; ++j) {
@@ -97,7 +97,9 @@ template <typename TY, typename TS>
 static cudaError_t combine_typed(const float* op, const int32_t* slot_of, const void* shared, void* y,
                                  int T, int D, int k, cudaStream_t s) {
   if (D % 4 == 0) {
-    combine_vec4_kernel<TY, TS><<<T, 128, 0, s>>>(reinterpret_cast<const float4*>(op), slot_of,
+    // few tokens: spread a row's columns over blocks too
+    dim3 grid(T, T >= 1024 ? 1 : (D / 4 + 127) / 128);
+    combine_vec4_kernel<TY, TS><<<grid, 128, 0, s>>>(reinterpret_cast<const float4*>(op), slot_of,
                                                   static_cast<const TS*>(shared), static_cast<TY*>(y), D / 4, k);
   } else {
     combine_kernel<TY, TS><<<T, 128, 0, s>>>(op, slot_of, static_cast<const TS*>(shared),

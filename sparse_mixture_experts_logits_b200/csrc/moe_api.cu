@@ -91,12 +91,18 @@ moe_status_t check_weights(const moe_layer_desc_t* d, const moe_weights_t* w, bo
 }
 
 // ---------------------------------------------------------------- layouts
+// fp32 [T, M] logits, followed on the small-T path by the split partials.
+inline int route_layout_splits(int T, int D, int dtype) {
+  const int n = route_splits(T, D, dtype);
+  return n > 1 ? n + 1 : 1;
+}
+
 struct RouteWs { size_t status, logits, wrT, total; };
 RouteWs route_layout(int T, int D, int M, int dtype) {
   Carve c;
   RouteWs L;
   L.status = c.take(4);
-  L.logits = c.take(static_cast<size_t>(T) * M * 4);
+  L.logits = c.take(static_cast<size_t>(route_layout_splits(T, D, dtype)) * T * M * 4);
   L.wrT = c.take(dtype == MOE_DTYPE_BF16 ? static_cast<size_t>(M) * D * 2 : 0);
   L.total = c.off;
   return L;
@@ -154,7 +160,7 @@ FwdWs forward_layout(const moe_layer_desc_t* d) {
   L.pub.row_token = c.take(pairs * 4);
   L.pub.row_w = c.take(pairs * 4);
   L.pub.out_perm = c.take(pairs * d->D * 4);
-  L.logits = c.take(static_cast<size_t>(d->T) * d->M * 4);
+  L.logits = c.take(static_cast<size_t>(route_layout_splits(d->T, d->D, d->dtype)) * d->T * d->M * 4);
   L.wrT = c.take(d->dtype == MOE_DTYPE_BF16 ? static_cast<size_t>(d->M) * d->D * 2 : 0);
   const size_t nch = static_cast<size_t>(d->M) * perm_num_chunks(static_cast<long long>(pairs));
   L.chunk_counts = c.take(nch * 4);
@@ -185,7 +191,12 @@ struct Marks {
 moe_status_t run_route(const void* x, const void* w_r, const float* e_bias, int T, int D, int M, int k,
                        int dtype, int gate, int norm, float alpha, float eps, int32_t* idx, float* w,
                        float* logits, void* wrT, int* status, cudaStream_t s) {
-  if (dtype == MOE_DTYPE_BF16) {
+  const int nsplit = route_splits(T, D, dtype);
+  if (dtype == MOE_DTYPE_BF16 && nsplit > 1) {
+    // few tokens: split-K SIMT logits (no transpose, no tensor-core launch)
+    float* partial = logits + static_cast<size_t>(T) * M;
+    MOE_CUDA(launch_logits_splitk_bf16(x, w_r, partial, logits, T, D, M, s));
+  } else if (dtype == MOE_DTYPE_BF16) {
     MOE_CUDA(launch_transpose_bf16(w_r, wrT, D, M, s));
     GemmLaunch L{};
     L.epi = EPI_STORE_F32;
@@ -204,8 +215,8 @@ moe_status_t run_route(const void* x, const void* w_r, const float* e_bias, int 
     MOE_CUDA(launch_logits_f32(static_cast<const float*>(x), static_cast<const float*>(w_r), logits, T,
                                D, M, s));
   }
-  MOE_CUDA(launch_topk(logits, gate == MOE_GATE_SIGMOID_BIAS ? e_bias : nullptr, T, M, k, gate, norm,
-                       alpha, eps, idx, w, s));
+  MOE_CUDA(launch_topk(logits, gate == MOE_GATE_SIGMOID_BIAS ? e_bias : nullptr, T, M, k, gate,
+                       norm, alpha, eps, idx, w, s));
   return MOE_OK;
 }
 
@@ -544,8 +555,8 @@ moe_status_t moe_forward_profiled(const moe_layer_desc_t* d, const moe_weights_t
 int moe_forward_launch_count(const moe_layer_desc_t* d) {
   if (check_desc(d) != MOE_OK || d->T == 0) return 0;
   const bool bf16 = d->dtype == MOE_DTYPE_BF16;
-  int n = bf16 ? 3 : 2;   // [transpose,] logits, top-k
-  n += 3;                 // histogram, scan, scatter
+  int n = bf16 ? 3 : 2;  // transpose + logits GEMM or split-K logits + reduction; top-k
+  n += static_cast<long long>(d->T) * d->k <= 2048 ? 1 : 3;          // counting sort (1 or 3 kernels)
   n += bf16 ? 3 : 2;      // [gather,] first GEMM, second GEMM
   n += d->I_sh > 0 ? 3 : 1;  // [shared first GEMM, shared second GEMM,] combine
   return n;

@@ -136,11 +136,70 @@ __global__ void __launch_bounds__(kPermThreads)
   }
 }
 
+// Small problems (T*k <= kSmallPairs): the whole counting sort in one block.
+// Pairs are staged in shared memory in j-major order; a pair's rank among
+// the pairs of its expert is the number of earlier pairs with that expert.
+constexpr int kSmallPairs = 2048;
+
+__global__ void __launch_bounds__(1024)
+    perm_small_kernel(const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_w, int T, int k,
+                      int M, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                      int32_t* __restrict__ slot_of, int32_t* __restrict__ row_token,
+                      float* __restrict__ row_w, int* status) {
+  extern __shared__ int sm_small[];
+  int* hist = sm_small;             // [M]
+  int* offs = sm_small + M;         // [M]
+  int* ex = sm_small + 2 * M;       // [pairs] expert of pair p (-1 if invalid)
+  __shared__ int s_tmp[33];
+  const int pairs = T * k;
+  for (int e = threadIdx.x; e < M; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  for (int p = threadIdx.x; p < pairs; p += blockDim.x) {
+    int e = pair_expert(topk_idx, p, T, k);
+    if (e < 0 || e >= M) {
+      set_status(status, MOE_DEVERR_BAD_EXPERT_INDEX);
+      e = -1;
+    } else {
+      atomicAdd(&hist[e], 1);
+    }
+    ex[p] = e;
+  }
+  __syncthreads();
+  const int total = block_exclusive_scan(hist, offs, M, s_tmp);
+  for (int e = threadIdx.x; e < M; e += blockDim.x) {
+    counts[e] = hist[e];
+    offsets[e] = offs[e];
+  }
+  if (threadIdx.x == 0) offsets[M] = total;
+  for (int p = threadIdx.x; p < pairs; p += blockDim.x) {
+    const int e = ex[p];
+    if (e < 0) continue;
+    int rank = 0;
+    for (int q = 0; q < p; ++q) rank += (ex[q] == e);
+    const int slot = offs[e] + rank;
+    const int t = p % T, j = p / T;
+    slot_of[t * k + j] = slot;
+    row_token[slot] = t;
+    row_w[slot] = topk_w[t * k + j];
+  }
+}
+
 cudaError_t launch_permute(const int32_t* topk_idx, const float* topk_w, int T, int k, int M,
                            int32_t* counts, int32_t* offsets, int32_t* slot_of, int32_t* row_token,
                            float* row_w, int32_t* chunk_counts, int32_t* chunk_base, int* status,
                            cudaStream_t s) {
   const long long pairs = static_cast<long long>(T) * k;
+  if (pairs <= kSmallPairs) {
+    const size_t smem = (2 * static_cast<size_t>(M) + pairs) * sizeof(int);
+    if (smem > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(perm_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+    }
+    perm_small_kernel<<<1, 1024, smem, s>>>(topk_idx, topk_w, T, k, M, counts, offsets, slot_of, row_token,
+                                            row_w, status);
+    return cudaGetLastError();
+  }
   const int nchunks = perm_num_chunks(pairs);
   perm_hist_kernel<<<nchunks, kPermThreads, M * sizeof(int), s>>>(topk_idx, T, k, M, nchunks,
                                                                   chunk_counts, status);

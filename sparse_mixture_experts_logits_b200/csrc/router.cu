@@ -61,14 +61,88 @@ __global__ void logits_f32_kernel(const float* __restrict__ x, const float* __re
   }
 }
 
+// Small-T bf16 logits, split over D: block (expert tile of 64, k-split ks)
+// computes partial[ks][t][e] = sum over its D range of x[t, d] W_r[d, e] for
+// every token t < T (T <= kSmallRouteT), each thread one expert and 16
+// tokens, summing in d order.  reduce_splits_kernel then adds the partials
+// in ks order, so the logits are deterministic.
+constexpr int kSmallRouteT = 64;
+constexpr int kSplitD = 128;
+
+__global__ void __launch_bounds__(256)
+    logits_splitk_bf16_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w_r,
+                              float* __restrict__ partial, int T, int D, int M) {
+  __shared__ __nv_bfloat16 xs[kSmallRouteT][kSplitD + 2];
+  __shared__ __nv_bfloat16 ws[kSplitD][64];
+  const int el = threadIdx.x & 63;
+  const int e = blockIdx.x * 64 + el;
+  const int tg = threadIdx.x >> 6;  // tokens tg*16 .. tg*16+15
+  const int d0 = blockIdx.y * kSplitD;
+  const int dn = min(kSplitD, D - d0);
+  const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
+  for (int i = threadIdx.x; i < kSmallRouteT * kSplitD; i += blockDim.x) {
+    const int t = i / kSplitD, d = i % kSplitD;
+    xs[t][d] = (t < T && d < dn) ? x[static_cast<size_t>(t) * D + d0 + d] : zero;
+  }
+  for (int i = threadIdx.x; i < kSplitD * 64; i += blockDim.x) {
+    const int d = i / 64, ee = blockIdx.x * 64 + (i % 64);
+    ws[d][i % 64] = (d < dn && ee < M) ? w_r[static_cast<size_t>(d0 + d) * M + ee] : zero;
+  }
+  __syncthreads();
+  float acc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+#pragma unroll 4
+  for (int d = 0; d < kSplitD; ++d) {
+    const float wv = __bfloat162float(ws[d][el]);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc[i] = fmaf(__bfloat162float(xs[tg * 16 + i][d]), wv, acc[i]);
+  }
+  if (e < M) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int t = tg * 16 + i;
+      if (t < T) partial[(static_cast<size_t>(blockIdx.y) * T + t) * M + e] = acc[i];
+    }
+  }
+}
+
+// logits[i] = sum_{ks} partial[ks][i], added in ks order.
+__global__ void reduce_splits_kernel(const float* __restrict__ partial, float* __restrict__ logits, int n,
+                                     int nsplit) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float acc = 0.f;
+#pragma unroll 8
+  for (int ks = 0; ks < nsplit; ++ks) acc += partial[static_cast<size_t>(ks) * n + i];
+  logits[i] = acc;
+}
+
+int route_splits(int T, int D, int dtype) {
+  return (dtype == MOE_DTYPE_BF16 && T <= kSmallRouteT) ? (D + kSplitD - 1) / kSplitD : 1;
+}
+
+cudaError_t launch_logits_splitk_bf16(const void* x, const void* w_r, float* partial, float* logits, int T,
+                                      int D, int M, cudaStream_t s) {
+  const int nsplit = (D + kSplitD - 1) / kSplitD;
+  dim3 grid((M + 63) / 64, nsplit);
+  logits_splitk_bf16_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
+                                                 static_cast<const __nv_bfloat16*>(w_r), partial, T, D, M);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int n = T * M;
+  reduce_splits_kernel<<<(n + 255) / 256, 256, 0, s>>>(partial, logits, n, nsplit);
+  return cudaGetLastError();
+}
+
 // One warp per token.  Selection score: the logit (softmax) or
 // sigmoid(logit) + e_bias (sigmoid router).  k rounds of a warp arg-max
 // with the lower expert index winning exact ties; slot j is the j-th round.
 constexpr int kTopkWarps = 8;
 
 __global__ void __launch_bounds__(kTopkWarps * 32)
-    topk_kernel(const float* __restrict__ logits, const float* __restrict__ e_bias, int T, int M,
-                int k, int gate, int norm_topk_prob, float alpha, float eps,
+    topk_kernel(const float* __restrict__ logits, const float* __restrict__ e_bias, int T,
+                int M, int k, int gate, int norm_topk_prob, float alpha, float eps,
                 int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
   extern __shared__ float topk_smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -146,7 +220,7 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
       float s = 0.f;
-      for (int e = lane; e < M; e += 32) s += expf(lrow[e] - m);
+      for (int e = lane; e < M; e += 32) s += expf(gv[e] - m);  // gv holds the logits (softmax gate)
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
       w = alpha * expf(chosen_val - m) / s;

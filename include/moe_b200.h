@@ -71,6 +71,7 @@ typedef enum { MOE_ACT_GELU_TANH = 0, MOE_ACT_SWIGLU = 1 } moe_act_t;
 #define MOE_DEVERR_NONE 0
 #define MOE_DEVERR_BAD_EXPERT_INDEX 1 /* topk_idx entry outside [0, M) */
 #define MOE_DEVERR_TIMEOUT 2          /* a bounded wait inside a kernel gave up */
+#define MOE_DEVERR_BAD_ROW_TOKEN 3    /* row_token entry outside [0, T) (row zero-filled) */
 
 /* One MoE layer's shape and options (HF config names in brackets). */
 typedef struct {
@@ -161,8 +162,11 @@ size_t moe_permute_workspace_size(int T, int k, int M);
  *   slot_of[T, k] (dispatch position of pair (t, j)), row_token[T k],
  *   row_w[T k] = topk_w[t, j] of the pair at each position.
  * Bit-exact and independent of scheduling (no atomics decide an order).
- * An out-of-range entry of topk_idx sets MOE_DEVERR_BAD_EXPERT_INDEX and
- * is skipped (its outputs are then unspecified). */
+ * An entry equal to M is the "no expert" sentinel of the GLM-5 page's
+ * GlmMoeDsaExperts.forward (one_hot over M + 1 classes, class M skipped):
+ * the pair is dispatched nowhere, slot_of = -1, and it is not counted.  An
+ * entry outside [0, M] is skipped the same way and sets
+ * MOE_DEVERR_BAD_EXPERT_INDEX. */
 moe_status_t moe_permute(const int32_t* topk_idx, const float* topk_w, int T, int k, int M,
                          int32_t* counts, int32_t* offsets, int32_t* slot_of,
                          int32_t* row_token, float* row_w,
@@ -197,7 +201,10 @@ size_t moe_expert_ffn_workspace_size(const moe_layer_desc_t* d);
  *   out_perm[s, :] = row_w[s] * E_e(x[row_token[s], :]) for every position s
  *   in expert e's segment [offsets[e], offsets[e+1]).
  * out_perm is fp32 [T k, D] (the accumulator, unrounded, so that the
- * combine rounds only once). */
+ * combine rounds only once).  Only the offsets[M] <= T k dispatched rows
+ * are read or written: when pairs were dropped through the sentinel index,
+ * row_token and row_w past offsets[M] may hold anything.  A row_token entry
+ * outside [0, T) is reported as MOE_DEVERR_BAD_ROW_TOKEN and read as zeros. */
 moe_status_t moe_expert_ffn(const moe_layer_desc_t* d, const moe_weights_t* w,
                             const void* x, const int32_t* offsets,
                             const int32_t* row_token, const float* row_w,
@@ -215,6 +222,7 @@ moe_status_t moe_shared_expert(const moe_layer_desc_t* d, const moe_weights_t* w
 /* ---- combine: "GLaM" eq. MoE; GLM-4.5 note eq. y ----------------------- */
 
 /* y[t, :] = sum_{j=0}^{k-1} out_perm[slot_of[t, j], :] (+ shared_out[t, :]),
+ * with slot_of < 0 (sentinel pairs) adding nothing,
  * out_perm fp32 [T k, D], shared_out and y [T, D] in dtype,
  * summed in fp32 in slot order and rounded once.  shared_out may be NULL. */
 moe_status_t moe_combine(const moe_layer_desc_t* d, const void* out_perm,

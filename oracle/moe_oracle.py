@@ -31,6 +31,10 @@ design notes):
     the order the quoted GlmMoeDsaExperts.forward enumerates with
     ``torch.where`` over the [k, T] expert mask.
   * The routed weight multiplies b2 too: w * (W2 h + b2).
+  * Expert index M (one past the last expert) is the "no expert" sentinel of
+    the quoted GlmMoeDsaExperts.forward (one_hot over M + 1 classes, class M
+    skipped): such a (token, slot) pair is dispatched nowhere and adds
+    nothing to y.
 
 Pins: every function here is checked, independently of its own code, by
 tests/test_oracle_pins.py (library routines, closed forms, invariants, brute
@@ -185,25 +189,30 @@ def adopt_topk(gpu_idx, sel, rel=1e-5):
 def permute(idx, w, M):
     """Dispatch order of the (token, slot) pairs.
 
-    [GLM5-SE] GlmMoeDsaExperts.forward: the expert mask one_hot(idx)
-    permuted to [M, k, T]; ``torch.where(expert_mask[e])`` lists expert e's
-    pairs as (slot j, token t) in row-major order.  Laying the experts'
-    lists end to end gives a stable sort by expert of the pairs taken in
-    (j, t) order.  Returns
-      counts[e]       pairs routed to expert e
-      offsets[e]      exclusive prefix sum of counts (offsets[M] = T k)
-      slot_of[t, j]   position of pair (t, j) in the dispatch order
+    [GLM5-SE] GlmMoeDsaExperts.forward: the expert mask one_hot(idx, M + 1)
+    permuted to [M + 1, k, T]; ``torch.where(expert_mask[e])`` lists expert
+    e's pairs as (slot j, token t) in row-major order, and class M (the
+    sentinel) is skipped.  Laying the experts' lists end to end gives a
+    stable sort by expert of the pairs taken in (j, t) order.  Returns
+      counts[e]       pairs routed to expert e (sentinel pairs not counted)
+      offsets[e]      exclusive prefix sum of counts (offsets[M] = pairs kept)
+      slot_of[t, j]   position of pair (t, j) in the dispatch order, -1 for
+                      a sentinel pair
       row_token[s]    token of the pair at position s
       row_w[s]        its gate weight w[t, j]
     """
     idx = np.asarray(idx, dtype=np.int64)
     T, k = idx.shape
-    counts = np.bincount(idx.reshape(-1), minlength=M).astype(np.int64)
+    if ((idx < 0) | (idx > M)).any():
+        raise ValueError("expert index outside [0, M]")
+    flat = idx.reshape(-1)
+    counts = np.bincount(flat[flat < M], minlength=M).astype(np.int64)
     offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
     jmajor = idx.T.reshape(-1)                      # position p = j*T + t
-    order = np.argsort(jmajor, kind="stable")       # dispatch position -> p
-    slot_jmajor = np.empty(T * k, dtype=np.int64)
-    slot_jmajor[order] = np.arange(T * k)
+    kept = np.nonzero(jmajor < M)[0]
+    order = kept[np.argsort(jmajor[kept], kind="stable")]  # dispatch position -> p
+    slot_jmajor = np.full(T * k, -1, dtype=np.int64)
+    slot_jmajor[order] = np.arange(order.size)
     slot_of = slot_jmajor.reshape(k, T).T.copy()
     row_token = (order % T).astype(np.int64) if T > 0 else order.astype(np.int64)
     row_w = None
@@ -252,19 +261,24 @@ def shared_expert(x, sh_w1, sh_w2):
     return expert_ffn(x, "swiglu", sh_w1, sh_w2)
 
 
-def moe_tokens(x_rows, idx_rows, w_rows, act, get_expert, shared=None):
+def moe_tokens(x_rows, idx_rows, w_rows, act, get_expert, shared=None, sentinel=None):
     """y_t = sum_{j} w_{t,j} E_{idx[t,j]}(x_t) (+ E_sh(x_t)) for given tokens.
 
     [GLaM] eq. MoE; [GLM45-SE] eq. y (a sum, no residual inside the layer).
     ``get_expert(e)`` returns (w1e, w2e, b1e, b2e); ``shared`` is
-    (sh_w1, sh_w2) or None.  Rows that chose expert e are batched into one
-    matmul; each row's value is that of its own matrix-vector product."""
+    (sh_w1, sh_w2) or None; pairs whose index equals ``sentinel`` (M) add
+    nothing.  Rows that chose expert e are batched into one matmul; each
+    row's value is that of its own matrix-vector product."""
     x_rows = _f64(x_rows)
     idx_rows = np.asarray(idx_rows, dtype=np.int64)
     w_rows = _f64(w_rows)
     n, k = idx_rows.shape
     y = np.zeros((n, x_rows.shape[1]), dtype=np.float64)
     for e in np.unique(idx_rows):
+        if e < 0:
+            raise ValueError("negative expert index")
+        if sentinel is not None and e == sentinel:
+            continue  # [GLM5-SE]: the sentinel class is skipped
         rr, jj = np.nonzero(idx_rows == e)
         w1e, w2e, b1e, b2e = get_expert(int(e))
         out = expert_ffn(x_rows[rr], act, w1e, w2e, b1e, b2e)

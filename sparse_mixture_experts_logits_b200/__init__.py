@@ -18,6 +18,6 @@ from .abi import (  # noqa: F401
     moe_forward_profiled, moe_forward_launch_count, NUM_STAGE_EVENTS, STAGE_NAMES,
     moe_algorithmic_work, EXPORTED_SYMBOLS,
     DTYPE_F32, DTYPE_BF16, GATE_SOFTMAX, GATE_SIGMOID_BIAS, ACT_GELU_TANH, ACT_SWIGLU,
-    DEVERR_NONE, DEVERR_BAD_EXPERT_INDEX, DEVERR_TIMEOUT,
+    DEVERR_NONE, DEVERR_BAD_EXPERT_INDEX, DEVERR_TIMEOUT, DEVERR_BAD_ROW_TOKEN,
 )
 from .layer import MoELayer, desc_from_config, weights_from_tensors  # noqa: F401

@@ -16,7 +16,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_DEVICE =
 DTYPE_F32, DTYPE_BF16 = 0, 1
 GATE_SOFTMAX, GATE_SIGMOID_BIAS = 0, 1
 ACT_GELU_TANH, ACT_SWIGLU = 0, 1
-DEVERR_NONE, DEVERR_BAD_EXPERT_INDEX, DEVERR_TIMEOUT = 0, 1, 2
+DEVERR_NONE, DEVERR_BAD_EXPERT_INDEX, DEVERR_TIMEOUT, DEVERR_BAD_ROW_TOKEN = 0, 1, 2, 3
 
 EXPORTED_SYMBOLS = [
     "moe_status_string", "moe_version", "moe_device_status",

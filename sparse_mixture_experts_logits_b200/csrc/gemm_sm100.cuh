@@ -205,6 +205,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tacc, 
           for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
           for (int j = 0; j < a.k; ++j) {
             const int slot = a.slot_of[static_cast<size_t>(row) * a.k + j];
+            if (slot < 0) continue;  // sentinel pair
             const float* src = a.comb_src + static_cast<size_t>(slot) * a.ldo + col;
             if (nv == 32) {
               const float4* s4 = reinterpret_cast<const float4*>(src);

@@ -138,8 +138,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   float* xbuf = reinterpret_cast<float*>(dyn_smem + (smem_base - smem_addr(dyn_smem)) + S * kSwStageBytes);
   const int G = args.num_groups;
 
-  for (int i = threadIdx.x; i <= G; i += blockDim.x)
-    s_off[i] = args.offsets != nullptr ? args.offsets[i] : (i == 0 ? 0 : args.rows);
+  // Segment bounds clamped to [0, rows], so that offsets that are not a
+  // valid dispatch cannot send a tile outside the token buffer (a segment
+  // whose end lies before its start gets no tile).
+  for (int i = threadIdx.x; i <= G; i += blockDim.x) {
+    const long long o = args.offsets != nullptr ? args.offsets[i] : (i == 0 ? 0 : args.rows);
+    s_off[i] = static_cast<int>(o < 0 ? 0 : (o > args.rows ? args.rows : o));
+  }
   __syncthreads();
   if (warp == 0) {
     int carry = 0;

@@ -29,8 +29,9 @@ cudaError_t launch_permute(const int32_t* topk_idx, const float* topk_w, int T, 
                            cudaStream_t s);
 
 // misc.cu
-cudaError_t launch_gather_rows(const void* x, const int32_t* row_token, void* x_perm, int rows,
-                               int D, int elem_bytes, cudaStream_t s);
+// Gathers rows r < min(rows, *n_rows) (n_rows device, may be null).
+cudaError_t launch_gather_rows(const void* x, const int32_t* row_token, const int32_t* n_rows, void* x_perm,
+                               int rows, int T, int D, int elem_bytes, int* status, cudaStream_t s);
 cudaError_t launch_combine(int dtype, const void* out_perm, const int32_t* slot_of,
                            const void* shared_out, bool shared_f32, void* y, int T, int D, int k,
                            cudaStream_t s);

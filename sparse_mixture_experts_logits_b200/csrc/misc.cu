@@ -4,43 +4,64 @@
 namespace moe {
 
 // x_perm[s, :] = x[row_token[s], :]; one warp per row, 16-byte vectors.
+// Rows r < min(rows, *n_rows) are gathered (n_rows = offsets[M] of the
+// dispatch, which is below T*k when pairs were dropped through the sentinel
+// index); a token index outside [0, T) is reported and its row zero-filled.
+__device__ __forceinline__ int gather_limit(const int32_t* n_rows, int rows) {
+  return n_rows ? max(0, min(rows, *n_rows)) : rows;
+}
+
 __global__ void gather_rows_vec_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ row_token,
-                                       uint4* __restrict__ x_perm, int rows, int vecs_per_row) {
+                                       const int32_t* __restrict__ n_rows, uint4* __restrict__ x_perm,
+                                       int rows, int T, int vecs_per_row, int* status) {
   const int warps_total = gridDim.x * (blockDim.x >> 5);
   const int lane = threadIdx.x & 31;
-  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps_total) {
-    const uint4* src = x + static_cast<size_t>(row_token[r]) * vecs_per_row;
+  const int n = gather_limit(n_rows, rows);
+  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < n; r += warps_total) {
+    const int tok = row_token[r];
     uint4* dst = x_perm + static_cast<size_t>(r) * vecs_per_row;
+    if (tok < 0 || tok >= T) {
+      if (lane == 0) set_status(status, MOE_DEVERR_BAD_ROW_TOKEN);
+      for (int v = lane; v < vecs_per_row; v += 32) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+      continue;
+    }
+    const uint4* src = x + static_cast<size_t>(tok) * vecs_per_row;
     for (int v = lane; v < vecs_per_row; v += 32) dst[v] = src[v];
   }
 }
 
 __global__ void gather_rows_f32_kernel(const float* __restrict__ x, const int32_t* __restrict__ row_token,
-                                       float* __restrict__ x_perm, int rows, int D) {
+                                       const int32_t* __restrict__ n_rows, float* __restrict__ x_perm,
+                                       int rows, int T, int D, int* status) {
   const int warps_total = gridDim.x * (blockDim.x >> 5);
   const int lane = threadIdx.x & 31;
-  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps_total) {
-    const float* src = x + static_cast<size_t>(row_token[r]) * D;
-    for (int d = lane; d < D; d += 32) x_perm[static_cast<size_t>(r) * D + d] = src[d];
+  const int n = gather_limit(n_rows, rows);
+  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < n; r += warps_total) {
+    const int tok = row_token[r];
+    const bool ok = tok >= 0 && tok < T;
+    if (!ok && lane == 0) set_status(status, MOE_DEVERR_BAD_ROW_TOKEN);
+    const float* src = x + static_cast<size_t>(ok ? tok : 0) * D;
+    for (int d = lane; d < D; d += 32) x_perm[static_cast<size_t>(r) * D + d] = ok ? src[d] : 0.f;
   }
 }
 
-cudaError_t launch_gather_rows(const void* x, const int32_t* row_token, void* x_perm, int rows,
-                               int D, int elem_bytes, cudaStream_t s) {
-  const int blocks = min((rows + 7) / 8, 4 * num_sms());
+cudaError_t launch_gather_rows(const void* x, const int32_t* row_token, const int32_t* n_rows, void* x_perm,
+                               int rows, int T, int D, int elem_bytes, int* status, cudaStream_t s) {
+  const int blocks = max(1, min((rows + 7) / 8, 4 * num_sms()));
   if ((static_cast<size_t>(D) * elem_bytes) % 16 == 0) {
-    gather_rows_vec_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(x), row_token,
-                                                  static_cast<uint4*>(x_perm), rows,
-                                                  static_cast<int>(static_cast<size_t>(D) * elem_bytes / 16));
+    gather_rows_vec_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(x), row_token, n_rows,
+                                                  static_cast<uint4*>(x_perm), rows, T,
+                                                  static_cast<int>(static_cast<size_t>(D) * elem_bytes / 16),
+                                                  status);
   } else {
-    gather_rows_f32_kernel<<<blocks, 256, 0, s>>>(static_cast<const float*>(x), row_token,
-                                                  static_cast<float*>(x_perm), rows, D);
+    gather_rows_f32_kernel<<<blocks, 256, 0, s>>>(static_cast<const float*>(x), row_token, n_rows,
+                                                  static_cast<float*>(x_perm), rows, T, D, status);
   }
   return cudaGetLastError();
 }
 
 // y[t, :] = sum_j out_perm[slot_of[t, j], :] (+ shared[t, :]) in fp32, in
-// slot order, rounded once.  out_perm is fp32; shared is fp32 or the layer's
+// slot order (slots < 0, sentinel pairs, add nothing), rounded once.  out_perm is fp32; shared is fp32 or the layer's
 // type; y has the layer's type.  Block (token, 128 four-column groups); every
 // row read is contiguous, and the k rows of a token are loaded together.
 template <typename TY, typename TS>
@@ -56,6 +77,7 @@ __global__ void __launch_bounds__(128) combine_vec4_kernel(const float4* __restr
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 8
     for (int j = 0; j < k; ++j) {
+      if (s_slot[j] < 0) continue;  // sentinel pair
       const float4 a = out_perm[static_cast<size_t>(s_slot[j]) * D4 + v];
       acc.x += a.x; acc.y += a.y; acc.z += a.z; acc.w += a.w;
     }
@@ -86,7 +108,7 @@ __global__ void combine_kernel(const float* __restrict__ out_perm, const int32_t
     float acc = 0.f;
     for (int j = 0; j < k; ++j) {
       const int slot = slot_of[static_cast<size_t>(t) * k + j];
-      acc += out_perm[static_cast<size_t>(slot) * D + d];
+      if (slot >= 0) acc += out_perm[static_cast<size_t>(slot) * D + d];
     }
     if (shared != nullptr) acc += to_f32(shared[static_cast<size_t>(t) * D + d]);
     y[static_cast<size_t>(t) * D + d] = from_f32<TY>(acc);

@@ -230,7 +230,7 @@ moe_status_t run_experts(const moe_layer_desc_t* d, const moe_weights_t* w, cons
   const void* b1 = (!swiglu && d->has_bias) ? w->b1 : nullptr;
   const void* b2 = (!swiglu && d->has_bias) ? w->b2 : nullptr;
   if (d->dtype == MOE_DTYPE_BF16) {
-    MOE_CUDA(launch_gather_rows(x, row_token, x_perm, pairs, d->D, 2, s));
+    MOE_CUDA(launch_gather_rows(x, row_token, offsets + d->M, x_perm, pairs, d->T, d->D, 2, status, s));
     MOE_TRY(mk.at(3));
     SwapLaunch g1{};
     g1.W = w->w1; g1.w_rows = static_cast<long long>(d->M) * n1;

@@ -2,8 +2,11 @@
 // expert.
 //
 // The GLM-5 page's GlmMoeDsaExperts.forward builds the expert mask
-// one_hot(top_k_index).permute(2, 1, 0) of shape [M, k, T] and lists expert
-// e's pairs with torch.where, i.e. in (slot j, token t) order.  Placing the
+// one_hot(top_k_index, M + 1).permute(2, 1, 0) of shape [M + 1, k, T], lists
+// expert e's pairs with torch.where, i.e. in (slot j, token t) order, and
+// skips class M, the "no expert" sentinel.  Here too a pair whose index is M
+// is dispatched nowhere (slot_of = -1); an index outside [0, M] is reported
+// through the status flag and skipped the same way.  Placing the
 // experts' lists end to end is a stable sort by expert of the pairs taken in
 // j-major order p = j*T + t.  The three kernels below compute it without
 // any atomic operation deciding an order:
@@ -77,7 +80,7 @@ __global__ void __launch_bounds__(kPermThreads)
   if (p < pairs) {
     const int e = pair_expert(topk_idx, p, T, k);
     if (e >= 0 && e < M) atomicAdd(&hist[e], 1);
-    else set_status(status, MOE_DEVERR_BAD_EXPERT_INDEX);
+    else if (e != M) set_status(status, MOE_DEVERR_BAD_EXPERT_INDEX);
   }
   __syncthreads();
   for (int e = threadIdx.x; e < M; e += blockDim.x)
@@ -133,6 +136,9 @@ __global__ void __launch_bounds__(kPermThreads)
     slot_of[t * k + j] = slot;
     row_token[slot] = static_cast<int32_t>(t);
     row_w[slot] = topk_w[t * k + j];
+  } else if (p < pairs) {
+    const long long t = p % T, j = p / T;
+    slot_of[t * k + j] = -1;  // sentinel (or invalid) pair: dispatched nowhere
   }
 }
 
@@ -157,7 +163,7 @@ __global__ void __launch_bounds__(1024)
   for (int p = threadIdx.x; p < pairs; p += blockDim.x) {
     int e = pair_expert(topk_idx, p, T, k);
     if (e < 0 || e >= M) {
-      set_status(status, MOE_DEVERR_BAD_EXPERT_INDEX);
+      if (e != M) set_status(status, MOE_DEVERR_BAD_EXPERT_INDEX);
       e = -1;
     } else {
       atomicAdd(&hist[e], 1);
@@ -173,7 +179,10 @@ __global__ void __launch_bounds__(1024)
   if (threadIdx.x == 0) offsets[M] = total;
   for (int p = threadIdx.x; p < pairs; p += blockDim.x) {
     const int e = ex[p];
-    if (e < 0) continue;
+    if (e < 0) {
+      slot_of[(p % T) * k + p / T] = -1;  // sentinel (or invalid) pair: dispatched nowhere
+      continue;
+    }
     int rank = 0;
     for (int q = 0; q < p; ++q) rank += (ex[q] == e);
     const int slot = offs[e] + rank;

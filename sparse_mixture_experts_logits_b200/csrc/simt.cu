@@ -29,9 +29,10 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const SimtArgs args) {
     int mt = blockIdx.y, g = -1, row0 = 0, rows = 0;
     const int G = L.num_groups;
     for (int gg = 0; gg < G; ++gg) {
-      const int b = L.offsets ? L.offsets[gg] : 0;
-      const int e = L.offsets ? L.offsets[gg + 1] : static_cast<int>(L.rows);
-      const int tiles = (e - b + kSBM - 1) / kSBM;
+      const int nr = static_cast<int>(L.rows);
+      const int b = L.offsets ? min(max(L.offsets[gg], 0), nr) : 0;
+      const int e = L.offsets ? min(max(L.offsets[gg + 1], 0), nr) : nr;
+      const int tiles = e > b ? (e - b + kSBM - 1) / kSBM : 0;
       if (mt < tiles) { g = gg; row0 = b + mt * kSBM; rows = min(kSBM, e - row0); break; }
       mt -= tiles;
     }
@@ -107,8 +108,10 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const SimtArgs args) {
         v *= L.row_scale[row];
       } else if constexpr (EPI == EPI_COMBINE) {
         float s = 0.f;
-        for (int jj = 0; jj < L.k; ++jj)
-          s += L.comb_src[static_cast<size_t>(L.slot_of[static_cast<size_t>(row) * L.k + jj]) * L.ldo + n];
+        for (int jj = 0; jj < L.k; ++jj) {
+          const int slot = L.slot_of[static_cast<size_t>(row) * L.k + jj];
+          if (slot >= 0) s += L.comb_src[static_cast<size_t>(slot) * L.ldo + n];
+        }
         v = s + v;
       }
       L.out[static_cast<size_t>(row) * L.ldo + n] = v;

@@ -141,6 +141,42 @@ def pin_bias_selects_only(O):
 # dispatch
 # ---------------------------------------------------------------------------
 
+def pin_sentinel(O):
+    """Index M is the "no expert" class ("GLM-5 - Shared expert", the quoted
+    GlmMoeDsaExperts.forward: one_hot over M + 1 classes, class M skipped):
+    a pair holding it is dispatched nowhere and contributes nothing."""
+    rng = np.random.default_rng(8)
+    T, k, M = 23, 3, 6
+    idx = np.stack([rng.choice(M, size=k, replace=False) for _ in range(T)])
+    drop = rng.random((T, k)) < 0.3
+    idx_s = np.where(drop, M, idx)
+    w = rng.random((T, k))
+    p = O.permute(idx_s, w, M)
+    assert p["counts"].sum() == (~drop).sum() == p["offsets"][M]
+    assert (p["slot_of"][drop] == -1).all()
+    s = 0
+    for e in range(M):
+        for j in range(k):
+            for t in range(T):
+                if idx_s[t, j] == e:
+                    assert p["slot_of"][t, j] == s and p["row_token"][s] == t
+                    s += 1
+    # contribution: the sentinel pairs add nothing, i.e. the same as weight 0
+    cfg = dict(TINY[2])
+    inp = tiny_inputs(cfg, 70)
+    r = O.route(inp["x"], inp["w_r"], inp["e_bias"], cfg["k"], cfg["gate"], 1, cfg["alpha"], cfg["eps"])
+    dropk = np.zeros_like(r["idx"], dtype=bool)
+    dropk[::2, 1] = True
+    idx2 = np.where(dropk, cfg["M"], r["idx"])
+    w0 = np.where(dropk, 0.0, r["w"])
+
+    def get(e):
+        return inp["w1"][e], inp["w2"][e], None, None
+    y_s = O.moe_tokens(inp["x"], idx2, r["w"], cfg["act"], get, None, sentinel=cfg["M"])
+    y_0 = O.moe_tokens(inp["x"], r["idx"], w0, cfg["act"], get, None)
+    assert np.allclose(y_s, y_0, rtol=1e-13, atol=1e-13)
+
+
 def pin_permute(O):
     rng = np.random.default_rng(5)
     for T, k, M in [(37, 3, 7), (64, 8, 16), (1, 1, 1), (5, 4, 64)]:
@@ -366,7 +402,7 @@ def pin_adopt_topk(O):
 
 ALL_PINS = [
     pin_gelu, pin_silu_sigmoid, pin_topk_bruteforce, pin_softmax_top2_closed_form,
-    pin_sigmoid_router, pin_bias_selects_only, pin_permute, pin_bruteforce_forward,
+    pin_sigmoid_router, pin_bias_selects_only, pin_permute, pin_sentinel, pin_bruteforce_forward,
     pin_single_expert_is_dense_ffn, pin_k_equals_m, pin_shared_branch,
     pin_sum_no_residual, pin_param_counts, pin_error_metrics, pin_adopt_topk,
 ]

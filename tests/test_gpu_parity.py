@@ -191,3 +191,90 @@ def test_bad_expert_index_is_reported_not_faulted(B):
     assert B.moe_device_status(ws.data_ptr(), s) == B.DEVERR_BAD_EXPERT_INDEX
     assert B.moe_device_status(ws.data_ptr(), s) == 0  # read clears it
     assert int(outs[0].sum()) == T * k - 2
+
+
+@pytest.mark.parametrize("name,frac", [("glm_small_bf16", 0.25), ("glam_small_bf16", 0.4),
+                                       ("glm_small_f32", 0.3), ("glm_medium_bf16", 0.6)])
+def test_sentinel_pairs_are_dispatched_nowhere(B, name, frac):
+    """Expert index M marks a dropped pair (the GLM-5 page's expert mask over
+    M + 1 classes, class M skipped): moe_permute dispatches it nowhere
+    (slot_of = -1, not counted), moe_combine adds nothing for it."""
+    cfg = ms.get_config(name)
+    inp = gpu_inputs(cfg)
+    T, D, M, k = cfg["T"], cfg["D"], cfg["M"], cfg["k"]
+    r = oracle_route(cfg, inp)
+    idx = r["idx"].copy()
+    drop = np.random.default_rng(3).random(idx.shape) < frac
+    idx[drop] = M
+    w32 = r["w"].astype(np.float32)
+    dev = "cuda"
+    s = torch.cuda.current_stream().cuda_stream
+    idx_d = torch.as_tensor(idx, dtype=torch.int32, device=dev)
+    w_d = torch.as_tensor(w32, device=dev)
+    counts = torch.empty(M, dtype=torch.int32, device=dev)
+    offsets = torch.empty(M + 1, dtype=torch.int32, device=dev)
+    slot_of = torch.empty(T, k, dtype=torch.int32, device=dev)
+    row_token = torch.empty(T * k, dtype=torch.int32, device=dev)
+    row_w = torch.empty(T * k, dtype=torch.float32, device=dev)
+    nbytes = B.moe_permute_workspace_size(T, k, M)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+    B.moe_permute(idx_d.data_ptr(), w_d.data_ptr(), T, k, M, counts.data_ptr(), offsets.data_ptr(),
+                  slot_of.data_ptr(), row_token.data_ptr(), row_w.data_ptr(), ws.data_ptr(), nbytes, s)
+    assert B.moe_device_status(ws.data_ptr(), s) == 0
+    p = oracle.permute(idx, w32.astype(np.float64), M)
+    kept = int(p["offsets"][M])
+    assert np.array_equal(counts.cpu().numpy(), p["counts"])
+    assert np.array_equal(offsets.cpu().numpy(), p["offsets"])
+    assert np.array_equal(slot_of.cpu().numpy(), p["slot_of"])
+    assert np.array_equal(row_token.cpu().numpy()[:kept], p["row_token"])
+    assert np.array_equal(row_w.cpu().numpy()[:kept].astype(np.float64), p["row_w"])
+
+    d = B.desc_from_config(cfg)
+    weights = B.weights_from_tensors(inp)
+    out_perm = torch.empty(T * k, D, dtype=torch.float32, device=dev)
+    wf = torch.zeros(B.moe_expert_ffn_workspace_size(d) + 256, dtype=torch.uint8, device=dev)
+    B.moe_expert_ffn(d, weights, inp["x"].data_ptr(), offsets.data_ptr(), row_token.data_ptr(),
+                     row_w.data_ptr(), out_perm.data_ptr(), wf.data_ptr(), wf.numel(), s)
+    shared_out = None
+    if cfg.get("I_sh"):
+        shared_out = torch.empty_like(inp["x"])
+        wsh = torch.zeros(B.moe_shared_expert_workspace_size(d) + 256, dtype=torch.uint8, device=dev)
+        B.moe_shared_expert(d, weights, inp["x"].data_ptr(), shared_out.data_ptr(), wsh.data_ptr(),
+                            wsh.numel(), s)
+    y = torch.empty_like(inp["x"])
+    B.moe_combine(d, out_perm.data_ptr(), slot_of.data_ptr(),
+                  None if shared_out is None else shared_out.data_ptr(), y.data_ptr(), s)
+    torch.cuda.synchronize()
+    shared = (np64(inp["sh_w1"]), np64(inp["sh_w2"])) if cfg.get("I_sh") else None
+    from gpu_common import HostExperts
+    y_ref = oracle.moe_tokens(np64(inp["x"]), idx, w32.astype(np.float64), cfg["act"], HostExperts(inp),
+                              shared, sentinel=M)
+    check_y(dict(cfg, named=False), np64(y), y_ref)
+
+
+def test_bad_row_token_is_reported_not_faulted(B):
+    """A dispatch row whose token index is outside [0, T) is read as zeros
+    and reported through the status flag; the other rows are unaffected."""
+    cfg = ms.get_config("glm_small_bf16")
+    inp = gpu_inputs(cfg)
+    layer, y, v = run_forward(B, cfg, inp)
+    d = layer.desc
+    T, D, k = cfg["T"], cfg["D"], cfg["k"]
+    dev = "cuda"
+    s = torch.cuda.current_stream().cuda_stream
+    offsets = torch.as_tensor(v["offsets"], device=dev)
+    row_token = torch.as_tensor(v["row_token"], device=dev).clone()
+    row_w = torch.as_tensor(v["row_w"], device=dev)
+    bad = [5, T * k // 2]
+    row_token[bad[0]] = T + 3
+    row_token[bad[1]] = -1
+    out_perm = torch.empty(T * k, D, dtype=torch.float32, device=dev)
+    wf = torch.zeros(B.moe_expert_ffn_workspace_size(d) + 256, dtype=torch.uint8, device=dev)
+    B.moe_expert_ffn(d, layer.weights, inp["x"].data_ptr(), offsets.data_ptr(), row_token.data_ptr(),
+                     row_w.data_ptr(), out_perm.data_ptr(), wf.data_ptr(), wf.numel(), s)
+    assert B.moe_device_status(wf.data_ptr(), s) == B.DEVERR_BAD_ROW_TOKEN
+    ref = layer.view("out_perm")
+    keep = torch.ones(T * k, dtype=torch.bool, device=dev)
+    keep[bad] = False
+    assert torch.equal(out_perm[keep].view(torch.int32), ref[keep].view(torch.int32))
+    assert torch.isfinite(out_perm[bad]).all()

@@ -39,8 +39,8 @@ L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # Files whose content defines the GEMM kernel measured by the recorded ncu
 # counters (a change voids the recorded traffic figure).
-GEMM_SOURCES = ["sparse_mixture_experts_logits_b200/csrc/gemm_sm100.cuh",
-                "sparse_mixture_experts_logits_b200/csrc/gemm_sm100.cu",
+GEMM_SOURCES = ["sparse_mixture_experts_logits_b200/csrc/gemm_swap_sm100.cuh",
+                "sparse_mixture_experts_logits_b200/csrc/gemm_swap_sm100.cu",
                 "sparse_mixture_experts_logits_b200/csrc/common.cuh"]
 
 

@@ -103,6 +103,15 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// Warp-wide form: every lane polls, and the warp leaves together with one
+// outcome (false when any lane saw the abort flag or the time limit).  Keeps
+// the caller's loop control warp-uniform.
+__device__ __forceinline__ bool mbar_wait_all(uint32_t bar, uint32_t parity, volatile int* abort,
+                                              int* status) {
+  const bool ok = mbar_wait(bar, parity, abort, status);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // Same, bounded by time only (used while draining after an abort).
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();

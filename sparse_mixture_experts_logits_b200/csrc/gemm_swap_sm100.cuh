@@ -41,6 +41,7 @@ constexpr int kSwXPitch = 33;                 // floats per row of the gate/up h
 constexpr int kSwXBytes = 4 * 32 * kSwXPitch * 4;
 constexpr int kSwDynSmem = kSwStages * kSwStageBytes + kSwXBytes + 1024;
 constexpr int kSwMaxTile = 256;               // tokens per tile
+static_assert(kBK == 64, "the MMA loop issues four K = 16 slices per stage");
 
 struct SwapArgs {
   int num_groups;
@@ -200,21 +201,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int num_kb = (args.K + kBK - 1) / kBK;
   volatile int* abort_flag = &s_abort;
 
+  // The producer and MMA loops run on whole warps with warp-uniform control
+  // (stage, phase, tile); only lane 0 issues the TMA copies, MMAs and
+  // commits.  Loop bookkeeping in a single divergent lane costs enough issue
+  // cycles per k-block to leave the tensor pipe idle between MMAs.
   if (warp == 0) {
     // -------------------------------------------------------- TMA producer
-    if (lane == 0) {
-      uint32_t kiter = 0;
-      bool ok = true;
-      constexpr uint32_t tx_bytes = 2u * kSwStageBytes;  // both CTAs: weight rows + 128 token rows
-      for (int tile = unit; ok && tile < total; tile += units) {
-        const SwapTile t = swap_decode(tile, G, s_tstart, s_off, args.w_tiles);
-        const int x_row = s_off[t.g] + t.tok0 + static_cast<int>(rank) * (t.n >> 1);
-        const int w_base = t.g * args.w_rows_per_group + t.wt * args.w_tile_step +
-                           static_cast<int>(rank) * args.w_cta_step;
-        for (int kb = 0; kb < num_kb; ++kb, ++kiter) {
-          const int s = kiter % S;
-          const uint32_t ph = (kiter / S) & 1u;
-          if (!mbar_wait(smem_addr(&s_empty[s]), ph ^ 1u, abort_flag, args.status)) { ok = false; break; }
+    uint32_t s = 0, ph = 0;
+    bool ok = true;
+    constexpr uint32_t tx_bytes = 2u * kSwStageBytes;  // both CTAs: weight rows + 128 token rows
+    for (int tile = unit; ok && tile < total; tile += units) {
+      const SwapTile t = swap_decode(tile, G, s_tstart, s_off, args.w_tiles);
+      const int x_row = s_off[t.g] + t.tok0 + static_cast<int>(rank) * (t.n >> 1);
+      const int w_base = t.g * args.w_rows_per_group + t.wt * args.w_tile_step +
+                         static_cast<int>(rank) * args.w_cta_step;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait_all(smem_addr(&s_empty[s]), ph ^ 1u, abort_flag, args.status)) { ok = false; break; }
+        if (lane == 0) {
           const uint32_t sa = smem_base + s * kSwStageBytes;
           const uint32_t sb = sa + kSwATileBytes;
           const uint32_t full_leader = mapa_shared(smem_addr(&s_full[s]), 0);
@@ -223,41 +226,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tma_load_2d_pair(sa + 64 * kBK * 2, &tmap_w, full_leader, kb * kBK, w_base + args.w_hi_offset);
           tma_load_2d_pair(sb, &tmap_x, full_leader, kb * kBK, x_row);
         }
+        __syncwarp();
+        if (++s == S) { s = 0; ph ^= 1u; }
       }
     }
-    __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0 && leader) {
+    if (leader) {
       // -------------------------------------------------------- MMA issuer
-      uint32_t kiter = 0, it = 0;
+      uint32_t it = 0, s = 0, ph = 0;
       bool ok = true;
+      // descriptors of stage 0; stage s and k-slice kk add s * stage/16 and 2 * kk
+      // to the 14-bit start-address field, which never carries (smem < 256 KB)
+      const uint64_t da0 = sw128_kmajor_desc(smem_base);
+      const uint64_t db0 = sw128_kmajor_desc(smem_base + kSwATileBytes);
       for (int tile = unit; ok && tile < total; tile += units, ++it) {
         const SwapTile t = swap_decode(tile, G, s_tstart, s_off, args.w_tiles);
         const uint32_t idesc = umma_idesc_bf16(256, t.n);
         const uint32_t buf = it & 1u;
         const uint32_t tph = (it >> 1) & 1u;
-        if (!mbar_wait(smem_addr(&s_tempty[buf]), tph ^ 1u, abort_flag, args.status)) break;
+        if (!mbar_wait_all(smem_addr(&s_tempty[buf]), tph ^ 1u, abort_flag, args.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * 256u;
-        for (int kb = 0; kb < num_kb; ++kb, ++kiter) {
-          const int s = kiter % S;
-          const uint32_t ph = (kiter / S) & 1u;
-          if (!mbar_wait(smem_addr(&s_full[s]), ph, abort_flag, args.status)) { ok = false; break; }
-          const uint32_t sa = smem_base + s * kSwStageBytes;
-          const uint32_t sb = sa + kSwATileBytes;
-#pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk)
-            umma_bf16_pair(d_tmem, sw128_kmajor_desc(sa + kk * 32), sw128_kmajor_desc(sb + kk * 32), idesc,
-                           (kb | kk) != 0 ? 1u : 0u);
-          umma_commit_pair(smem_addr(&s_empty[s]), 0x3);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait_all(smem_addr(&s_full[s]), ph, abort_flag, args.status)) { ok = false; break; }
+          if (lane == 0) {
+            const uint64_t off = static_cast<uint64_t>(s * (kSwStageBytes >> 4));
+            umma_bf16_pair(d_tmem, da0 + off, db0 + off, idesc, kb != 0 ? 1u : 0u);
+            umma_bf16_pair(d_tmem, da0 + off + 2, db0 + off + 2, idesc, 1u);
+            umma_bf16_pair(d_tmem, da0 + off + 4, db0 + off + 4, idesc, 1u);
+            umma_bf16_pair(d_tmem, da0 + off + 6, db0 + off + 6, idesc, 1u);
+            umma_commit_pair(smem_addr(&s_empty[s]), 0x3);
+          }
+          __syncwarp();
+          if (++s == S) { s = 0; ph ^= 1u; }
         }
         if (!ok) break;
-        umma_commit_pair(smem_addr(&s_tfull[buf]), 0x3);
+        if (lane == 0) umma_commit_pair(smem_addr(&s_tfull[buf]), 0x3);
+        __syncwarp();
       }
-      umma_commit_pair(smem_addr(&s_drain), 0x1);
-      mbar_wait_drain(smem_addr(&s_drain), 0, kWaitTimeoutNs);
+      if (lane == 0) {
+        umma_commit_pair(smem_addr(&s_drain), 0x1);
+        mbar_wait_drain(smem_addr(&s_drain), 0, kWaitTimeoutNs);
+      }
+      __syncwarp();
     }
-    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;           // TMEM lane quarter

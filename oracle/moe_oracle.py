@@ -31,6 +31,12 @@ design notes):
     the order the quoted GlmMoeDsaExperts.forward enumerates with
     ``torch.where`` over the [k, T] expert mask.
   * The routed weight multiplies b2 too: w * (W2 h + b2).
+  * Group-limited routing ([GLM45-SE]: the router "optionally masks by
+    expert group"; the note gives no rule): the M experts form n_group equal
+    groups of consecutive indices; a group scores the sum of its two largest
+    selection scores (its only score when a group holds one expert); the
+    topk_group best groups (ties to the lower group index) stay eligible and
+    every other expert is excluded from the top-k.  n_group = 1 is no mask.
   * Expert index M (one past the last expert) is the "no expert" sentinel of
     the quoted GlmMoeDsaExperts.forward (one_hot over M + 1 classes, class M
     skipped): such a (token, slot) pair is dispatched nowhere and adds
@@ -48,7 +54,7 @@ import numpy as np
 
 __all__ = [
     "gelu_tanh", "silu", "sigmoid", "router_logits", "selection_scores",
-    "topk_select", "topk_weights", "route", "permute", "expert_ffn",
+    "topk_select", "group_limit", "topk_weights", "route", "permute", "expert_ffn",
     "shared_expert", "moe_tokens", "moe_forward", "adopt_topk",
     "param_count", "error_metrics",
 ]
@@ -118,6 +124,34 @@ def topk_select(sel, k):
     return order[:, :k].astype(np.int64)
 
 
+def group_limit(sel, n_group, topk_group):
+    """Group-limited selection scores ([GLM45-SE]: the router "optionally
+    masks by expert group" before keeping the top k).
+
+    Reading (the note names the step only): experts e in
+    [i * M / n_group, (i + 1) * M / n_group) form group i; the group's score
+    is the sum of its two largest selection scores (the single score of a
+    one-expert group); the topk_group groups with the largest scores stay
+    eligible (ties to the lower group index) and the selection score of every
+    expert outside them becomes -inf, so the top-k never takes it.  The
+    weights still come from the gate values of the chosen experts.
+    n_group <= 1 returns the scores unchanged."""
+    sel = _f64(sel)
+    if n_group is None or n_group <= 1:
+        return sel
+    T, M = sel.shape
+    if M % n_group != 0 or not 1 <= topk_group <= n_group:
+        raise ValueError("bad expert grouping")
+    size = M // n_group
+    per_group = sel.reshape(T, n_group, size)
+    best = -np.sort(-per_group, axis=2)[:, :, :min(2, size)]
+    group_score = best.sum(axis=2)
+    kept = np.argsort(-group_score, axis=1, kind="stable")[:, :topk_group]
+    eligible = np.zeros((T, n_group), dtype=bool)
+    np.put_along_axis(eligible, kept, True, axis=1)
+    return np.where(np.repeat(eligible, size, axis=1), sel, -np.inf)
+
+
 def topk_weights(idx, logits, g, gate, norm_topk_prob, alpha, eps):
     """Gate weights of the selected experts.
 
@@ -148,11 +182,12 @@ def topk_weights(idx, logits, g, gate, norm_topk_prob, alpha, eps):
     raise ValueError(gate)
 
 
-def route(x, w_r, e_bias, k, gate, norm_topk_prob, alpha, eps):
-    """The whole router: logits, selection, weights."""
+def route(x, w_r, e_bias, k, gate, norm_topk_prob, alpha, eps, n_group=1, topk_group=1):
+    """The whole router: logits, selection (group-limited when n_group > 1),
+    weights.  ``sel`` is the unmasked selection score."""
     logits = router_logits(x, w_r)
     sel, g = selection_scores(logits, gate, e_bias)
-    idx = topk_select(sel, k)
+    idx = topk_select(group_limit(sel, n_group, topk_group), k)
     w = topk_weights(idx, logits, g, gate, norm_topk_prob, alpha, eps)
     return {"logits": logits, "sel": sel, "g": g, "idx": idx, "w": w}
 
@@ -296,7 +331,8 @@ def moe_forward(cfg, inp, idx=None):
     (w1/w2/b1/b2 indexable by expert).  ``idx`` overrides the selection
     (used when the oracle adopts the GPU's choice at a near-tie)."""
     r = route(inp["x"], inp["w_r"], inp.get("e_bias"), cfg["k"], cfg["gate"],
-              cfg["norm_topk_prob"], cfg["alpha"], cfg["eps"])
+              cfg["norm_topk_prob"], cfg["alpha"], cfg["eps"], cfg.get("n_group", 1),
+              cfg.get("topk_group", 1))
     if idx is not None:
         r["idx"] = np.asarray(idx, dtype=np.int64)
         r["w"] = topk_weights(r["idx"], r["logits"], r["g"], cfg["gate"],

@@ -137,6 +137,53 @@ def pin_bias_selects_only(O):
     assert np.allclose(r["w"], gs / gs.sum(1, keepdims=True), rtol=1e-13)
 
 
+def _brute_group_topk(s, k, n_group, topk_group):
+    """Group-limited top-k with Python scalars: group score = sum of the two
+    largest member scores, the topk_group best groups (lower index on ties),
+    then the k best eligible experts (lower index on ties)."""
+    T, M = s.shape
+    size = M // n_group
+    out = np.zeros((T, k), dtype=np.int64)
+    for t in range(T):
+        row = [float(v) for v in s[t]]
+        gscore = []
+        for gi in range(n_group):
+            members = sorted(row[gi * size:(gi + 1) * size], reverse=True)
+            gscore.append(sum(members[:2]))
+        groups = sorted(range(n_group), key=lambda gi: (-gscore[gi], gi))[:topk_group]
+        eligible = [e for e in range(M) if e // size in groups]
+        best = sorted(eligible, key=lambda e: (-row[e], e))[:k]
+        out[t] = best
+    return out
+
+
+def pin_group_limit(O):
+    """Group-limited routing ("Shared Expert" GLM-4.5 note: the router
+    "optionally masks by expert group") against a scalar brute force, and the
+    two groupings that must reduce to the plain top-k."""
+    rng = np.random.default_rng(11)
+    for M, n_group, topk_group, k in [(8, 4, 2, 3), (12, 4, 2, 4), (12, 3, 1, 2), (16, 8, 3, 5),
+                                      (6, 6, 2, 2)]:
+        for s in (rng.standard_normal((48, M)) - 0.5,                            # negative scores too
+                  rng.integers(-3, 4, size=(48, M)).astype(np.float64) * 0.5):  # many exact ties
+            got = O.topk_select(O.group_limit(s, n_group, topk_group), k)
+            assert np.array_equal(got, _brute_group_topk(s, k, n_group, topk_group)), (M, n_group)
+    s = rng.standard_normal((64, 16))
+    plain = _brute_topk(s, 4)
+    assert np.array_equal(O.topk_select(O.group_limit(s, 4, 4), 4), plain)    # every group kept
+    assert np.array_equal(O.topk_select(O.group_limit(s, 16, 4), 4), plain)   # one expert per group
+    assert np.array_equal(O.topk_select(O.group_limit(s, 1, 1), 4), plain)    # no grouping
+    # through the router: selection masked by group, weights from the gate values
+    x = rng.standard_normal((30, 12))
+    w_r = rng.standard_normal((12, 16)) * 0.4
+    bias = rng.uniform(-0.3, 0.1, 16)
+    r = O.route(x, w_r, bias, 4, "sigmoid_bias", 1, 2.5, 1e-20, 4, 2)
+    g = torch.sigmoid(_t(x @ w_r)).numpy()
+    assert np.array_equal(r["idx"], _brute_group_topk(g + bias[None, :], 4, 4, 2))
+    gs = np.take_along_axis(g, r["idx"], axis=1)
+    assert np.allclose(r["w"], 2.5 * gs / gs.sum(1, keepdims=True), rtol=1e-13)
+
+
 # ---------------------------------------------------------------------------
 # dispatch
 # ---------------------------------------------------------------------------
@@ -402,7 +449,7 @@ def pin_adopt_topk(O):
 
 ALL_PINS = [
     pin_gelu, pin_silu_sigmoid, pin_topk_bruteforce, pin_softmax_top2_closed_form,
-    pin_sigmoid_router, pin_bias_selects_only, pin_permute, pin_sentinel, pin_bruteforce_forward,
+    pin_sigmoid_router, pin_bias_selects_only, pin_group_limit, pin_permute, pin_sentinel, pin_bruteforce_forward,
     pin_single_expert_is_dense_ffn, pin_k_equals_m, pin_shared_branch,
     pin_sum_no_residual, pin_param_counts, pin_error_metrics, pin_adopt_topk,
 ]

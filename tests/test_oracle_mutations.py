@@ -51,6 +51,44 @@ def m_bias_in_weights(O):
         orig(logits, gate, e_bias)[0], orig(logits, gate, e_bias)[0])
 
 
+def _grouped(O, group_score, masked_value=-np.inf, tie_high=False):
+    def group_limit(sel, n_group, topk_group):
+        sel = np.asarray(sel, np.float64)
+        if n_group <= 1:
+            return sel
+        T, M = sel.shape
+        size = M // n_group
+        gs = group_score(sel.reshape(T, n_group, size))
+        if tie_high:
+            order = n_group - 1 - np.argsort(-gs[:, ::-1], axis=1, kind="stable")
+        else:
+            order = np.argsort(-gs, axis=1, kind="stable")
+        keep = np.zeros((T, n_group), bool)
+        np.put_along_axis(keep, order[:, :topk_group], True, axis=1)
+        return np.where(np.repeat(keep, size, axis=1), sel, masked_value)
+    O.group_limit = group_limit
+
+
+def _top2_sum(g):
+    return (-np.sort(-g, axis=2))[:, :, :2].sum(axis=2)
+
+
+def m_group_score_max(O):
+    _grouped(O, lambda g: g.max(axis=2))
+
+
+def m_group_score_all(O):
+    _grouped(O, lambda g: g.sum(axis=2))
+
+
+def m_group_mask_zero(O):
+    _grouped(O, _top2_sum, masked_value=0.0)
+
+
+def m_group_tie_high(O):
+    _grouped(O, _top2_sum, tie_high=True)
+
+
 def m_tie_to_higher_index(O):
     def topk(sel, k):
         sel = np.asarray(sel, np.float64)
@@ -104,7 +142,8 @@ def m_wrong_param_count(O):
 
 MUTANTS = [m_swap_gate_up, m_drop_b2, m_bias_in_weights, m_tie_to_higher_index,
            m_no_renorm, m_no_alpha, m_token_major_dispatch, m_gelu_erf,
-           m_shared_missing, m_transposed_router, m_wrong_param_count]
+           m_shared_missing, m_transposed_router, m_wrong_param_count, m_group_score_max,
+           m_group_score_all, m_group_mask_zero, m_group_tie_high]
 
 
 @pytest.mark.parametrize("mutant", MUTANTS, ids=lambda f: f.__name__)

@@ -89,6 +89,9 @@ typedef struct {
   float eps;                   /* sigmoid renormalisation epsilon (1e-20) */
   int I_sh;                    /* shared expert width, 0 = no shared expert
                                   [moe_intermediate_size * n_shared_experts] */
+  int n_group;                 /* expert groups of the group-limited selection
+                                  (0 or 1 = no group limit) [n_group] */
+  int topk_group;              /* groups kept per token [topk_group] */
 } moe_layer_desc_t;
 
 /* Device pointers to one layer's weights.  Unused fields may be NULL. */
@@ -145,10 +148,17 @@ size_t moe_route_workspace_size(int T, int D, int M, int dtype);
  *   the k selected (norm_topk_prob) or the full softmax probability.
  *   SIGMOID_BIAS: selection on sigmoid(s) + e_bias; w = alpha * g /
  *   (sum_S g + eps) (norm_topk_prob) or alpha * g; the bias never enters w.
+ *   Group limit (the GLM-4.5 note: the router "optionally masks by expert
+ *   group"), on when n_group > 1: experts [i M/n_group, (i+1) M/n_group)
+ *   form group i, scored by the sum of its two largest selection scores; the
+ *   topk_group best groups (lower index on ties) stay eligible and the top-k
+ *   is taken over their experts only.  Needs M % n_group == 0,
+ *   n_group <= 32, 1 <= topk_group <= n_group, k <= topk_group M / n_group.
  * Limits: 1 <= k <= min(M, 32), M <= 1024; bf16 needs D % 16 == 0. */
 moe_status_t moe_route_topk(const void* x, const void* w_r, const float* e_bias,
                             int T, int D, int M, int k, int dtype, int gate,
                             int norm_topk_prob, float routed_scaling_factor, float eps,
+                            int n_group, int topk_group,
                             int32_t* topk_idx, float* topk_w,
                             void* ws, size_t ws_bytes, void* stream);
 

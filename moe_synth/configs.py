@@ -76,6 +76,14 @@ TEST_CONFIGS = {
         dtype="f32", T=77, D=64, M=12, k=3, gate="sigmoid_bias", act="swiglu",
         I=96, has_bias=0, norm_topk_prob=1, alpha=2.5, eps=1e-20, I_sh=64,
         w_r_std=0.05, bias_std=0.0, e_bias=("uniform", -0.1, 0.1)),
+    "glm_grouped_bf16": dict(
+        dtype="bf16", T=700, D=256, M=64, k=6, gate="sigmoid_bias", act="swiglu",
+        I=128, has_bias=0, norm_topk_prob=1, alpha=2.5, eps=1e-20, I_sh=128,
+        w_r_std=0.05, bias_std=0.0, e_bias=("uniform", -0.1, 0.1), n_group=8, topk_group=3),
+    "glm_grouped_f32": dict(
+        dtype="f32", T=90, D=64, M=32, k=4, gate="sigmoid_bias", act="swiglu",
+        I=64, has_bias=0, norm_topk_prob=1, alpha=1.0, eps=1e-20, I_sh=0,
+        w_r_std=0.05, bias_std=0.0, e_bias=("uniform", -0.1, 0.1), n_group=4, topk_group=2),
     "glam_nonorm_f32": dict(
         dtype="f32", T=50, D=64, M=8, k=2, gate="softmax", act="gelu_tanh",
         I=128, has_bias=1, norm_topk_prob=0, alpha=1.0, eps=1e-20, I_sh=0,

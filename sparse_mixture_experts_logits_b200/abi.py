@@ -44,6 +44,7 @@ class LayerDesc(ctypes.Structure):
         ("k", ctypes.c_int), ("gate", ctypes.c_int), ("act", ctypes.c_int), ("I", ctypes.c_int),
         ("has_bias", ctypes.c_int), ("norm_topk_prob", ctypes.c_int),
         ("routed_scaling_factor", ctypes.c_float), ("eps", ctypes.c_float), ("I_sh", ctypes.c_int),
+        ("n_group", ctypes.c_int), ("topk_group", ctypes.c_int),
     ]
 
 
@@ -83,7 +84,8 @@ _decl("moe_status_string", ctypes.c_char_p, [_i])
 _decl("moe_version", ctypes.c_char_p, [])
 _decl("moe_device_status", _i, [_vp, _vp, _P(_i)])
 _decl("moe_route_workspace_size", _sz, [_i, _i, _i, _i])
-_decl("moe_route_topk", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _f, _vp, _vp, _vp, _sz, _vp])
+_decl("moe_route_topk", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _f, _i, _i, _vp, _vp, _vp, _sz,
+                            _vp])
 _decl("moe_permute_workspace_size", _sz, [_i, _i, _i])
 _decl("moe_permute", _i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
 _decl("moe_permute_static_scratch", _i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp])
@@ -128,10 +130,10 @@ def moe_route_workspace_size(T, D, M, dtype) -> int:
 
 
 def moe_route_topk(x, w_r, e_bias, T, D, M, k, dtype, gate, norm_topk_prob, routed_scaling_factor,
-                   eps, topk_idx, topk_w, ws, ws_bytes, stream=None):
+                   eps, n_group, topk_group, topk_idx, topk_w, ws, ws_bytes, stream=None):
     _check("moe_route_topk", lib.moe_route_topk(
         x, w_r, e_bias, T, D, M, k, dtype, gate, norm_topk_prob, routed_scaling_factor, eps,
-        topk_idx, topk_w, ws, ws_bytes, stream))
+        n_group, topk_group, topk_idx, topk_w, ws, ws_bytes, stream))
 
 
 def moe_permute_workspace_size(T, k, M) -> int:

@@ -15,8 +15,11 @@ cudaError_t launch_logits_f32(const float* x, const float* w_r, float* logits, i
 int route_splits(int T, int D, int dtype);
 cudaError_t launch_logits_splitk_bf16(const void* x, const void* w_r, float* partial, float* logits, int T,
                                       int D, int M, cudaStream_t s);
+// n_group <= 1: no group limit (otherwise the caller checked M % n_group == 0,
+// n_group <= 32, 1 <= topk_group <= n_group and k <= topk_group * M / n_group).
 cudaError_t launch_topk(const float* logits, const float* e_bias, int T, int M, int k, int gate,
-                        int norm, float alpha, float eps, int32_t* idx, float* w, cudaStream_t s);
+                        int norm, float alpha, float eps, int n_group, int topk_group, int32_t* idx,
+                        float* w, cudaStream_t s);
 
 // permute.cu
 constexpr int kPermChunk = 512;  // (slot, token) pairs per chunk of the counting sort

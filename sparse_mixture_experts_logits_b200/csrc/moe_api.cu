@@ -65,9 +65,21 @@ moe_status_t check_router_args(int T, int D, int M, int k, int dtype, int gate) 
   return MOE_OK;
 }
 
+// Group-limited selection: n_group <= 1 is off; otherwise M splits into
+// n_group equal groups (at most 32), 1 <= topk_group <= n_group, and the
+// eligible groups hold at least k experts.
+moe_status_t check_groups(int M, int k, int n_group, int topk_group) {
+  if (n_group <= 1) return MOE_OK;
+  if (n_group > 32) return MOE_ERR_UNSUPPORTED;
+  if (M % n_group != 0 || topk_group < 1 || topk_group > n_group) return MOE_ERR_INVALID_ARG;
+  if (static_cast<long long>(topk_group) * (M / n_group) < k) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
 moe_status_t check_desc(const moe_layer_desc_t* d) {
   if (d == nullptr) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_router_args(d->T, d->D, d->M, d->k, d->dtype, d->gate));
+  MOE_TRY(check_groups(d->M, d->k, d->n_group, d->topk_group));
   if (d->act != MOE_ACT_GELU_TANH && d->act != MOE_ACT_SWIGLU) return MOE_ERR_INVALID_ARG;
   if (d->I < 1 || d->I_sh < 0 || !(d->eps >= 0.0f)) return MOE_ERR_INVALID_ARG;
   if (d->dtype == MOE_DTYPE_BF16 && (d->I % 16 != 0 || d->I_sh % 16 != 0)) return MOE_ERR_UNSUPPORTED;
@@ -189,8 +201,8 @@ struct Marks {
 };
 
 moe_status_t run_route(const void* x, const void* w_r, const float* e_bias, int T, int D, int M, int k,
-                       int dtype, int gate, int norm, float alpha, float eps, int32_t* idx, float* w,
-                       float* logits, void* wrT, int* status, cudaStream_t s) {
+                       int dtype, int gate, int norm, float alpha, float eps, int n_group, int topk_group,
+                       int32_t* idx, float* w, float* logits, void* wrT, int* status, cudaStream_t s) {
   const int nsplit = route_splits(T, D, dtype);
   if (dtype == MOE_DTYPE_BF16 && nsplit > 1) {
     // few tokens: split-K SIMT logits (no transpose, no tensor-core launch)
@@ -216,7 +228,7 @@ moe_status_t run_route(const void* x, const void* w_r, const float* e_bias, int 
                                D, M, s));
   }
   MOE_CUDA(launch_topk(logits, gate == MOE_GATE_SIGMOID_BIAS ? e_bias : nullptr, T, M, k, gate,
-                       norm, alpha, eps, idx, w, s));
+                       norm, alpha, eps, n_group > 1 ? n_group : 1, topk_group, idx, w, s));
   return MOE_OK;
 }
 
@@ -380,9 +392,11 @@ size_t moe_route_workspace_size(int T, int D, int M, int dtype) {
 
 moe_status_t moe_route_topk(const void* x, const void* w_r, const float* e_bias, int T, int D, int M,
                             int k, int dtype, int gate, int norm_topk_prob,
-                            float routed_scaling_factor, float eps, int32_t* topk_idx, float* topk_w,
-                            void* ws, size_t ws_bytes, void* stream) {
+                            float routed_scaling_factor, float eps, int n_group, int topk_group,
+                            int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
+                            void* stream) {
   MOE_TRY(check_router_args(T, D, M, k, dtype, gate));
+  MOE_TRY(check_groups(M, k, n_group, topk_group));
   if (!(eps >= 0.0f)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   if (!x || !w_r || !topk_idx || !topk_w || !ws || !aligned_ws(ws)) return MOE_ERR_INVALID_ARG;
@@ -393,7 +407,8 @@ moe_status_t moe_route_topk(const void* x, const void* w_r, const float* e_bias,
   int* status = at<int*>(ws, L.status);
   MOE_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
   return run_route(x, w_r, e_bias, T, D, M, k, dtype, gate, norm_topk_prob, routed_scaling_factor, eps,
-                   topk_idx, topk_w, at<float*>(ws, L.logits), at<void*>(ws, L.wrT), status, s);
+                   n_group, topk_group, topk_idx, topk_w, at<float*>(ws, L.logits), at<void*>(ws, L.wrT),
+                   status, s);
 }
 
 size_t moe_permute_workspace_size(int T, int k, int M) {
@@ -517,8 +532,8 @@ static moe_status_t forward_impl(const moe_layer_desc_t* d, const moe_weights_t*
   MOE_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
   MOE_TRY(mk.at(0));
   MOE_TRY(run_route(x, w->w_r, w->e_bias, d->T, d->D, d->M, d->k, d->dtype, d->gate, d->norm_topk_prob,
-                    d->routed_scaling_factor, d->eps, idx, tw, at<float*>(ws, L.logits),
-                    at<void*>(ws, L.wrT), status, s));
+                    d->routed_scaling_factor, d->eps, d->n_group, d->topk_group, idx, tw,
+                    at<float*>(ws, L.logits), at<void*>(ws, L.wrT), status, s));
   MOE_TRY(mk.at(1));
   MOE_CUDA(launch_permute(idx, tw, d->T, d->k, d->M, counts, offsets, slot_of, row_token, row_w,
                           at<int32_t*>(ws, L.chunk_counts), at<int32_t*>(ws, L.chunk_base), status, s));

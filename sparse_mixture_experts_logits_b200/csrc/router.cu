@@ -142,8 +142,8 @@ constexpr int kTopkWarps = 8;
 
 __global__ void __launch_bounds__(kTopkWarps * 32)
     topk_kernel(const float* __restrict__ logits, const float* __restrict__ e_bias, int T,
-                int M, int k, int gate, int norm_topk_prob, float alpha, float eps,
-                int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+                int M, int k, int gate, int norm_topk_prob, float alpha, float eps, int n_group,
+                int topk_group, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
   extern __shared__ float topk_smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float* sel = topk_smem + static_cast<size_t>(warp) * 2 * M;  // selection score
@@ -165,6 +165,38 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
     lmax = fmaxf(lmax, l);
   }
   __syncwarp();
+  if (n_group > 1) {
+    // Group-limited selection (the GLM-4.5 note's optional mask by expert
+    // group): lane g scores group g (experts g*gsz .. g*gsz+gsz-1) by the sum
+    // of its two largest selection scores; the topk_group best groups (lower
+    // index on ties) stay eligible, every other expert's score becomes -inf.
+    const int gsz = M / n_group;
+    float gscore = -INFINITY;
+    if (lane < n_group) {
+      float b1 = -INFINITY, b2 = -INFINITY;
+      for (int i = 0; i < gsz; ++i) {
+        const float v = sel[lane * gsz + i];
+        if (v > b1) { b2 = b1; b1 = v; } else if (v > b2) { b2 = v; }
+      }
+      gscore = gsz > 1 ? b1 + b2 : b1;
+    }
+    unsigned keep = 0u;
+    for (int r = 0; r < topk_group; ++r) {
+      const bool cand = lane < n_group && ((keep >> lane) & 1u) == 0u;
+      float bv = cand ? gscore : -INFINITY;
+      int bi = cand ? lane : 32;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+        if (oi < 32 && (bi >= 32 || ov > bv || (ov == bv && oi < bi))) { bv = ov; bi = oi; }
+      }
+      if (bi < 32) keep |= 1u << bi;
+    }
+    for (int e = lane; e < M; e += 32)
+      if (((keep >> (e / gsz)) & 1u) == 0u) sel[e] = -INFINITY;
+    __syncwarp();
+  }
   // A chosen entry's selection score is replaced by NaN, which never wins a
   // comparison.  If only NaN scores remain (NaN inputs), the lowest index
   // not yet chosen is taken so that the k indices stay distinct.
@@ -235,7 +267,8 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
 size_t topk_smem_bytes(int M) { return static_cast<size_t>(kTopkWarps) * 2 * M * sizeof(float); }
 
 cudaError_t launch_topk(const float* logits, const float* e_bias, int T, int M, int k, int gate,
-                        int norm, float alpha, float eps, int32_t* idx, float* w, cudaStream_t s) {
+                        int norm, float alpha, float eps, int n_group, int topk_group, int32_t* idx,
+                        float* w, cudaStream_t s) {
   const size_t smem = topk_smem_bytes(M);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -244,7 +277,7 @@ cudaError_t launch_topk(const float* logits, const float* e_bias, int T, int M, 
   }
   const int blocks = (T + kTopkWarps - 1) / kTopkWarps;
   topk_kernel<<<blocks, kTopkWarps * 32, smem, s>>>(logits, e_bias, T, M, k, gate, norm, alpha, eps,
-                                                     idx, w);
+                                                     n_group, topk_group, idx, w);
   return cudaGetLastError();
 }
 

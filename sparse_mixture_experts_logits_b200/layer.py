@@ -24,6 +24,8 @@ def desc_from_config(cfg: dict, T: int | None = None) -> abi.LayerDesc:
     d.routed_scaling_factor = float(cfg.get("alpha", 1.0))
     d.eps = float(cfg.get("eps", 1e-20))
     d.I_sh = int(cfg.get("I_sh", 0) or 0)
+    d.n_group = int(cfg.get("n_group", 1) or 1)
+    d.topk_group = int(cfg.get("topk_group", 1) or 1)
     return d
 
 

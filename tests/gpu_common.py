@@ -51,13 +51,46 @@ class HostExperts:
 def oracle_route(cfg, inp):
     b = inp.get("e_bias")
     return oracle.route(np64(inp["x"]), np64(inp["w_r"]), None if b is None else np64(b), cfg["k"],
-                        cfg["gate"], cfg["norm_topk_prob"], cfg["alpha"], cfg["eps"])
+                        cfg["gate"], cfg["norm_topk_prob"], cfg["alpha"], cfg["eps"],
+                        cfg.get("n_group", 1) or 1, cfg.get("topk_group", 1) or 1)
+
+
+def _check_grouped_topk(cfg, sel, gpu_idx):
+    """Group-limited top-k: equal to the oracle's, or explained by near-ties.
+
+    Where the GPU differs, its choice must be the top-k (per-slot near-ties
+    allowed) over a set of at most topk_group groups that holds every group
+    scoring clearly above the oracle's cut, and whose other groups score
+    within the near-tie band of the cut."""
+    n_group, topk_group, k = cfg["n_group"], cfg["topk_group"], cfg["k"]
+    T, M = sel.shape
+    size = M // n_group
+    masked = oracle.group_limit(sel, n_group, topk_group)
+    ref = oracle.topk_select(masked, k)
+    differ = np.nonzero((gpu_idx != ref).any(axis=1))[0]
+    for t in differ:
+        row = sel[t]
+        gscore = (-np.sort(-row.reshape(n_group, size), axis=1))[:, :min(2, size)].sum(axis=1)
+        cut = np.sort(gscore)[::-1][topk_group - 1]
+        band = TIE_REL * np.abs(gscore).max()
+        picked = set((np.asarray(gpu_idx[t]) // size).tolist())
+        forced = set(np.nonzero(gscore > cut + band)[0].tolist())
+        groups = forced | picked
+        assert len(groups) <= topk_group, f"token {t}: GPU experts span too many groups"
+        assert all(gscore[g] >= cut - band for g in picked), f"token {t}: GPU took an ineligible group"
+        allowed = np.repeat(np.isin(np.arange(n_group), sorted(groups)), size)
+        ok, _, _ = oracle.adopt_topk(gpu_idx[t:t + 1], np.where(allowed, row, -np.inf)[None, :], TIE_REL)
+        assert ok, f"token {t}: top-k inside the eligible groups differs beyond the near-tie band"
+    return len(differ)
 
 
 def check_routing(cfg, r, gpu_idx, gpu_w):
     """Top-k bit-exact up to near-ties (adopted), weights within W_ABS*alpha."""
-    ok, ndiff, bad = oracle.adopt_topk(gpu_idx, r["sel"], TIE_REL)
-    assert ok, f"top-k differs beyond the near-tie band at token {bad}"
+    if (cfg.get("n_group", 1) or 1) > 1:
+        ndiff = _check_grouped_topk(cfg, r["sel"], np.asarray(gpu_idx, dtype=np.int64))
+    else:
+        ok, ndiff, bad = oracle.adopt_topk(gpu_idx, r["sel"], TIE_REL)
+        assert ok, f"top-k differs beyond the near-tie band at token {bad}"
     w_ref = oracle.topk_weights(gpu_idx, r["logits"], r["g"], cfg["gate"], cfg["norm_topk_prob"],
                                 cfg["alpha"], cfg["eps"])
     err = np.abs(gpu_w - w_ref).max() if gpu_w.size else 0.0

@@ -48,7 +48,7 @@ def test_version_and_status_strings(B):
 
 
 def test_struct_layout_matches_header(B):
-    assert ctypes.sizeof(B.LayerDesc) == 13 * 4
+    assert ctypes.sizeof(B.LayerDesc) == 15 * 4
     assert ctypes.sizeof(B.Weights) == 8 * 8
     assert ctypes.sizeof(B.WsLayout) == 10 * 8
 
@@ -83,9 +83,26 @@ def test_invalid_arguments_are_rejected_on_the_host(B):
         B.moe_forward(d, w, 256, 256, 255, need)
     assert e.value.status == 1
     with pytest.raises(B.MoEError):
-        B.moe_route_topk(256, 256, None, 10, 64, 8, 9, 1, 0, 1, 1.0, 1e-20, 256, 256, 256, 1 << 20)
+        B.moe_route_topk(256, 256, None, 10, 64, 8, 9, 1, 0, 1, 1.0, 1e-20, 1, 1, 256, 256, 256, 1 << 20)
     with pytest.raises(B.MoEError):
         B.moe_permute(256, 256, 10, 2, 8, 256, 256, 256, 256, 256, 256, 0)
+
+
+@pytest.mark.parametrize("M,k,n_group,topk_group,status", [
+    (8, 2, 3, 1, 1),     # M not a multiple of the group count
+    (64, 2, 64, 4, 2),   # more than 32 groups
+    (8, 2, 4, 0, 1),     # no group kept
+    (8, 2, 4, 5, 1),     # more groups kept than exist
+    (16, 5, 4, 1, 1),    # the kept groups hold fewer than k experts
+])
+def test_bad_group_limits_rejected_before_launch(B, M, k, n_group, topk_group, status):
+    with pytest.raises(B.MoEError) as e:
+        B.moe_route_topk(256, 256, None, 10, 64, M, k, 1, 1, 1, 1.0, 1e-20, n_group, topk_group,
+                         256, 256, 256, 1 << 20)
+    assert e.value.status == status
+    d = _desc(B, "glm_small_bf16")
+    d.M, d.k, d.n_group, d.topk_group = M, k, n_group, topk_group
+    assert B.moe_workspace_size(d) == 0
 
 
 def test_zero_tokens_launch_nothing(B):
@@ -93,7 +110,7 @@ def test_zero_tokens_launch_nothing(B):
     w = B.Weights()
     w.w_r, w.w1, w.w2, w.sh_w1, w.sh_w2 = 256, 256, 256, 256, 256
     B.moe_forward(d, w, None, None, None, 0)
-    B.moe_route_topk(None, None, None, 0, 64, 8, 2, 1, 0, 1, 1.0, 1e-20, None, None, None, 0)
+    B.moe_route_topk(None, None, None, 0, 64, 8, 2, 1, 0, 1, 1.0, 1e-20, 1, 1, None, None, None, 0)
     B.moe_expert_ffn(d, w, None, None, None, None, None, None, 0)
     B.moe_combine(d, None, None, None, None)
 

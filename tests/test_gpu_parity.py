@@ -12,7 +12,7 @@ from gpu_common import (check_permutation, check_routing, check_y, gpu_inputs, n
 pytestmark = pytest.mark.gpu
 
 SMALL = ["glam_tiny_f32", "glam_small_bf16", "glm_small_bf16", "glm_medium_bf16", "glm_small_f32",
-         "glam_nonorm_f32"]
+         "glam_nonorm_f32", "glm_grouped_bf16", "glm_grouped_f32"]
 FULL = ["glam_prefill_bf16", "glm45_decode_bf16", "glm45_prefill_bf16", "glm5_skewed_prefill_bf16"]
 
 
@@ -59,6 +59,12 @@ def test_full_size_layer_sampled(B, name):
     check_layer(B, ms.get_config(name), all_tokens=False)
 
 
+def test_group_limited_full_size_sampled(B):
+    """The GLM-5 skewed prefill layer with the router limited to the 4 best
+    of 8 expert groups (32 experts each)."""
+    check_layer(B, ms.get_config("glm5_skewed_prefill_bf16", n_group=8, topk_group=4), all_tokens=False)
+
+
 @pytest.mark.parametrize("name,over", [
     ("glm_small_bf16", dict(T=1)),
     ("glm_small_bf16", dict(T=129)),
@@ -70,6 +76,10 @@ def test_full_size_layer_sampled(B, name):
     ("glm_small_bf16", dict(e_bias=("const", 0.0), alpha=1.0)),
     ("glm_medium_bf16", dict(e_bias=("zipf", 1.1, 1.0))),  # literal beta = 1: most experts empty
     ("glam_tiny_f32", dict(T=1)),
+    ("glm_small_bf16", dict(n_group=16, topk_group=4)),  # one expert per group
+    ("glm_small_bf16", dict(n_group=4, topk_group=4)),   # every group kept
+    ("glm_small_bf16", dict(n_group=4, topk_group=1)),   # k = the whole kept group
+    ("glam_small_bf16", dict(n_group=2, topk_group=1)),  # softmax router, groups of 4
 ])
 def test_edge_cases(B, name, over):
     check_layer(B, ms.get_config(name, **over), all_tokens=True)
@@ -120,7 +130,8 @@ def test_stage_entry_points_match_forward(B):
     w = torch.empty(T, k, dtype=torch.float32, device=dev)
     wr = ws(B.moe_route_workspace_size(T, D, M, d.dtype))
     B.moe_route_topk(inp["x"].data_ptr(), inp["w_r"].data_ptr(), inp["e_bias"].data_ptr(), T, D, M, k,
-                     d.dtype, d.gate, d.norm_topk_prob, d.routed_scaling_factor, d.eps, idx.data_ptr(),
+                     d.dtype, d.gate, d.norm_topk_prob, d.routed_scaling_factor, d.eps, d.n_group,
+                     d.topk_group, idx.data_ptr(),
                      w.data_ptr(), wr.data_ptr(), wr.numel(), s)
     torch.cuda.synchronize()
     assert np.array_equal(idx.cpu().numpy(), v["topk_idx"])

@@ -215,3 +215,22 @@ def layer_inputs(cfg, device="cpu") -> dict:
         "sh_w1": shared_w1(cfg, device),
         "sh_w2": shared_w2(cfg, device),
     }
+
+
+def addend_tokens(cfg, device="cpu") -> torch.Tensor:
+    """The other term of a block sum (attention output or residual), [T, D]."""
+    return normal((cfg["T"], cfg["D"]), 1.0, _key(cfg, "addend"), device, act_dtype(cfg))
+
+
+def dense_inputs(cfg, device="cpu") -> dict:
+    """Every input of one dense FFN layer call (the layer's weights are drawn
+    like one expert's, under the name "dense")."""
+    bias = bool(cfg.get("has_bias"))
+    return {
+        "x": x_tokens(cfg, device),
+        "w1": expert_w1(cfg, "dense", device),
+        "b1": expert_b1(cfg, "dense", device) if bias else None,
+        "w2": expert_w2(cfg, "dense", device),
+        "b2": expert_b2(cfg, "dense", device) if bias else None,
+        "addend": addend_tokens(cfg, device),
+    }

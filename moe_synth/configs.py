@@ -91,8 +91,24 @@ TEST_CONFIGS = {
 }
 
 
+# Dense FFN layers (no router): the "GLaM" note's DenseFFN between its MoE
+# layers (the GLaM prefill layer's own shapes), and small test cases.
+DENSE_CONFIGS = {
+    "glam_dense_bf16": dict(
+        dtype="bf16", T=8192, D=2048, I=8192, act="gelu_tanh", has_bias=1, bias_std=0.01),
+    "glam_dense_small_bf16": dict(
+        dtype="bf16", T=333, D=192, I=320, act="gelu_tanh", has_bias=1, bias_std=0.01),
+    "glm_dense_small_bf16": dict(
+        dtype="bf16", T=300, D=256, I=384, act="swiglu", has_bias=0, bias_std=0.0),
+    "glm_dense_small_f32": dict(
+        dtype="f32", T=77, D=64, I=96, act="swiglu", has_bias=0, bias_std=0.0),
+    "glam_dense_small_f32": dict(
+        dtype="f32", T=50, D=64, I=128, act="gelu_tanh", has_bias=1, bias_std=0.01),
+}
+
+
 def get_config(name: str, **overrides) -> dict:
-    base = CONFIGS.get(name) or TEST_CONFIGS.get(name)
+    base = CONFIGS.get(name) or TEST_CONFIGS.get(name) or DENSE_CONFIGS.get(name)
     if base is None:
         raise KeyError(name)
     cfg = dict(base)
@@ -105,4 +121,4 @@ def get_config(name: str, **overrides) -> dict:
 
 
 def all_config_names():
-    return list(CONFIGS) + list(TEST_CONFIGS)
+    return list(CONFIGS) + list(TEST_CONFIGS) + list(DENSE_CONFIGS)

@@ -55,7 +55,7 @@ import numpy as np
 __all__ = [
     "gelu_tanh", "silu", "sigmoid", "router_logits", "selection_scores",
     "topk_select", "group_limit", "topk_weights", "route", "permute", "expert_ffn",
-    "shared_expert", "moe_tokens", "moe_forward", "adopt_topk",
+    "shared_expert", "moe_tokens", "moe_forward", "dense_layer", "adopt_topk",
     "param_count", "error_metrics",
 ]
 
@@ -323,13 +323,16 @@ def moe_tokens(x_rows, idx_rows, w_rows, act, get_expert, shared=None, sentinel=
     return y
 
 
-def moe_forward(cfg, inp, idx=None):
+def moe_forward(cfg, inp, idx=None, addend=None):
     """Whole layer: route, dispatch order, experts, combine, shared add.
 
     ``cfg`` holds T, D, M, k, gate, act, norm_topk_prob, alpha, eps, I_sh;
     ``inp`` holds numpy arrays x, w_r, e_bias, w1, b1, w2, b2, sh_w1, sh_w2
     (w1/w2/b1/b2 indexable by expert).  ``idx`` overrides the selection
-    (used when the oracle adopts the GPU's choice at a near-tie)."""
+    (used when the oracle adopts the GPU's choice at a near-tie).  With
+    ``addend`` the output is the sparse block sum of the "GLaM" note, section
+    "Interleaving Dense and Sparse Layers": addend + MoE-FFN(x), addend
+    standing for Attention(h)."""
     r = route(inp["x"], inp["w_r"], inp.get("e_bias"), cfg["k"], cfg["gate"],
               cfg["norm_topk_prob"], cfg["alpha"], cfg["eps"], cfg.get("n_group", 1),
               cfg.get("topk_group", 1))
@@ -349,10 +352,23 @@ def moe_forward(cfg, inp, idx=None):
     if cfg.get("I_sh"):
         shared = (inp["sh_w1"], inp["sh_w2"])
     y = moe_tokens(inp["x"], r["idx"], r["w"], cfg["act"], get_expert, shared)
+    if addend is not None:
+        y = _f64(addend) + y
     out = dict(r)
     out.update(p)
     out["y"] = y
     return out
+
+
+def dense_layer(x, act, w1, w2, b1=None, b2=None, addend=None):
+    """A dense FFN layer: the "GLaM" note, section "Interleaving Dense and
+    Sparse Layers", h^{l+1} = Attention(h^l) + DenseFFN(h^l), with the FFN of
+    eq. FFN (GELU form, biases b1, b2); the GLM-4.5 note's dense prefix
+    layers, one wide SwiGLU (the same form as an expert, w1 = [gate; up]).
+    ``addend`` stands for the other term of the sum (Attention(h), or the
+    residual stream); without it the FFN output alone is returned."""
+    y = expert_ffn(x, act, w1, w2, b1, b2)
+    return y if addend is None else _f64(addend) + y
 
 
 # ---------------------------------------------------------------------------

@@ -408,6 +408,29 @@ def pin_sum_no_residual(O):
         inp[key] = np.zeros_like(inp[key])
     y = O.moe_forward(cfg, inp)["y"]
     assert np.array_equal(y, np.zeros_like(y))
+    # the block sum adds the other term outside the layer: with zero experts it is all that is left
+    a = np.random.default_rng(13).standard_normal(np.asarray(inp["x"]).shape)
+    assert np.array_equal(O.moe_forward(cfg, inp, addend=a)["y"], a)
+
+
+def pin_dense_layer(O):
+    """The dense FFN layer and the block sum ("GLaM" note, "Interleaving
+    Dense and Sparse Layers": h^{l+1} = Attention(h^l) + DenseFFN(h^l))
+    against torch.nn.functional.linear and the library activations."""
+    rng = np.random.default_rng(12)
+    T, D, I = 9, 12, 20
+    x = rng.standard_normal((T, D))
+    a = rng.standard_normal((T, D))
+    w1 = rng.standard_normal((I, D)) * 0.3
+    b1 = rng.standard_normal(I) * 0.1
+    w2 = rng.standard_normal((D, I)) * 0.3
+    b2 = rng.standard_normal(D) * 0.1
+    ref = (_t(a) + F.linear(F.gelu(F.linear(_t(x), _t(w1), _t(b1)), approximate="tanh"), _t(w2), _t(b2))).numpy()
+    assert np.allclose(O.dense_layer(x, "gelu_tanh", w1, w2, b1, b2, addend=a), ref, rtol=1e-12, atol=1e-12)
+    wgu = rng.standard_normal((2 * I, D)) * 0.3
+    ref = F.linear(F.silu(F.linear(_t(x), _t(wgu[:I]))) * F.linear(_t(x), _t(wgu[I:])), _t(w2)).numpy()
+    assert np.allclose(O.dense_layer(x, "swiglu", wgu, w2), ref, rtol=1e-12, atol=1e-12)
+    assert np.allclose(O.dense_layer(x, "swiglu", wgu, w2, addend=a), ref + a, rtol=1e-12, atol=1e-12)
 
 
 def pin_param_counts(O):
@@ -451,5 +474,5 @@ ALL_PINS = [
     pin_gelu, pin_silu_sigmoid, pin_topk_bruteforce, pin_softmax_top2_closed_form,
     pin_sigmoid_router, pin_bias_selects_only, pin_group_limit, pin_permute, pin_sentinel, pin_bruteforce_forward,
     pin_single_expert_is_dense_ffn, pin_k_equals_m, pin_shared_branch,
-    pin_sum_no_residual, pin_param_counts, pin_error_metrics, pin_adopt_topk,
+    pin_sum_no_residual, pin_dense_layer, pin_param_counts, pin_error_metrics, pin_adopt_topk,
 ]

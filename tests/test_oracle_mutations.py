@@ -140,10 +140,27 @@ def m_wrong_param_count(O):
     O.param_count = lambda D, M, I, act, I_sh=0, **kw: orig(D, M, I, act, I_sh=I_sh, **kw) - (2 * D * I_sh)
 
 
+def m_dense_drops_addend(O):
+    orig = O.dense_layer
+    O.dense_layer = lambda x, act, w1, w2, b1=None, b2=None, addend=None: orig(x, act, w1, w2, b1, b2)
+
+
+def m_block_drops_addend(O):
+    orig = O.moe_forward
+    O.moe_forward = lambda cfg, inp, idx=None, addend=None: orig(cfg, inp, idx)
+
+
+def m_dense_no_b2(O):
+    orig = O.dense_layer
+    O.dense_layer = lambda x, act, w1, w2, b1=None, b2=None, addend=None: orig(x, act, w1, w2, b1, None,
+                                                                                addend)
+
+
 MUTANTS = [m_swap_gate_up, m_drop_b2, m_bias_in_weights, m_tie_to_higher_index,
            m_no_renorm, m_no_alpha, m_token_major_dispatch, m_gelu_erf,
            m_shared_missing, m_transposed_router, m_wrong_param_count, m_group_score_max,
-           m_group_score_all, m_group_mask_zero, m_group_tie_high]
+           m_group_score_all, m_group_mask_zero, m_group_tie_high, m_dense_drops_addend, m_dense_no_b2,
+           m_block_drops_addend]
 
 
 @pytest.mark.parametrize("mutant", MUTANTS, ids=lambda f: f.__name__)

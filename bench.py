@@ -215,6 +215,14 @@ def workload_config(args):
     return ms.get_config(args.config, **over)
 
 
+def is_dense(cfg) -> bool:
+    return cfg["name"] in ms.DENSE_CONFIGS
+
+
+def metric_name(cfg) -> str:
+    return METRIC.replace("MoE-layer", "dense FFN layer") if is_dense(cfg) else METRIC
+
+
 # --------------------------------------------------------------------------
 # the GPU arm
 # --------------------------------------------------------------------------
@@ -390,6 +398,202 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def dense_stage_work(cfg):
+    """Algorithmic FLOPs and bytes of the dense layer's two GEMMs (weights,
+    biases and the addend; the hidden activations are not credited)."""
+    T, D, I = cfg["T"], cfg["D"], cfg["I"]
+    es = 2 if cfg["dtype"] == "bf16" else 4
+    n1 = 2 * I if cfg["act"] == "swiglu" else I
+    bias = cfg["act"] != "swiglu" and cfg.get("has_bias")
+    return {
+        "dense_up": (2.0 * T * D * n1, (n1 * D + (I if bias else 0) + T * D) * es),
+        "dense_down": (2.0 * T * I * D, (D * I + (D if bias else 0) + 2 * T * D) * es),
+    }
+
+
+def library_dense_ms(cfg, inp, flush, stream, steps=5):
+    """The same dense layer through PyTorch's library GEMMs (cuBLAS), timed
+    the same way: context for the tensor-core kernels, not the product."""
+    import torch.nn.functional as F
+    x, a = inp["x"], inp["addend"]
+    I = cfg["I"]
+
+    def layer():
+        if cfg["act"] == "swiglu":
+            gu = F.linear(x, inp["w1"])
+            h = F.silu(gu[:, :I]) * gu[:, I:]
+            return a + F.linear(h, inp["w2"])
+        h = F.gelu(F.linear(x, inp["w1"], inp.get("b1")), approximate="tanh")
+        return a + F.linear(h, inp["w2"], inp.get("b2"))
+
+    for _ in range(3):
+        layer()
+    times = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        layer()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return sum(times) / len(times)
+
+
+def run_dense(args):
+    """The dense FFN layer of the GLaM note's interleaved blocks:
+    y = addend + FFN(x), through moe_dense_ffn_profiled."""
+    import sparse_mixture_experts_logits_b200 as B
+
+    rank, local_rank, world = dist_env()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = dist_init(world, local_rank)
+    cfg = workload_config(args)
+    T, D = cfg["T"], cfg["D"]
+    inp = ms.dense_inputs(dict(cfg, T=1), dev)
+    r0, r1 = token_rows(rank, T)
+    rows = torch.arange(r0, r1, device=dev)
+    inp["x"] = ms.normal_rows(rows, D, 1.0, ms._key(cfg, "x"), ms.act_dtype(cfg))
+    inp["addend"] = ms.normal_rows(rows, D, 1.0, ms._key(cfg, "addend"), ms.act_dtype(cfg))
+    layer = B.DenseLayer(cfg, inp)
+    x, a = inp["x"], inp["addend"]
+    y = torch.empty_like(x)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    wargs = layer.args()
+
+    for _ in range(max(3, args.warmup)):
+        B.moe_dense_ffn(layer.desc, *wargs, x.data_ptr(), a.data_ptr(), y.data_ptr(), layer.ws_ptr,
+                        layer.ws_bytes, sh)
+    torch.cuda.synchronize()
+    if layer.device_status() != 0:
+        raise RuntimeError("device status flag set during warm-up")
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(B.NUM_DENSE_EVENTS)] for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    for evs in ev + [ends]:
+        for e in evs:
+            e.record(stream)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    for i in range(K):
+        flush.zero_()
+        B.moe_dense_ffn_profiled(layer.desc, *wargs, x.data_ptr(), a.data_ptr(), y.data_ptr(), layer.ws_ptr,
+                                 layer.ws_bytes, sh, [e.cuda_event for e in ev[i]])
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    if dist is not None:
+        dist.barrier()
+    if layer.device_status() != 0:
+        raise RuntimeError("device status flag set during the timed steps")
+    ms_local = sum(ev[i][0].elapsed_time(ends[i]) for i in range(K)) / K
+    stage_ms = {"dense_up": sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(K)) / K,
+                "dense_down": sum(ev[i][1].elapsed_time(ev[i][2]) for i in range(K)) / K}
+    ms_step = max_over_ranks(dist, ms_local, dev)
+
+    e2e = None
+    if not args.no_e2e:
+        x_host = x.cpu().pin_memory()
+        a_host = a.cpu().pin_memory()
+        y_host = torch.empty_like(x_host).pin_memory()
+        x_dev, a_dev = torch.empty_like(x), torch.empty_like(a)
+
+        def e2e_step():
+            x_dev.copy_(x_host, non_blocking=True)
+            a_dev.copy_(a_host, non_blocking=True)
+            B.moe_dense_ffn(layer.desc, *wargs, x_dev.data_ptr(), a_dev.data_ptr(), y.data_ptr(), layer.ws_ptr,
+                            layer.ws_bytes, sh)
+            y_host.copy_(y, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        e_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        for i in range(K):
+            flush.zero_()
+            e_s[i].record(stream)
+            e2e_step()
+            e_e[i].record(stream)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        e2e_ms = max_over_ranks(dist, sum(e_s[i].elapsed_time(e_e[i]) for i in range(K)) / K, dev)
+        nbytes = x.numel() * x.element_size()
+        e2e = {"value": world * T / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": 2 * nbytes, "d2h_bytes_per_step": nbytes}
+
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+    lib_ms = library_dense_ms(cfg, inp, flush, stream) if world == 1 else None
+    peaks, peak_src = load_peaks()
+    work = dense_stage_work(cfg)
+    dom = max(stage_ms, key=lambda k: stage_ms[k])
+    f, b = work[dom]
+    t_s = stage_ms[dom] / 1e3
+    peak_tf = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    peak_bw = peaks["hbm_gbs"]
+    if f / (peak_tf * 1e12) >= b / (peak_bw * 1e9):
+        roof = {"bound": "tensor", "achieved": f / t_s / 1e12, "peak": peak_tf, "unit": "TFLOP/s",
+                "frac_of_burst_peak": f / t_s / 1e12 / peaks["bf16_tflops"]}
+    else:
+        roof = {"bound": "hbm", "achieved": b / t_s / 1e9, "peak": peak_bw, "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = recorded_traffic(dom, args.config)
+    roof["kernel"] = f"moe_gemm_swap_kernel ({dom})"
+    roof["peak_source"] = (f"{peak_src}: " + ("bf16_tflops_sustained (kernel timed inside a long loop)"
+                                             if roof["bound"] == "tensor" else "hbm_gbs"))
+    roof["algorithmic"] = {"flops": f, "bytes": b}
+    flops_total = sum(v[0] for v in work.values())
+    out = {
+        "metric": metric_name(cfg),
+        "value": world * T / (ms_step / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": cfg["dtype"],
+        "data": "synthetic (seeded counter-based generator; random-init weights)",
+        "config": {"workload": args.config + ("" if cfg["T"] == ms.DENSE_CONFIGS[cfg["name"]]["T"]
+                                              else " (overridden: T=%d)" % T),
+                   "T_per_gpu": T, "D": D, "I": cfg["I"], "act": cfg["act"],
+                   "has_bias": int(bool(cfg.get("has_bias"))), "addend": True,
+                   "l2": "flushed between steps (256 MiB write outside the timed events)",
+                   "parallelism": f"replicas x{world} (token batches, no data-path collective)"},
+        "roofline": roof,
+        "layer": {"tflops": flops_total / (ms_step / 1e3) / 1e12, "algorithmic_flops": flops_total},
+        "stages_ms": stage_ms,
+        "library_gemms": None if lib_ms is None else {
+            "what": "the same layer through torch.nn.functional.linear (cuBLAS) and torch activations",
+            "ms_per_step": lib_ms, "tflops": flops_total / (lib_ms / 1e3) / 1e12},
+        "e2e": e2e,
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(cfg, inp, args.cpu_seconds)
+    print(json.dumps(out), flush=True)
+    del layer
+    if dist is not None:
+        dist.destroy_process_group()
+
+
 # --------------------------------------------------------------------------
 # the oracle on the host cores
 # --------------------------------------------------------------------------
@@ -437,12 +641,37 @@ class OracleRunner:
     def run(self, xs):
         c = self.cfg
         r = self.oracle.route(xs, self.w_r, self.e_bias, c["k"], c["gate"], c["norm_topk_prob"],
-                              c["alpha"], c["eps"])
+                              c["alpha"], c["eps"], c.get("n_group", 1) or 1, c.get("topk_group", 1) or 1)
         return self.oracle.moe_tokens(xs, r["idx"], r["w"], c["act"], self.get_expert, self.shared)
 
 
+class DenseOracleRunner:
+    """The CPU oracle's dense FFN layer (with its addend) on token blocks."""
+
+    def __init__(self, cfg, inp):
+        import oracle
+        self.oracle = oracle
+        self.cfg = cfg
+        self.x = inp["x"]
+        self.addend = inp["addend"]
+        host = {k: (None if v is None else v.cpu().double().numpy()) for k, v in inp.items()
+                if k not in ("x", "addend")}
+        self.w = host
+
+    def x_block(self, t0, n):
+        T = self.x.shape[0]
+        rows = (torch.arange(t0, t0 + n) % T).to(self.x.device)
+        return self.x[rows].double().cpu().numpy(), self.addend[rows].double().cpu().numpy()
+
+    def run(self, block):
+        xs, a = block
+        w = self.w
+        return self.oracle.dense_layer(xs, self.cfg["act"], w["w1"], w["w2"], w.get("b1"), w.get("b2"),
+                                       addend=a)
+
+
 def cpu_baseline(cfg, inp, target_s):
-    runner = OracleRunner(cfg, inp)
+    runner = DenseOracleRunner(cfg, inp) if is_dense(cfg) else OracleRunner(cfg, inp)
     n = 16
     while True:
         xs = runner.x_block(0, n)
@@ -453,9 +682,11 @@ def cpu_baseline(cfg, inp, target_s):
             break
         n = int(min(cfg["T"], max(2 * n, n * target_s / max(dt, 1e-3))))
     cores, api = _blas_threads()
+    widen = ("weights widened from bf16 once, outside the timed run" if is_dense(cfg) else
+             "weights widened from bf16 per expert inside the timed run")
     return {"value": n / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"first {n} of the workload's {cfg['T']} tokens through the fp64 NumPy oracle "
-                      f"({api} BLAS); weights widened from bf16 per expert inside the timed run",
+                      f"({api} BLAS); {widen}",
             "seconds": dt}
 
 
@@ -465,8 +696,10 @@ def run_reference(args):
         return
     cfg = workload_config(args)
     dev = torch.device("cuda", local_rank) if torch.cuda.is_available() else torch.device("cpu")
-    inp = ms.layer_inputs(cfg, dev)
-    runner = OracleRunner(cfg, inp)
+    if is_dense(cfg):
+        runner = DenseOracleRunner(cfg, ms.dense_inputs(cfg, dev))
+    else:
+        runner = OracleRunner(cfg, ms.layer_inputs(cfg, dev))
     # size one step's token sample from a probe so that the whole run stays short
     probe_n = 8
     t0 = time.perf_counter()
@@ -491,12 +724,14 @@ def run_reference(args):
     sample = (f"{n} consecutive tokens per step of the {cfg['T']}-token workload, fp64 NumPy oracle "
               f"({api} BLAS)")
     out = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "impl": "reference", "metric": metric_name(cfg), "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_s * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded counter-based generator; random-init weights)",
-        "config": {"workload": args.config, "T_per_gpu": cfg["T"], "D": cfg["D"], "M": cfg["M"],
-                   "k": cfg["k"], "I": cfg["I"], "I_sh": cfg.get("I_sh", 0)},
+        "config": ({"workload": args.config, "T_per_gpu": cfg["T"], "D": cfg["D"], "I": cfg["I"],
+                    "act": cfg["act"]} if is_dense(cfg) else
+                   {"workload": args.config, "T_per_gpu": cfg["T"], "D": cfg["D"], "M": cfg["M"],
+                    "k": cfg["k"], "I": cfg["I"], "I_sh": cfg.get("I_sh", 0)}),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -508,6 +743,8 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif is_dense(workload_config(args)):
+        run_dense(args)
     else:
         run_ours(args)
 

@@ -231,13 +231,16 @@ moe_status_t moe_shared_expert(const moe_layer_desc_t* d, const moe_weights_t* w
 
 /* ---- combine: "GLaM" eq. MoE; GLM-4.5 note eq. y ----------------------- */
 
-/* y[t, :] = sum_{j=0}^{k-1} out_perm[slot_of[t, j], :] (+ shared_out[t, :]),
+/* y[t, :] = sum_{j=0}^{k-1} out_perm[slot_of[t, j], :] (+ shared_out[t, :])
+ *           (+ addend[t, :]),
  * with slot_of < 0 (sentinel pairs) adding nothing,
- * out_perm fp32 [T k, D], shared_out and y [T, D] in dtype,
- * summed in fp32 in slot order and rounded once.  shared_out may be NULL. */
+ * out_perm fp32 [T k, D], shared_out, addend and y [T, D] in dtype,
+ * summed in fp32 in slot order and rounded once.  shared_out and addend may
+ * be NULL; addend is the other term of the "GLaM" block sum (see
+ * moe_forward_add). */
 moe_status_t moe_combine(const moe_layer_desc_t* d, const void* out_perm,
-                         const int32_t* slot_of, const void* shared_out, void* y,
-                         void* stream);
+                         const int32_t* slot_of, const void* shared_out,
+                         const void* addend, void* y, void* stream);
 
 /* ---- the whole layer --------------------------------------------------- */
 
@@ -251,6 +254,17 @@ moe_status_t moe_workspace_layout(const moe_layer_desc_t* d, moe_ws_layout_t* ou
  * synchronisation. */
 moe_status_t moe_forward(const moe_layer_desc_t* d, const moe_weights_t* w,
                          const void* x, void* y, void* ws, size_t ws_bytes, void* stream);
+
+/* y[T, D] = addend[T, D] + MoE-FFN(x): the sparse layer of the "GLaM" note,
+ * section "Interleaving Dense and Sparse Layers",
+ *   h^{l+1} = Attention(h^l) + MoE-FFN(h^l),
+ * with addend the other term (the attention output, or the residual
+ * stream).  The addend is added in fp32 inside the combine, before the one
+ * rounding of y.  addend (dtype) must not be NULL when T > 0 and must not
+ * overlap y.  Otherwise as moe_forward. */
+moe_status_t moe_forward_add(const moe_layer_desc_t* d, const moe_weights_t* w,
+                             const void* x, const void* addend, void* y,
+                             void* ws, size_t ws_bytes, void* stream);
 
 /* Stage boundaries recorded by moe_forward_profiled (the "routing overhead"
  * breakdown of the GLaM note's reporting table: gate, dispatch, expert
@@ -279,6 +293,44 @@ int moe_forward_launch_count(const moe_layer_desc_t* d);
  * intermediate buffers are not counted. */
 void moe_algorithmic_work(const moe_layer_desc_t* d, const int32_t* counts_host,
                           double* flops, double* bytes);
+
+/* ---- dense FFN layer: "GLaM" section "Interleaving Dense and Sparse
+ * Layers" (DenseFFN); GLM-4.5 note: dense prefix layers are one wide SwiGLU -- */
+
+typedef struct {
+  int dtype;    /* moe_dtype_t */
+  int T;        /* tokens */
+  int D;        /* model width [hidden_size] */
+  int I;        /* hidden width [intermediate_size] */
+  int act;      /* moe_act_t */
+  int has_bias; /* GELU: b1, b2 present (ignored for SWIGLU) */
+} moe_dense_desc_t;
+
+size_t moe_dense_ffn_workspace_size(const moe_dense_desc_t* d);
+
+/* y[T, D] = (addend[T, D] +) FFN(x), the dense layer of the "GLaM" note,
+ * h^{l+1} = Attention(h^l) + DenseFFN(h^l):
+ *   GELU_TANH: FFN(x) = W2 GELU(W1 x + b1) + b2 ("GLaM" eq. FFN),
+ *              w1 [I, D], b1 [I], w2 [D, I], b2 [D];
+ *   SWIGLU:    FFN(x) = W_down(SiLU(W_gate x) * W_up x),
+ *              w1 [2I, D] (gate rows first), w2 [D, I].
+ * All tensors in dtype, nn.Linear layout; addend may be NULL and must not
+ * overlap y.  The hidden
+ * activations are kept in the workspace in dtype; the second GEMM adds b2 and
+ * the addend in fp32 and rounds y once.  Limits: bf16 needs D % 16 == 0 and
+ * I % 16 == 0.  Errors as moe_forward. */
+moe_status_t moe_dense_ffn(const moe_dense_desc_t* d, const void* w1, const void* b1,
+                           const void* w2, const void* b2, const void* x,
+                           const void* addend, void* y, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* moe_dense_ffn recording events[0] at the start, events[1] after the first
+ * GEMM and events[2] after the second (n_events == MOE_NUM_DENSE_EVENTS). */
+#define MOE_NUM_DENSE_EVENTS 3
+moe_status_t moe_dense_ffn_profiled(const moe_dense_desc_t* d, const void* w1, const void* b1,
+                                    const void* w2, const void* b2, const void* x,
+                                    const void* addend, void* y, void* ws, size_t ws_bytes,
+                                    void* stream, void* const* events, int n_events);
 
 #ifdef __cplusplus
 }

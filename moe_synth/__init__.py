@@ -31,7 +31,7 @@ import math
 
 import torch
 
-from .configs import CONFIGS, TEST_CONFIGS, get_config, all_config_names  # noqa: F401
+from .configs import CONFIGS, DENSE_CONFIGS, TEST_CONFIGS, get_config, all_config_names, dense_config_names  # noqa: F401,E501
 
 _MASK32 = 0xFFFFFFFF
 _MIX = 0x45D9F3B

@@ -121,4 +121,9 @@ def get_config(name: str, **overrides) -> dict:
 
 
 def all_config_names():
-    return list(CONFIGS) + list(TEST_CONFIGS) + list(DENSE_CONFIGS)
+    """Names of the MoE layer workloads (named and test cases)."""
+    return list(CONFIGS) + list(TEST_CONFIGS)
+
+
+def dense_config_names():
+    return list(DENSE_CONFIGS)

@@ -16,8 +16,9 @@ from .abi import (  # noqa: F401
     moe_shared_expert_workspace_size, moe_shared_expert,
     moe_combine, moe_workspace_size, moe_workspace_layout, moe_forward,
     moe_forward_profiled, moe_forward_launch_count, NUM_STAGE_EVENTS, STAGE_NAMES,
-    moe_algorithmic_work, EXPORTED_SYMBOLS,
+    moe_algorithmic_work, EXPORTED_SYMBOLS, moe_forward_add,
+    DenseDesc, moe_dense_ffn_workspace_size, moe_dense_ffn, moe_dense_ffn_profiled, NUM_DENSE_EVENTS,
     DTYPE_F32, DTYPE_BF16, GATE_SOFTMAX, GATE_SIGMOID_BIAS, ACT_GELU_TANH, ACT_SWIGLU,
     DEVERR_NONE, DEVERR_BAD_EXPERT_INDEX, DEVERR_TIMEOUT, DEVERR_BAD_ROW_TOKEN,
 )
-from .layer import MoELayer, desc_from_config, weights_from_tensors  # noqa: F401
+from .layer import DenseLayer, MoELayer, dense_desc_from_config, desc_from_config, weights_from_tensors  # noqa: F401,E501

@@ -26,8 +26,10 @@ EXPORTED_SYMBOLS = [
     "moe_shared_expert_workspace_size", "moe_shared_expert",
     "moe_combine", "moe_workspace_size", "moe_workspace_layout", "moe_forward",
     "moe_forward_profiled", "moe_forward_launch_count", "moe_algorithmic_work",
+    "moe_forward_add", "moe_dense_ffn_workspace_size", "moe_dense_ffn", "moe_dense_ffn_profiled",
 ]
 NUM_STAGE_EVENTS = 9
+NUM_DENSE_EVENTS = 3
 STAGE_NAMES = ["route", "dispatch", "gather", "expert_up", "expert_down", "shared_up", "shared_down",
                "combine"]
 
@@ -46,6 +48,10 @@ class LayerDesc(ctypes.Structure):
         ("routed_scaling_factor", ctypes.c_float), ("eps", ctypes.c_float), ("I_sh", ctypes.c_int),
         ("n_group", ctypes.c_int), ("topk_group", ctypes.c_int),
     ]
+
+
+class DenseDesc(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("dtype", "T", "D", "I", "act", "has_bias")]
 
 
 class Weights(ctypes.Structure):
@@ -93,13 +99,18 @@ _decl("moe_expert_ffn_workspace_size", _sz, [_P(LayerDesc)])
 _decl("moe_expert_ffn", _i, [_P(LayerDesc), _P(Weights), _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
 _decl("moe_shared_expert_workspace_size", _sz, [_P(LayerDesc)])
 _decl("moe_shared_expert", _i, [_P(LayerDesc), _P(Weights), _vp, _vp, _vp, _sz, _vp])
-_decl("moe_combine", _i, [_P(LayerDesc), _vp, _vp, _vp, _vp, _vp])
+_decl("moe_combine", _i, [_P(LayerDesc), _vp, _vp, _vp, _vp, _vp, _vp])
 _decl("moe_workspace_size", _sz, [_P(LayerDesc)])
 _decl("moe_workspace_layout", _i, [_P(LayerDesc), _P(WsLayout)])
 _decl("moe_forward", _i, [_P(LayerDesc), _P(Weights), _vp, _vp, _vp, _sz, _vp])
 _decl("moe_forward_profiled", _i, [_P(LayerDesc), _P(Weights), _vp, _vp, _vp, _sz, _vp, _P(_vp), _i])
 _decl("moe_forward_launch_count", _i, [_P(LayerDesc)])
 _decl("moe_algorithmic_work", None, [_P(LayerDesc), _vp, _P(ctypes.c_double), _P(ctypes.c_double)])
+_decl("moe_forward_add", _i, [_P(LayerDesc), _P(Weights), _vp, _vp, _vp, _vp, _sz, _vp])
+_decl("moe_dense_ffn_workspace_size", _sz, [_P(DenseDesc)])
+_decl("moe_dense_ffn", _i, [_P(DenseDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
+_decl("moe_dense_ffn_profiled", _i, [_P(DenseDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp,
+                                     _P(_vp), _i])
 
 
 def _status_name(s: int) -> str:
@@ -171,8 +182,9 @@ def moe_shared_expert(desc, weights, x, y_sh, ws, ws_bytes, stream=None):
                                                       y_sh, ws, ws_bytes, stream))
 
 
-def moe_combine(desc, out_perm, slot_of, shared_out, y, stream=None):
-    _check("moe_combine", lib.moe_combine(ctypes.byref(desc), out_perm, slot_of, shared_out, y, stream))
+def moe_combine(desc, out_perm, slot_of, shared_out, addend, y, stream=None):
+    _check("moe_combine", lib.moe_combine(ctypes.byref(desc), out_perm, slot_of, shared_out, addend, y,
+                                          stream))
 
 
 def moe_workspace_size(desc: LayerDesc) -> int:
@@ -212,3 +224,24 @@ def moe_algorithmic_work(desc: LayerDesc, counts_host=None):
         ptr = counts_host.ctypes.data
     lib.moe_algorithmic_work(ctypes.byref(desc), ptr, ctypes.byref(f), ctypes.byref(b))
     return f.value, b.value
+
+
+def moe_forward_add(desc, weights, x, addend, y, ws, ws_bytes, stream=None):
+    _check("moe_forward_add", lib.moe_forward_add(ctypes.byref(desc), ctypes.byref(weights), x, addend, y,
+                                                  ws, ws_bytes, stream))
+
+
+def moe_dense_ffn_workspace_size(desc: DenseDesc) -> int:
+    return lib.moe_dense_ffn_workspace_size(ctypes.byref(desc))
+
+
+def moe_dense_ffn(desc, w1, b1, w2, b2, x, addend, y, ws, ws_bytes, stream=None):
+    _check("moe_dense_ffn", lib.moe_dense_ffn(ctypes.byref(desc), w1, b1, w2, b2, x, addend, y, ws,
+                                              ws_bytes, stream))
+
+
+def moe_dense_ffn_profiled(desc, w1, b1, w2, b2, x, addend, y, ws, ws_bytes, stream, events):
+    """events: NUM_DENSE_EVENTS raw cudaEvent_t handles (ints)."""
+    arr = (ctypes.c_void_p * len(events))(*events)
+    _check("moe_dense_ffn_profiled", lib.moe_dense_ffn_profiled(
+        ctypes.byref(desc), w1, b1, w2, b2, x, addend, y, ws, ws_bytes, stream, arr, len(events)))

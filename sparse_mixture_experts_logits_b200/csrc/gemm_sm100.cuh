@@ -44,6 +44,8 @@ enum GemmEpilogue : int {
   EPI_COMBINE = 4,     // out bf16 = acc + sum_j src[slot_of[r, j], n] (shared down + combine,
                        //            src fp32)
   EPI_STORE_BF16 = 5,  // out bf16 = acc                         (standalone shared down projection)
+  EPI_BIAS_ADD = 6,    // out (layer dtype) = acc + b[n] + addend[r, n]   (dense FFN down projection;
+                       //            bias and addend optional)
 };
 
 constexpr int kBK = 64;

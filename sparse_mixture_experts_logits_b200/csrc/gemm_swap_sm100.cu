@@ -105,6 +105,7 @@ cudaError_t launch_gemm_swap(const SwapLaunch& L, cudaStream_t s) {
   a.out = L.out;
   a.row_scale = L.row_scale;
   a.bias = static_cast<const __nv_bfloat16*>(L.bias);
+  a.addend = static_cast<const __nv_bfloat16*>(L.addend);
   a.status = L.status;
   // token tiles of a segment: ceil(rows_g / 256) at most, so the total is at most rows/256 + #groups
   const long long tt_ub = L.offsets ? L.rows / kSwMaxTile + std::min<long long>(L.num_groups, L.rows)
@@ -116,6 +117,7 @@ cudaError_t launch_gemm_swap(const SwapLaunch& L, cudaStream_t s) {
     case EPI_SCALE_BIAS: return launch_swap_epi<EPI_SCALE_BIAS>(tw, tx, a, tiles_ub, s);
     case EPI_STORE_F32: return launch_swap_epi<EPI_STORE_F32>(tw, tx, a, tiles_ub, s);
     case EPI_STORE_BF16: return launch_swap_epi<EPI_STORE_BF16>(tw, tx, a, tiles_ub, s);
+    case EPI_BIAS_ADD: return launch_swap_epi<EPI_BIAS_ADD>(tw, tx, a, tiles_ub, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -58,7 +58,8 @@ struct SwapArgs {
   int ldo;
   void* out;
   const float* row_scale;      // EPI_SCALE_BIAS: [rows]
-  const __nv_bfloat16* bias;   // EPI_GELU_BIAS / EPI_SCALE_BIAS: [G, out_cols] or nullptr
+  const __nv_bfloat16* bias;   // EPI_GELU_BIAS / EPI_SCALE_BIAS / EPI_BIAS_ADD: [G, out_cols] or nullptr
+  const __nv_bfloat16* addend; // EPI_BIAS_ADD: [rows, ldo] or nullptr
   int* status;
 };
 
@@ -292,7 +293,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                               : t.wt * args.cols_per_tile + static_cast<int>(rank) * 128 + m;
       const bool col_ok = col < args.out_cols;
       float bias = 0.f;
-      if constexpr (EPI == EPI_GELU_BIAS || EPI == EPI_SCALE_BIAS) {
+      if constexpr (EPI == EPI_GELU_BIAS || EPI == EPI_SCALE_BIAS || EPI == EPI_BIAS_ADD) {
         if (args.bias != nullptr && col_ok)
           bias = __bfloat162float(args.bias[static_cast<size_t>(t.g) * args.out_cols + col]);
       }
@@ -332,6 +333,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             float v = __uint_as_float(r[i]) + bias;
             if constexpr (EPI == EPI_GELU_BIAS) v = gelu_tanh_fast(v);
             if constexpr (EPI == EPI_SCALE_BIAS) v *= __shfl_sync(0xffffffffu, rs, i);
+            if constexpr (EPI == EPI_BIAS_ADD) {
+              if (args.addend != nullptr && col_ok && i < nv)
+                v += __bfloat162float(args.addend[(row0 + c + i) * args.ldo + col]);
+            }
             if (col_ok && i < nv) swap_store<EPI>(args, row0 + c + i, col, v);
           }
         }

@@ -35,9 +35,10 @@ cudaError_t launch_permute(const int32_t* topk_idx, const float* topk_w, int T, 
 // Gathers rows r < min(rows, *n_rows) (n_rows device, may be null).
 cudaError_t launch_gather_rows(const void* x, const int32_t* row_token, const int32_t* n_rows, void* x_perm,
                                int rows, int T, int D, int elem_bytes, int* status, cudaStream_t s);
+// y = sum of the k routed rows (+ shared_out) (+ addend, layer dtype), in fp32, rounded once.
 cudaError_t launch_combine(int dtype, const void* out_perm, const int32_t* slot_of,
-                           const void* shared_out, bool shared_f32, void* y, int T, int D, int k,
-                           cudaStream_t s);
+                           const void* shared_out, bool shared_f32, const void* addend, void* y, int T,
+                           int D, int k, cudaStream_t s);
 
 // gemm_sm100.cu: grouped bf16 GEMM on tcgen05.  `epi` is a GemmEpilogue.
 struct GemmLaunch {
@@ -77,6 +78,7 @@ struct SwapLaunch {
   void* out;
   const float* row_scale;
   const void* bias;
+  const void* addend;        // EPI_BIAS_ADD: bf16 [rows, ldo] or nullptr
   int* status;
 };
 cudaError_t launch_gemm_swap(const SwapLaunch& L, cudaStream_t s);
@@ -98,6 +100,7 @@ struct SimtLaunch {
   const float* comb_src;
   const int32_t* slot_of;
   int k;
+  const float* addend;  // EPI_BIAS_ADD: [rows, ldo] or nullptr
 };
 cudaError_t launch_simt_gemm(const SimtLaunch& L, cudaStream_t s);
 

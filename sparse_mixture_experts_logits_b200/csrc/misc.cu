@@ -60,14 +60,15 @@ cudaError_t launch_gather_rows(const void* x, const int32_t* row_token, const in
   return cudaGetLastError();
 }
 
-// y[t, :] = sum_j out_perm[slot_of[t, j], :] (+ shared[t, :]) in fp32, in
+// y[t, :] = sum_j out_perm[slot_of[t, j], :] (+ shared[t, :]) (+ addend[t, :]) in fp32, in
 // slot order (slots < 0, sentinel pairs, add nothing), rounded once.  out_perm is fp32; shared is fp32 or the layer's
 // type; y has the layer's type.  Block (token, 128 four-column groups); every
 // row read is contiguous, and the k rows of a token are loaded together.
 template <typename TY, typename TS>
 __global__ void __launch_bounds__(128) combine_vec4_kernel(const float4* __restrict__ out_perm,
                                                            const int32_t* __restrict__ slot_of,
-                                                           const TS* __restrict__ shared, TY* __restrict__ y,
+                                                           const TS* __restrict__ shared,
+                                                           const TY* __restrict__ addend, TY* __restrict__ y,
                                                            int D4, int k) {
   __shared__ int s_slot[kMaxTopK];
   const int t = blockIdx.x;
@@ -86,6 +87,11 @@ __global__ void __launch_bounds__(128) combine_vec4_kernel(const float4* __restr
       acc.x += to_f32(shared[e]); acc.y += to_f32(shared[e + 1]);
       acc.z += to_f32(shared[e + 2]); acc.w += to_f32(shared[e + 3]);
     }
+    if (addend != nullptr) {
+      const size_t e = (static_cast<size_t>(t) * D4 + v) * 4;
+      acc.x += to_f32(addend[e]); acc.y += to_f32(addend[e + 1]);
+      acc.z += to_f32(addend[e + 2]); acc.w += to_f32(addend[e + 3]);
+    }
     const size_t o = (static_cast<size_t>(t) * D4 + v) * 4;
     if constexpr (sizeof(TY) == 2) {
       __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
@@ -102,7 +108,8 @@ __global__ void __launch_bounds__(128) combine_vec4_kernel(const float4* __restr
 // Any D: one element per thread step.
 template <typename TY, typename TS>
 __global__ void combine_kernel(const float* __restrict__ out_perm, const int32_t* __restrict__ slot_of,
-                               const TS* __restrict__ shared, TY* __restrict__ y, int D, int k) {
+                               const TS* __restrict__ shared, const TY* __restrict__ addend,
+                               TY* __restrict__ y, int D, int k) {
   const int t = blockIdx.x;
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
     float acc = 0.f;
@@ -111,34 +118,37 @@ __global__ void combine_kernel(const float* __restrict__ out_perm, const int32_t
       if (slot >= 0) acc += out_perm[static_cast<size_t>(slot) * D + d];
     }
     if (shared != nullptr) acc += to_f32(shared[static_cast<size_t>(t) * D + d]);
+    if (addend != nullptr) acc += to_f32(addend[static_cast<size_t>(t) * D + d]);
     y[static_cast<size_t>(t) * D + d] = from_f32<TY>(acc);
   }
 }
 
 template <typename TY, typename TS>
-static cudaError_t combine_typed(const float* op, const int32_t* slot_of, const void* shared, void* y,
-                                 int T, int D, int k, cudaStream_t s) {
+static cudaError_t combine_typed(const float* op, const int32_t* slot_of, const void* shared,
+                                 const void* addend, void* y, int T, int D, int k, cudaStream_t s) {
   if (D % 4 == 0) {
     // few tokens: spread a row's columns over blocks too
     dim3 grid(T, T >= 1024 ? 1 : (D / 4 + 127) / 128);
     combine_vec4_kernel<TY, TS><<<grid, 128, 0, s>>>(reinterpret_cast<const float4*>(op), slot_of,
-                                                  static_cast<const TS*>(shared), static_cast<TY*>(y), D / 4, k);
+                                                  static_cast<const TS*>(shared), static_cast<const TY*>(addend),
+                                                  static_cast<TY*>(y), D / 4, k);
   } else {
     combine_kernel<TY, TS><<<T, 128, 0, s>>>(op, slot_of, static_cast<const TS*>(shared),
-                                             static_cast<TY*>(y), D, k);
+                                             static_cast<const TY*>(addend), static_cast<TY*>(y), D, k);
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_combine(int dtype, const void* out_perm, const int32_t* slot_of,
-                           const void* shared_out, bool shared_f32, void* y, int T, int D, int k,
-                           cudaStream_t s) {
+                           const void* shared_out, bool shared_f32, const void* addend, void* y, int T,
+                           int D, int k, cudaStream_t s) {
   const float* op = static_cast<const float*>(out_perm);
   if (dtype == MOE_DTYPE_BF16) {
-    return shared_f32 ? combine_typed<__nv_bfloat16, float>(op, slot_of, shared_out, y, T, D, k, s)
-                      : combine_typed<__nv_bfloat16, __nv_bfloat16>(op, slot_of, shared_out, y, T, D, k, s);
+    return shared_f32
+               ? combine_typed<__nv_bfloat16, float>(op, slot_of, shared_out, addend, y, T, D, k, s)
+               : combine_typed<__nv_bfloat16, __nv_bfloat16>(op, slot_of, shared_out, addend, y, T, D, k, s);
   }
-  return combine_typed<float, float>(op, slot_of, shared_out, y, T, D, k, s);
+  return combine_typed<float, float>(op, slot_of, shared_out, addend, y, T, D, k, s);
 }
 
 }  // namespace moe

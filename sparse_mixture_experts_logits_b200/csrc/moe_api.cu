@@ -484,14 +484,149 @@ moe_status_t moe_shared_expert(const moe_layer_desc_t* d, const moe_weights_t* w
 }
 
 moe_status_t moe_combine(const moe_layer_desc_t* d, const void* out_perm, const int32_t* slot_of,
-                         const void* shared_out, void* y, void* stream) {
+                         const void* shared_out, const void* addend, void* y, void* stream) {
   MOE_TRY(check_desc(d));
   if (d->T == 0) return MOE_OK;
   if (!out_perm || !slot_of || !y) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_device());
-  MOE_CUDA(launch_combine(d->dtype, out_perm, slot_of, shared_out, false, y, d->T, d->D, d->k,
+  MOE_CUDA(launch_combine(d->dtype, out_perm, slot_of, shared_out, false, addend, y, d->T, d->D, d->k,
                           static_cast<cudaStream_t>(stream)));
   return MOE_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------ dense FFN layer
+
+namespace {
+
+moe_status_t check_dense(const moe_dense_desc_t* d) {
+  if (d == nullptr) return MOE_ERR_INVALID_ARG;
+  if (d->T < 0 || d->D < 1 || d->I < 1) return MOE_ERR_INVALID_ARG;
+  if (d->dtype != MOE_DTYPE_F32 && d->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (d->act != MOE_ACT_GELU_TANH && d->act != MOE_ACT_SWIGLU) return MOE_ERR_INVALID_ARG;
+  if (d->dtype == MOE_DTYPE_BF16 && (d->D % 16 != 0 || d->I % 16 != 0)) return MOE_ERR_UNSUPPORTED;
+  const long long wide = std::max<long long>(d->D, 2ll * d->I);
+  if (static_cast<long long>(d->T) * wide >= (1ll << 40) || d->T >= (1 << 30)) return MOE_ERR_UNSUPPORTED;
+  if (2ll * d->I * std::max(d->D, d->I) >= (1ll << 40)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+struct DenseWs { size_t status, h, total; };
+DenseWs dense_layout(const moe_dense_desc_t* d) {
+  Carve c;
+  DenseWs L;
+  L.status = c.take(4);
+  L.h = c.take(static_cast<size_t>(d->T) * d->I * esize(d->dtype));
+  L.total = c.off;
+  return L;
+}
+
+moe_status_t dense_impl(const moe_dense_desc_t* d, const void* w1, const void* b1, const void* w2,
+                        const void* b2, const void* x, const void* addend, void* y, void* ws,
+                        size_t ws_bytes, cudaStream_t s, void* const* events) {
+  MOE_TRY(check_dense(d));
+  if (d->T == 0) return MOE_OK;
+  const bool swiglu = d->act == MOE_ACT_SWIGLU;
+  const bool bias = !swiglu && d->has_bias;
+  if (!w1 || !w2 || !x || !y || !ws || !aligned_ws(ws)) return MOE_ERR_INVALID_ARG;
+  if (bias && (!b1 || !b2)) return MOE_ERR_INVALID_ARG;
+  const DenseWs L = dense_layout(d);
+  if (ws_bytes < L.total) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_device());
+  Marks mk;
+  mk.ev = events;
+  mk.s = s;
+  int* status = at<int*>(ws, L.status);
+  void* h = at<void*>(ws, L.h);
+  MOE_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
+  MOE_TRY(mk.at(0));
+  if (d->dtype == MOE_DTYPE_BF16) {
+    SwapLaunch g1{};
+    g1.W = w1; g1.w_rows = swiglu ? 2ll * d->I : d->I;
+    g1.X = x; g1.x_rows = d->T;
+    g1.K = d->D;
+    g1.num_groups = 1; g1.offsets = nullptr; g1.rows = d->T;
+    if (swiglu) {
+      g1.epi = EPI_SWIGLU;
+      g1.w_rows_per_group = 2 * d->I; g1.w_tile_step = 128; g1.w_hi_offset = d->I; g1.w_cta_step = 64;
+      g1.cols_per_tile = 128;
+    } else {
+      g1.epi = EPI_GELU_BIAS;
+      g1.w_rows_per_group = d->I; g1.w_tile_step = 256; g1.w_hi_offset = 64; g1.w_cta_step = 128;
+      g1.cols_per_tile = 256;
+      g1.bias = bias ? b1 : nullptr;
+    }
+    g1.w_tiles = (d->I + g1.cols_per_tile - 1) / g1.cols_per_tile;
+    g1.out_cols = d->I; g1.ldo = d->I; g1.out = h;
+    g1.status = status;
+    MOE_CUDA(launch_gemm_swap(g1, s));
+    MOE_TRY(mk.at(1));
+    SwapLaunch g2{};
+    g2.epi = EPI_BIAS_ADD;
+    g2.W = w2; g2.w_rows = d->D;
+    g2.X = h; g2.x_rows = d->T;
+    g2.K = d->I;
+    g2.num_groups = 1; g2.offsets = nullptr; g2.rows = d->T;
+    g2.w_rows_per_group = d->D; g2.w_tile_step = 256; g2.w_hi_offset = 64; g2.w_cta_step = 128;
+    g2.cols_per_tile = 256; g2.w_tiles = (d->D + 255) / 256;
+    g2.out_cols = d->D; g2.ldo = d->D; g2.out = y;
+    g2.bias = bias ? b2 : nullptr;
+    g2.addend = addend;
+    g2.status = status;
+    MOE_CUDA(launch_gemm_swap(g2, s));
+    MOE_TRY(mk.at(2));
+  } else {
+    SimtLaunch g1{};
+    g1.epi = swiglu ? EPI_SWIGLU : EPI_GELU_BIAS;
+    g1.A = static_cast<const float*>(x); g1.K = d->D;
+    g1.B = static_cast<const float*>(w1);
+    g1.num_groups = 1; g1.offsets = nullptr; g1.rows = d->T;
+    g1.b_rows_per_group = swiglu ? 2 * d->I : d->I; g1.swiglu_hi = swiglu ? d->I : 0;
+    g1.out_cols = d->I; g1.ldo = d->I; g1.out = static_cast<float*>(h);
+    g1.bias = bias ? static_cast<const float*>(b1) : nullptr;
+    MOE_CUDA(launch_simt_gemm(g1, s));
+    MOE_TRY(mk.at(1));
+    SimtLaunch g2{};
+    g2.epi = EPI_BIAS_ADD;
+    g2.A = static_cast<const float*>(h); g2.K = d->I;
+    g2.B = static_cast<const float*>(w2);
+    g2.num_groups = 1; g2.offsets = nullptr; g2.rows = d->T;
+    g2.b_rows_per_group = d->D;
+    g2.out_cols = d->D; g2.ldo = d->D; g2.out = static_cast<float*>(y);
+    g2.bias = bias ? static_cast<const float*>(b2) : nullptr;
+    g2.addend = static_cast<const float*>(addend);
+    MOE_CUDA(launch_simt_gemm(g2, s));
+    MOE_TRY(mk.at(2));
+  }
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_dense_ffn_workspace_size(const moe_dense_desc_t* d) {
+  if (check_dense(d) != MOE_OK) return 0;
+  return dense_layout(d).total;
+}
+
+moe_status_t moe_dense_ffn(const moe_dense_desc_t* d, const void* w1, const void* b1, const void* w2,
+                           const void* b2, const void* x, const void* addend, void* y, void* ws,
+                           size_t ws_bytes, void* stream) {
+  return dense_impl(d, w1, b1, w2, b2, x, addend, y, ws, ws_bytes, static_cast<cudaStream_t>(stream),
+                    nullptr);
+}
+
+moe_status_t moe_dense_ffn_profiled(const moe_dense_desc_t* d, const void* w1, const void* b1,
+                                    const void* w2, const void* b2, const void* x, const void* addend,
+                                    void* y, void* ws, size_t ws_bytes, void* stream,
+                                    void* const* events, int n_events) {
+  if (events == nullptr || n_events != MOE_NUM_DENSE_EVENTS) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < n_events; ++i)
+    if (events[i] == nullptr) return MOE_ERR_INVALID_ARG;
+  return dense_impl(d, w1, b1, w2, b2, x, addend, y, ws, ws_bytes, static_cast<cudaStream_t>(stream),
+                    events);
 }
 
 size_t moe_workspace_size(const moe_layer_desc_t* d) {
@@ -507,7 +642,7 @@ moe_status_t moe_workspace_layout(const moe_layer_desc_t* d, moe_ws_layout_t* ou
 }
 
 static moe_status_t forward_impl(const moe_layer_desc_t* d, const moe_weights_t* w, const void* x,
-                                 void* y, void* ws, size_t ws_bytes, cudaStream_t s,
+                                 const void* addend, void* y, void* ws, size_t ws_bytes, cudaStream_t s,
                                  void* const* events) {
   MOE_TRY(check_desc(d));
   MOE_TRY(check_weights(d, w, true, true));
@@ -548,14 +683,20 @@ static moe_status_t forward_impl(const moe_layer_desc_t* d, const moe_weights_t*
     MOE_TRY(mk.at(6));
     MOE_TRY(mk.at(7));
   }
-  MOE_CUDA(launch_combine(d->dtype, out_perm, slot_of, y_sh, true, y, d->T, d->D, d->k, s));
+  MOE_CUDA(launch_combine(d->dtype, out_perm, slot_of, y_sh, true, addend, y, d->T, d->D, d->k, s));
   MOE_TRY(mk.at(8));
   return MOE_OK;
 }
 
 moe_status_t moe_forward(const moe_layer_desc_t* d, const moe_weights_t* w, const void* x, void* y,
                          void* ws, size_t ws_bytes, void* stream) {
-  return forward_impl(d, w, x, y, ws, ws_bytes, static_cast<cudaStream_t>(stream), nullptr);
+  return forward_impl(d, w, x, nullptr, y, ws, ws_bytes, static_cast<cudaStream_t>(stream), nullptr);
+}
+
+moe_status_t moe_forward_add(const moe_layer_desc_t* d, const moe_weights_t* w, const void* x,
+                             const void* addend, void* y, void* ws, size_t ws_bytes, void* stream) {
+  if (d != nullptr && d->T > 0 && addend == nullptr) return MOE_ERR_INVALID_ARG;
+  return forward_impl(d, w, x, addend, y, ws, ws_bytes, static_cast<cudaStream_t>(stream), nullptr);
 }
 
 moe_status_t moe_forward_profiled(const moe_layer_desc_t* d, const moe_weights_t* w, const void* x,
@@ -564,7 +705,7 @@ moe_status_t moe_forward_profiled(const moe_layer_desc_t* d, const moe_weights_t
   if (events == nullptr || n_events != MOE_NUM_STAGE_EVENTS) return MOE_ERR_INVALID_ARG;
   for (int i = 0; i < n_events; ++i)
     if (events[i] == nullptr) return MOE_ERR_INVALID_ARG;
-  return forward_impl(d, w, x, y, ws, ws_bytes, static_cast<cudaStream_t>(stream), events);
+  return forward_impl(d, w, x, nullptr, y, ws, ws_bytes, static_cast<cudaStream_t>(stream), events);
 }
 
 int moe_forward_launch_count(const moe_layer_desc_t* d) {

@@ -29,6 +29,16 @@ def desc_from_config(cfg: dict, T: int | None = None) -> abi.LayerDesc:
     return d
 
 
+def dense_desc_from_config(cfg: dict, T: int | None = None) -> abi.DenseDesc:
+    d = abi.DenseDesc()
+    d.dtype = _DTYPES[cfg["dtype"]]
+    d.T = cfg["T"] if T is None else T
+    d.D, d.I = cfg["D"], cfg["I"]
+    d.act = _ACTS[cfg["act"]]
+    d.has_bias = int(bool(cfg.get("has_bias", 0)))
+    return d
+
+
 def _ptr(t):
     return None if t is None else t.data_ptr()
 
@@ -70,11 +80,17 @@ class MoELayer:
     def ws_ptr(self) -> int:
         return self.ws.data_ptr() + self._ws_off
 
-    def forward(self, x: torch.Tensor, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    def forward(self, x: torch.Tensor, y: torch.Tensor | None = None, stream=None,
+                addend: torch.Tensor | None = None) -> torch.Tensor:
+        """y = MoE-FFN(x), or addend + MoE-FFN(x) when ``addend`` is given."""
         if y is None:
             y = torch.empty_like(x)
-        abi.moe_forward(self.desc, self.weights, x.data_ptr(), y.data_ptr(), self.ws_ptr, self.ws_bytes,
-                        _stream_handle(stream))
+        if addend is None:
+            abi.moe_forward(self.desc, self.weights, x.data_ptr(), y.data_ptr(), self.ws_ptr, self.ws_bytes,
+                            _stream_handle(stream))
+        else:
+            abi.moe_forward_add(self.desc, self.weights, x.data_ptr(), addend.data_ptr(), y.data_ptr(),
+                                self.ws_ptr, self.ws_bytes, _stream_handle(stream))
         return y
 
     def device_status(self, stream=None) -> int:
@@ -98,3 +114,41 @@ class MoELayer:
             n *= s
         nbytes = n * torch.empty((), dtype=dt).element_size()
         return self.ws[off:off + nbytes].view(dt).view(*shape)
+
+
+class DenseLayer:
+    """One dense FFN layer (w1, b1, w2, b2 device tensors, kept alive here)."""
+
+    def __init__(self, cfg: dict, tensors: dict, T: int | None = None):
+        self.cfg = cfg
+        self.tensors = tensors
+        self.desc = dense_desc_from_config(cfg, T)
+        for name in ("w1", "b1", "w2", "b2"):
+            v = tensors.get(name)
+            if v is not None and not v.is_contiguous():
+                raise ValueError(f"{name} must be contiguous")
+        self.ws_bytes = abi.moe_dense_ffn_workspace_size(self.desc)
+        if self.ws_bytes == 0:
+            raise abi.MoEError("moe_dense_ffn_workspace_size", abi.MOE_ERR_INVALID_ARG)
+        self.ws = torch.zeros(self.ws_bytes + 256, dtype=torch.uint8, device=tensors["w1"].device)
+        self._ws_off = (-self.ws.data_ptr()) % 256
+
+    @property
+    def ws_ptr(self) -> int:
+        return self.ws.data_ptr() + self._ws_off
+
+    def args(self):
+        t = self.tensors
+        return (_ptr(t["w1"]), _ptr(t.get("b1")), _ptr(t["w2"]), _ptr(t.get("b2")))
+
+    def forward(self, x: torch.Tensor, addend: torch.Tensor | None = None, y: torch.Tensor | None = None,
+                stream=None) -> torch.Tensor:
+        """y = (addend +) FFN(x)."""
+        if y is None:
+            y = torch.empty_like(x)
+        abi.moe_dense_ffn(self.desc, *self.args(), x.data_ptr(), _ptr(addend), y.data_ptr(), self.ws_ptr,
+                          self.ws_bytes, _stream_handle(stream))
+        return y
+
+    def device_status(self, stream=None) -> int:
+        return abi.moe_device_status(self.ws_ptr, _stream_handle(stream))

@@ -112,7 +112,7 @@ def test_zero_tokens_launch_nothing(B):
     B.moe_forward(d, w, None, None, None, 0)
     B.moe_route_topk(None, None, None, 0, 64, 8, 2, 1, 0, 1, 1.0, 1e-20, 1, 1, None, None, None, 0)
     B.moe_expert_ffn(d, w, None, None, None, None, None, None, 0)
-    B.moe_combine(d, None, None, None, None)
+    B.moe_combine(d, None, None, None, None, None)
 
 
 def test_workspace_layout_is_aligned_and_ordered(B):
@@ -125,6 +125,28 @@ def test_workspace_layout_is_aligned_and_ordered(B):
         assert offs == sorted(offs) and L.total >= offs[-1] + d.T * d.k * d.D * (2 if d.dtype else 4)
         assert B.moe_workspace_size(d) == L.total
         assert B.moe_expert_ffn_workspace_size(d) > 0
+
+
+def test_dense_workspace_and_bad_descs(B):
+    for name in ms.dense_config_names():
+        cfg = ms.get_config(name)
+        d = B.dense_desc_from_config(cfg)
+        es = 2 if cfg["dtype"] == "bf16" else 4
+        assert B.moe_dense_ffn_workspace_size(d) >= cfg["T"] * cfg["I"] * es
+    d = B.dense_desc_from_config(ms.get_config("glm_dense_small_bf16"))
+    for field, value, status in [("D", 24, 2), ("I", 40, 2), ("act", 7, 1), ("dtype", 5, 2), ("T", -1, 1)]:
+        bad = B.DenseDesc.from_buffer_copy(d)
+        setattr(bad, field, value)
+        assert B.moe_dense_ffn_workspace_size(bad) == 0
+        with pytest.raises(B.MoEError) as e:
+            B.moe_dense_ffn(bad, 256, None, 256, None, 256, None, 256, 256, 1 << 30)
+        assert e.value.status == status
+    # T = 0 launches nothing; missing weights are rejected before any launch
+    zero = B.DenseDesc.from_buffer_copy(d)
+    zero.T = 0
+    B.moe_dense_ffn(zero, None, None, None, None, None, None, None, None, 0)
+    with pytest.raises(B.MoEError):
+        B.moe_dense_ffn(d, None, None, 256, None, 256, None, 256, 256, 1 << 30)
 
 
 def test_algorithmic_work_closed_form(B):

@@ -173,7 +173,7 @@ def test_stage_entry_points_match_forward(B):
     B.moe_shared_expert(d, layer.weights, inp["x"].data_ptr(), y_sh.data_ptr(), wsh.data_ptr(),
                         wsh.numel(), s)
     y_c = torch.empty(T, D, dtype=torch.bfloat16, device=dev)
-    B.moe_combine(d, out_perm.data_ptr(), slot_of.data_ptr(), y_sh.data_ptr(), y_c.data_ptr(), s)
+    B.moe_combine(d, out_perm.data_ptr(), slot_of.data_ptr(), y_sh.data_ptr(), None, y_c.data_ptr(), s)
     torch.cuda.synchronize()
     sh_ref = oracle.shared_expert(xs, np64(inp["sh_w1"]), np64(inp["sh_w2"]))
     m = oracle.error_metrics(np64(y_sh), sh_ref)
@@ -254,7 +254,7 @@ def test_sentinel_pairs_are_dispatched_nowhere(B, name, frac):
                             wsh.numel(), s)
     y = torch.empty_like(inp["x"])
     B.moe_combine(d, out_perm.data_ptr(), slot_of.data_ptr(),
-                  None if shared_out is None else shared_out.data_ptr(), y.data_ptr(), s)
+                  None if shared_out is None else shared_out.data_ptr(), None, y.data_ptr(), s)
     torch.cuda.synchronize()
     shared = (np64(inp["sh_w1"]), np64(inp["sh_w2"])) if cfg.get("I_sh") else None
     from gpu_common import HostExperts

@@ -1,0 +1,75 @@
+"""The forward pass makes no host synchronisation and no allocation, so it
+can be captured once into a CUDA graph and replayed (the decode loop's way
+of removing launch overhead), and it runs on any stream."""
+import pytest
+import torch
+
+import moe_synth as ms
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def B():
+    import sparse_mixture_experts_logits_b200 as B
+    return B
+
+
+@pytest.mark.parametrize("name", ["glm45_decode_bf16", "glam_small_bf16", "glm_grouped_bf16"])
+def test_graph_replay_matches_eager(B, name):
+    cfg = ms.get_config(name)
+    inp = ms.layer_inputs(cfg, "cuda")
+    layer = B.MoELayer(cfg, inp)
+    x_static = inp["x"].clone()
+    y_eager = layer.forward(x_static)          # first call also configures the kernels
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    y_static = torch.empty_like(x_static)
+    with torch.cuda.graph(g, stream=side):
+        layer.forward(x_static, y=y_static, stream=side)
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y_static.view(torch.int16), y_eager.view(torch.int16))
+    assert layer.device_status() == 0
+    # new tokens in the captured input buffer: the replay follows them
+    x2 = ms.normal((cfg["T"], cfg["D"]), 1.0, ms._key(cfg, "x2"), "cuda", ms.act_dtype(cfg))
+    x_static.copy_(x2)
+    g.replay()
+    y2_eager = layer.forward(x2)
+    torch.cuda.synchronize()
+    assert torch.equal(y_static.view(torch.int16), y2_eager.view(torch.int16))
+
+
+def test_dense_layer_graph_replay(B):
+    cfg = ms.get_config("glm_dense_small_bf16")
+    inp = ms.dense_inputs(cfg, "cuda")
+    layer = B.DenseLayer(cfg, inp)
+    y_eager = layer.forward(inp["x"], addend=inp["addend"])
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    y_static = torch.empty_like(y_eager)
+    with torch.cuda.graph(g, stream=side):
+        layer.forward(inp["x"], addend=inp["addend"], y=y_static, stream=side)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y_static.view(torch.int16), y_eager.view(torch.int16))
+
+
+def test_forward_on_a_side_stream(B):
+    cfg = ms.get_config("glm_small_bf16")
+    inp = ms.layer_inputs(cfg, "cuda")
+    layer = B.MoELayer(cfg, inp)
+    y0 = layer.forward(inp["x"])
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        y1 = torch.empty_like(y0)
+        layer.forward(inp["x"], y=y1, stream=s)
+    s.synchronize()
+    assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))

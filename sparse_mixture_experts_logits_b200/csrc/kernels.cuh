@@ -32,6 +32,9 @@ cudaError_t launch_permute(const int32_t* topk_idx, const float* topk_w, int T, 
                            cudaStream_t s);
 
 // misc.cu
+// bf16 rows of x into dispatch order by token: x_perm[slot_of[t, j]] = x[t] (D % 8 == 0).
+cudaError_t launch_scatter_rows(const void* x, const int32_t* slot_of, void* x_perm, int T, int k, int D,
+                                int* status, cudaStream_t s);
 // Gathers rows r < min(rows, *n_rows) (n_rows device, may be null).
 cudaError_t launch_gather_rows(const void* x, const int32_t* row_token, const int32_t* n_rows, void* x_perm,
                                int rows, int T, int D, int elem_bytes, int* status, cudaStream_t s);

@@ -1,4 +1,6 @@
 // Row gather (dispatch of x into expert order) and the standalone combine.
+#include <algorithm>
+
 #include "kernels.cuh"
 
 namespace moe {
@@ -43,6 +45,43 @@ __global__ void gather_rows_f32_kernel(const float* __restrict__ x, const int32_
     const float* src = x + static_cast<size_t>(ok ? tok : 0) * D;
     for (int d = lane; d < D; d += 32) x_perm[static_cast<size_t>(r) * D + d] = ok ? src[d] : 0.f;
   }
+}
+
+// The same rows written the other way round: token t's row is read once and
+// stored at its k dispatch positions slot_of[t, j] (sentinel pairs, slot < 0,
+// are skipped; a slot >= rows is reported and skipped).  Each x row is read
+// from memory once instead of k times.
+__global__ void scatter_rows_vec_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ slot_of,
+                                        uint4* __restrict__ x_perm, int T, int k, int rows,
+                                        int vecs_per_row, int* status) {
+  const int warps_total = gridDim.x * (blockDim.x >> 5);
+  const int lane = threadIdx.x & 31;
+  for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps_total) {
+    int my_slot = -1;
+    if (lane < k) {
+      my_slot = slot_of[static_cast<size_t>(t) * k + lane];
+      if (my_slot >= rows) {
+        set_status(status, MOE_DEVERR_BAD_ROW_TOKEN);
+        my_slot = -1;
+      }
+    }
+    const uint4* src = x + static_cast<size_t>(t) * vecs_per_row;
+    for (int v = lane; v < vecs_per_row; v += 32) {
+      const uint4 val = src[v];
+      for (int j = 0; j < k; ++j) {
+        const int slot = __shfl_sync(0xffffffffu, my_slot, j);
+        if (slot >= 0) x_perm[static_cast<size_t>(slot) * vecs_per_row + v] = val;
+      }
+    }
+  }
+}
+
+cudaError_t launch_scatter_rows(const void* x, const int32_t* slot_of, void* x_perm, int T, int k, int D,
+                                int* status, cudaStream_t s) {
+  const int blocks = std::max(1, std::min((T + 7) / 8, 4 * num_sms()));
+  scatter_rows_vec_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(x), slot_of,
+                                                 static_cast<uint4*>(x_perm), T, k, T * k, D / 8, status);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_gather_rows(const void* x, const int32_t* row_token, const int32_t* n_rows, void* x_perm,

@@ -232,17 +232,22 @@ moe_status_t run_route(const void* x, const void* w_r, const float* e_bias, int 
   return MOE_OK;
 }
 
+// slot_of (may be null): when given, x is copied into dispatch order by token
+// (each row read once) instead of by dispatch row.
 moe_status_t run_experts(const moe_layer_desc_t* d, const moe_weights_t* w, const void* x,
                          const int32_t* offsets, const int32_t* row_token, const float* row_w,
                          void* out_perm, void* x_perm, void* h, int* status, cudaStream_t s,
-                         const Marks& mk = Marks()) {
+                         const Marks& mk = Marks(), const int32_t* slot_of = nullptr) {
   const int pairs = d->T * d->k;
   const bool swiglu = d->act == MOE_ACT_SWIGLU;
   const int n1 = swiglu ? 2 * d->I : d->I;
   const void* b1 = (!swiglu && d->has_bias) ? w->b1 : nullptr;
   const void* b2 = (!swiglu && d->has_bias) ? w->b2 : nullptr;
   if (d->dtype == MOE_DTYPE_BF16) {
-    MOE_CUDA(launch_gather_rows(x, row_token, offsets + d->M, x_perm, pairs, d->T, d->D, 2, status, s));
+    if (slot_of != nullptr)
+      MOE_CUDA(launch_scatter_rows(x, slot_of, x_perm, d->T, d->k, d->D, status, s));
+    else
+      MOE_CUDA(launch_gather_rows(x, row_token, offsets + d->M, x_perm, pairs, d->T, d->D, 2, status, s));
     MOE_TRY(mk.at(3));
     SwapLaunch g1{};
     g1.W = w->w1; g1.w_rows = static_cast<long long>(d->M) * n1;
@@ -673,8 +678,12 @@ static moe_status_t forward_impl(const moe_layer_desc_t* d, const moe_weights_t*
   MOE_CUDA(launch_permute(idx, tw, d->T, d->k, d->M, counts, offsets, slot_of, row_token, row_w,
                           at<int32_t*>(ws, L.chunk_counts), at<int32_t*>(ws, L.chunk_base), status, s));
   MOE_TRY(mk.at(2));
+  // x larger than half the L2: copy it into dispatch order by token, so that each row is read
+  // from HBM once (measured: GLM-4.5 prefill 0.43 -> 0.30 ms); smaller x is read through L2
+  // either way and the per-row gather has more parallelism (decode, GLaM)
+  const bool by_token = static_cast<double>(d->T) * d->D * esize(d->dtype) > 64.0 * 1024 * 1024;
   MOE_TRY(run_experts(d, w, x, offsets, row_token, row_w, out_perm, at<void*>(ws, L.x_perm),
-                      at<void*>(ws, L.h), status, s, mk));
+                      at<void*>(ws, L.h), status, s, mk, by_token ? slot_of : nullptr));
   void* y_sh = nullptr;
   if (d->I_sh > 0) {
     y_sh = at<void*>(ws, L.y_sh);

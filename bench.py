@@ -388,7 +388,10 @@ def run_ours(args):
         "gpu_launches": B.moe_forward_launch_count(layer.desc) * K,
         "clocks": clocks,
         "routing": {"touched_experts": int((counts > 0).sum()), "max_over_mean":
-                    float(counts.max() / max(1e-9, counts.mean()))},
+                    float(counts.max() / max(1e-9, counts.mean())),
+                    "min": int(counts.min()), "median": float(np.median(counts)), "max": int(counts.max()),
+                    "cv": float(counts.std() / max(1e-9, counts.mean()))},
+        "reporting": glam_reporting(cfg, stage_ms, ms_step),
     }
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(cfg, inp, args.cpu_seconds)
@@ -396,6 +399,25 @@ def run_ours(args):
     del layer
     if dist is not None:
         dist.destroy_process_group()
+
+
+def glam_reporting(cfg, stage_ms, ms_step):
+    """The quantities the GLaM note's "Capacity, Active Compute, and
+    Reporting" table keeps apart: total parameters, active parameters per
+    token, FLOPs per token, routing overhead (gate, dispatch, expert batching,
+    combination) and the wall-clock cost."""
+    D, M, k, I, Ish = cfg["D"], cfg["M"], cfg["k"], cfg["I"], cfg.get("I_sh") or 0
+    swiglu = cfg["act"] == "swiglu"
+    expert = (3 if swiglu else 2) * D * I + ((I + D) if cfg.get("has_bias") and not swiglu else 0)
+    shared = 3 * D * Ish
+    router = D * M + (M if cfg.get("e_bias") is not None else 0)
+    active = router + k * expert + shared
+    matmul_active = D * M + k * (3 if swiglu else 2) * D * I + shared
+    overhead = {n: stage_ms.get(n, 0.0) for n in ("route", "dispatch", "gather", "combine")}
+    return {"total_params": router + M * expert + shared, "active_params_per_token": active,
+            "flops_per_token": 2 * matmul_active,
+            "routing_overhead_ms": overhead, "routing_overhead_share": sum(overhead.values()) / ms_step,
+            "wall_clock_ms": ms_step}
 
 
 def dense_stage_work(cfg):

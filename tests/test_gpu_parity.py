@@ -80,6 +80,11 @@ def test_group_limited_full_size_sampled(B):
     ("glm_small_bf16", dict(n_group=4, topk_group=4)),   # every group kept
     ("glm_small_bf16", dict(n_group=4, topk_group=1)),   # k = the whole kept group
     ("glam_small_bf16", dict(n_group=2, topk_group=1)),  # softmax router, groups of 4
+    ("glm_small_bf16", dict(M=1024, k=32)),              # the largest M and k the library takes
+    ("glm_small_f32", dict(M=1024, k=32, T=40)),         # the same on the fp32 path
+    ("glam_small_bf16", dict(M=64, k=32)),               # softmax router, k = 32
+    ("glam_small_bf16", dict(T=40000)),                  # many dispatch chunks, ragged tail
+    ("glm_small_bf16", dict(M=1024, k=32, n_group=32, topk_group=4)),  # 32 groups of 32
 ])
 def test_edge_cases(B, name, over):
     check_layer(B, ms.get_config(name, **over), all_tokens=True)

@@ -33,10 +33,15 @@
 
 namespace moe {
 
-constexpr int kSwStages = 6;
-constexpr int kSwATileBytes = 128 * kBK * 2;  // 128 weight rows per CTA
-constexpr int kSwBTileBytes = 128 * kBK * 2;  // up to 128 token rows per CTA
-constexpr int kSwStageBytes = kSwATileBytes + kSwBTileBytes;
+// A pipeline stage holds kSwKB consecutive k-blocks of 64: the MMA thread waits
+// once and commits once per stage.  Each barrier wait and commit costs the
+// single issuing thread as much as an N = 256 MMA takes to run, so fewer of
+// them per MMA keeps the tensor pipe fed.
+constexpr int kSwKB = 2;
+constexpr int kSwStages = 3;
+constexpr int kSwATileBytes = 128 * kBK * 2;  // 128 weight rows per CTA, one k-block
+constexpr int kSwBTileBytes = 128 * kBK * 2;  // up to 128 token rows per CTA, one k-block
+constexpr int kSwStageBytes = kSwKB * (kSwATileBytes + kSwBTileBytes);
 constexpr int kSwXPitch = 33;                 // floats per row of the gate/up hand-off buffer
 constexpr int kSwXBytes = 4 * 32 * kSwXPitch * 4;
 constexpr int kSwDynSmem = kSwStages * kSwStageBytes + kSwXBytes + 1024;
@@ -210,22 +215,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // -------------------------------------------------------- TMA producer
     uint32_t s = 0, ph = 0;
     bool ok = true;
-    constexpr uint32_t tx_bytes = 2u * kSwStageBytes;  // both CTAs: weight rows + 128 token rows
+    // both CTAs' bytes of one k-block: weight rows + 128 token rows each
+    constexpr uint32_t kb_bytes = 2u * (kSwATileBytes + kSwBTileBytes);
     for (int tile = unit; ok && tile < total; tile += units) {
       const SwapTile t = swap_decode(tile, G, s_tstart, s_off, args.w_tiles);
       const int x_row = s_off[t.g] + t.tok0 + static_cast<int>(rank) * (t.n >> 1);
       const int w_base = t.g * args.w_rows_per_group + t.wt * args.w_tile_step +
                          static_cast<int>(rank) * args.w_cta_step;
-      for (int kb = 0; kb < num_kb; ++kb) {
+      for (int kb0 = 0; kb0 < num_kb; kb0 += kSwKB) {
+        const int nk = min(kSwKB, num_kb - kb0);
         if (!mbar_wait_all(smem_addr(&s_empty[s]), ph ^ 1u, abort_flag, args.status)) { ok = false; break; }
         if (lane == 0) {
           const uint32_t sa = smem_base + s * kSwStageBytes;
-          const uint32_t sb = sa + kSwATileBytes;
+          const uint32_t sb = sa + kSwKB * kSwATileBytes;
           const uint32_t full_leader = mapa_shared(smem_addr(&s_full[s]), 0);
-          if (leader) mbar_arrive_expect_tx(smem_addr(&s_full[s]), tx_bytes);
-          tma_load_2d_pair(sa, &tmap_w, full_leader, kb * kBK, w_base);
-          tma_load_2d_pair(sa + 64 * kBK * 2, &tmap_w, full_leader, kb * kBK, w_base + args.w_hi_offset);
-          tma_load_2d_pair(sb, &tmap_x, full_leader, kb * kBK, x_row);
+          if (leader) mbar_arrive_expect_tx(smem_addr(&s_full[s]), static_cast<uint32_t>(nk) * kb_bytes);
+          for (int i = 0; i < nk; ++i) {
+            const int kc = (kb0 + i) * kBK;
+            const uint32_t ai = sa + i * kSwATileBytes;
+            tma_load_2d_pair(ai, &tmap_w, full_leader, kc, w_base);
+            tma_load_2d_pair(ai + 64 * kBK * 2, &tmap_w, full_leader, kc, w_base + args.w_hi_offset);
+            tma_load_2d_pair(sb + i * kSwBTileBytes, &tmap_x, full_leader, kc, x_row);
+          }
         }
         __syncwarp();
         if (++s == S) { s = 0; ph ^= 1u; }
@@ -239,7 +250,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // descriptors of stage 0; stage s and k-slice kk add s * stage/16 and 2 * kk
       // to the 14-bit start-address field, which never carries (smem < 256 KB)
       const uint64_t da0 = sw128_kmajor_desc(smem_base);
-      const uint64_t db0 = sw128_kmajor_desc(smem_base + kSwATileBytes);
+      const uint64_t db0 = sw128_kmajor_desc(smem_base + kSwKB * kSwATileBytes);
       for (int tile = unit; ok && tile < total; tile += units, ++it) {
         const SwapTile t = swap_decode(tile, G, s_tstart, s_off, args.w_tiles);
         const uint32_t idesc = umma_idesc_bf16(256, t.n);
@@ -248,14 +259,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!mbar_wait_all(smem_addr(&s_tempty[buf]), tph ^ 1u, abort_flag, args.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * 256u;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb0 = 0; kb0 < num_kb; kb0 += kSwKB) {
+          const int nk = min(kSwKB, num_kb - kb0);
           if (!mbar_wait_all(smem_addr(&s_full[s]), ph, abort_flag, args.status)) { ok = false; break; }
           if (lane == 0) {
             const uint64_t off = static_cast<uint64_t>(s * (kSwStageBytes >> 4));
-            umma_bf16_pair(d_tmem, da0 + off, db0 + off, idesc, kb != 0 ? 1u : 0u);
-            umma_bf16_pair(d_tmem, da0 + off + 2, db0 + off + 2, idesc, 1u);
-            umma_bf16_pair(d_tmem, da0 + off + 4, db0 + off + 4, idesc, 1u);
-            umma_bf16_pair(d_tmem, da0 + off + 6, db0 + off + 6, idesc, 1u);
+#pragma unroll
+            for (int i = 0; i < kSwKB; ++i) {
+              if (i < nk) {
+                const uint64_t a = da0 + off + i * (kSwATileBytes >> 4);
+                const uint64_t b = db0 + off + i * (kSwBTileBytes >> 4);
+                umma_bf16_pair(d_tmem, a, b, idesc, (kb0 | i) != 0 ? 1u : 0u);
+                umma_bf16_pair(d_tmem, a + 2, b + 2, idesc, 1u);
+                umma_bf16_pair(d_tmem, a + 4, b + 4, idesc, 1u);
+                umma_bf16_pair(d_tmem, a + 6, b + 6, idesc, 1u);
+              }
+            }
             umma_commit_pair(smem_addr(&s_empty[s]), 0x3);
           }
           __syncwarp();

@@ -243,7 +243,54 @@ moe_status_t run_experts(const moe_layer_desc_t* d, const moe_weights_t* w, cons
   const int n1 = swiglu ? 2 * d->I : d->I;
   const void* b1 = (!swiglu && d->has_bias) ? w->b1 : nullptr;
   const void* b2 = (!swiglu && d->has_bias) ? w->b2 : nullptr;
-  if (d->dtype == MOE_DTYPE_BF16) {
+  // A handful of rows per expert (decode): tokens on M with single-CTA MMAs. The 128-row token
+  // tile is mostly padding, but a single-CTA MMA issues far faster than a pair's, and the
+  // weights still stream once (measured: GLM-4.5 decode expert GEMMs 0.837 -> 0.810 ms).
+  const bool few_rows = static_cast<long long>(d->T) * d->k < 4ll * d->M;
+  if (d->dtype == MOE_DTYPE_BF16 && few_rows) {
+    MOE_CUDA(launch_gather_rows(x, row_token, offsets + d->M, x_perm, pairs, d->T, d->D, 2, status, s));
+    MOE_TRY(mk.at(3));
+    GemmLaunch g1{};
+    g1.ncta = 1;
+    g1.A = x_perm; g1.a_rows = pairs;
+    g1.B = w->w1; g1.b_rows = static_cast<long long>(d->M) * n1;
+    g1.K = d->D;
+    g1.num_groups = d->M; g1.offsets = offsets; g1.rows_upper = pairs;
+    if (swiglu) {
+      const int half = std::min(128, round_up(d->I, 16));
+      g1.epi = EPI_SWIGLU;
+      g1.bn = 2 * half;
+      g1.n_tiles = (d->I + half - 1) / half;
+      g1.b_rows_per_group = n1; g1.b_row_step = half; g1.b_hi_offset = d->I;
+      g1.out_col_step = half;
+    } else {
+      g1.epi = EPI_GELU_BIAS;
+      g1.bn = std::min(256, round_up(d->I, 16));
+      g1.n_tiles = (d->I + g1.bn - 1) / g1.bn;
+      g1.b_rows_per_group = n1; g1.b_row_step = g1.bn; g1.b_hi_offset = g1.bn / 2;
+      g1.out_col_step = g1.bn;
+      g1.bias = b1;
+    }
+    g1.out_cols = d->I; g1.ldo = d->I; g1.out = h;
+    g1.status = status;
+    MOE_CUDA(launch_gemm_sm100(g1, s));
+    MOE_TRY(mk.at(4));
+    GemmLaunch g2{};
+    g2.ncta = 1;
+    g2.epi = EPI_SCALE_BIAS;
+    g2.A = h; g2.a_rows = pairs;
+    g2.B = w->w2; g2.b_rows = static_cast<long long>(d->M) * d->D;
+    g2.K = d->I;
+    g2.num_groups = d->M; g2.offsets = offsets; g2.rows_upper = pairs;
+    g2.bn = std::min(256, round_up(d->D, 16));
+    g2.n_tiles = (d->D + g2.bn - 1) / g2.bn;
+    g2.b_rows_per_group = d->D; g2.b_row_step = g2.bn; g2.b_hi_offset = g2.bn / 2;
+    g2.out_cols = d->D; g2.out_col_step = g2.bn; g2.ldo = d->D;
+    g2.out = out_perm; g2.row_scale = row_w; g2.bias = b2;
+    g2.status = status;
+    MOE_CUDA(launch_gemm_sm100(g2, s));
+    MOE_TRY(mk.at(5));
+  } else if (d->dtype == MOE_DTYPE_BF16) {
     if (slot_of != nullptr)
       MOE_CUDA(launch_scatter_rows(x, slot_of, x_perm, d->T, d->k, d->D, status, s));
     else

@@ -129,9 +129,6 @@ cudaError_t launch_gemm_sm100(const GemmLaunch& L, cudaStream_t s) {
   a.out = L.out;
   a.row_scale = L.row_scale;
   a.bias = static_cast<const __nv_bfloat16*>(L.bias);
-  a.comb_src = static_cast<const float*>(L.comb_src);
-  a.slot_of = L.slot_of;
-  a.k = L.k;
   a.idesc = umma_idesc_bf16(tile_rows, L.bn);
   a.status = L.status;
   // upper bound of the tile count: sum_g ceil(rows_g / tile_rows) <= rows/tile_rows + (#non-empty groups)
@@ -146,7 +143,6 @@ cudaError_t launch_gemm_sm100(const GemmLaunch& L, cudaStream_t s) {
     MOE_GEMM_CASE(EPI_GELU_BIAS)
     MOE_GEMM_CASE(EPI_SWIGLU)
     MOE_GEMM_CASE(EPI_SCALE_BIAS)
-    MOE_GEMM_CASE(EPI_COMBINE)
   }
 #undef MOE_GEMM_CASE
   return cudaErrorInvalidValue;

@@ -25,7 +25,7 @@
 //   warp 0      TMA producer: A tile 128 x 64 and this CTA's B rows x 64
 //   warp 1      TMEM allocator; MMA issuer (one thread of the first CTA)
 //   warps 2..9  epilogue: tcgen05.ld of the fp32 accumulator, fused
-//               activation / scaling / combine, stores to global; warp w
+//               activation / scaling, stores to global; warp w
 //               reads TMEM lane quarter w % 4, column chunks (w - 2) / 4
 //               (mod 2)
 // Two TMEM accumulators (2 x 256 columns) let the epilogue of one tile
@@ -41,8 +41,7 @@ enum GemmEpilogue : int {
   EPI_GELU_BIAS = 1,   // out bf16 = GELU_tanh(acc + b1[g, n])  (GELU expert, first GEMM)
   EPI_SWIGLU = 2,      // out bf16 = SiLU(acc_gate) * acc_up     (SwiGLU, fused gate/up)
   EPI_SCALE_BIAS = 3,  // out fp32 = (acc + b2[g, n]) * row_scale[r]   (second GEMM)
-  EPI_COMBINE = 4,     // out bf16 = acc + sum_j src[slot_of[r, j], n] (shared down + combine,
-                       //            src fp32)
+  // 4: unused (kept free so that the values of the others stay stable)
   EPI_STORE_BF16 = 5,  // out bf16 = acc                         (standalone shared down projection)
   EPI_BIAS_ADD = 6,    // out (layer dtype) = acc + b[n] + addend[r, n]   (dense FFN down projection;
                        //            bias and addend optional)
@@ -86,9 +85,6 @@ struct GemmArgs {
   void* out;
   const float* row_scale;        // EPI_SCALE_BIAS: [rows]
   const __nv_bfloat16* bias;     // EPI_GELU_BIAS / EPI_SCALE_BIAS: [G, out_cols] or nullptr
-  const float* comb_src;         // EPI_COMBINE: fp32 [*, ldo]
-  const int* slot_of;            // EPI_COMBINE: [rows, k]
-  int k;
   uint32_t idesc;
   int* status;
 };
@@ -200,33 +196,6 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tacc, 
           if (a.bias != nullptr) add_bias32(v, a.bias + static_cast<size_t>(g) * a.out_cols + col, nv);
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = gelu_tanh_fast(v[i]);
-        }
-        if constexpr (EPI == EPI_COMBINE) {
-          float acc[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
-          for (int j = 0; j < a.k; ++j) {
-            const int slot = a.slot_of[static_cast<size_t>(row) * a.k + j];
-            if (slot < 0) continue;  // sentinel pair
-            const float* src = a.comb_src + static_cast<size_t>(slot) * a.ldo + col;
-            if (nv == 32) {
-              const float4* s4 = reinterpret_cast<const float4*>(src);
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                const float4 f = s4[q];
-                acc[4 * q] += f.x;
-                acc[4 * q + 1] += f.y;
-                acc[4 * q + 2] += f.z;
-                acc[4 * q + 3] += f.w;
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (i < nv) acc[i] += src[i];
-            }
-          }
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = acc[i] + v[i];
         }
         store_row32_bf16(out, v, nv);
       }

@@ -58,9 +58,6 @@ struct GemmLaunch {
   void* out;
   const float* row_scale;
   const void* bias;
-  const void* comb_src;
-  const int32_t* slot_of;
-  int k;
   int* status;
 };
 cudaError_t launch_gemm_sm100(const GemmLaunch& L, cudaStream_t s);
@@ -100,9 +97,6 @@ struct SimtLaunch {
   float* out;
   const float* row_scale;
   const float* bias;
-  const float* comb_src;
-  const int32_t* slot_of;
-  int k;
   const float* addend;  // EPI_BIAS_ADD: [rows, ldo] or nullptr
 };
 cudaError_t launch_simt_gemm(const SimtLaunch& L, cudaStream_t s);

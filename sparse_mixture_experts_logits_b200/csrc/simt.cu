@@ -109,13 +109,6 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const SimtArgs args) {
       } else if constexpr (EPI == EPI_BIAS_ADD) {
         if (L.bias) v += L.bias[static_cast<size_t>(g) * L.out_cols + n];
         if (L.addend) v += L.addend[static_cast<size_t>(row) * L.ldo + n];
-      } else if constexpr (EPI == EPI_COMBINE) {
-        float s = 0.f;
-        for (int jj = 0; jj < L.k; ++jj) {
-          const int slot = L.slot_of[static_cast<size_t>(row) * L.k + jj];
-          if (slot >= 0) s += L.comb_src[static_cast<size_t>(slot) * L.ldo + n];
-        }
-        v = s + v;
       }
       L.out[static_cast<size_t>(row) * L.ldo + n] = v;
     }
@@ -134,7 +127,6 @@ cudaError_t launch_simt_gemm(const SimtLaunch& L, cudaStream_t s) {
     case EPI_GELU_BIAS: simt_gemm_kernel<EPI_GELU_BIAS><<<grid, 256, 0, s>>>(a); break;
     case EPI_SWIGLU: simt_gemm_kernel<EPI_SWIGLU><<<grid, 256, 0, s>>>(a); break;
     case EPI_SCALE_BIAS: simt_gemm_kernel<EPI_SCALE_BIAS><<<grid, 256, 0, s>>>(a); break;
-    case EPI_COMBINE: simt_gemm_kernel<EPI_COMBINE><<<grid, 256, 0, s>>>(a); break;
     case EPI_BIAS_ADD: simt_gemm_kernel<EPI_BIAS_ADD><<<grid, 256, 0, s>>>(a); break;
     default: simt_gemm_kernel<EPI_STORE_F32><<<grid, 256, 0, s>>>(a); break;
   }

@@ -7,10 +7,14 @@
 // and every output column n.  W is a bf16 stack of per-group [rows, K]
 // weight blocks (nn.Linear layout, K-major) and is the MMA's A operand;
 // the token rows X[r] (dispatch order: x gathered per expert, or h) are the
-// B operand.  Each CTA loads one 128-row TMA box of token rows per stage and
-// the MMA reads the first N/2 of them.  (Loading the rows by index with
+// B operand.  Each CTA loads one 128-row TMA box of token rows per k-block
+// and the MMA reads the first N/2 of them.  (Loading the rows by index with
 // tile::gather4 instead, 4 rows per TMA instruction, measured 2-3x slower:
 // the TMA instruction rate, not the bytes, became the limit.)
+//
+// Decode-shaped layers (a handful of rows per expert) do not come here: a
+// single-CTA MMA issues much faster than a pair's, so those run on the
+// tokens-on-M kernel of gemm_sm100.cuh with NCTA = 1.
 //
 // Why tokens on N: an expert's segment is cut into token tiles of at most
 // 256 rows whose width N is rounded up only to a multiple of 16, so the
@@ -25,8 +29,9 @@
 // of the up lanes hand their values to the gate lanes through shared memory.
 //
 // Warp roles (320 threads per CTA): warp 0 TMA producer, warp 1 TMEM
-// allocator and (first CTA) MMA issuer, warps 2..9 epilogue.  Every wait is bounded (kWaitTimeoutNs) and reports
-// MOE_DEVERR_TIMEOUT through the status word instead of hanging.
+// allocator and (first CTA) MMA issuer, warps 2..9 epilogue.  Every wait is
+// bounded (kWaitTimeoutNs) and reports MOE_DEVERR_TIMEOUT through the status
+// word instead of hanging.
 #pragma once
 
 #include "gemm_sm100.cuh"

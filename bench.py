@@ -54,6 +54,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU-baseline run time")
+    ap.add_argument("--ref-seconds", type=float, default=150.0,
+                    help="target run time of the whole --impl reference run")
     ap.add_argument("--T", type=int, default=None, help="override tokens per GPU (profiling runs)")
     ap.add_argument("--M", type=int, default=None, help="override routed experts (profiling runs)")
     return ap.parse_args()
@@ -728,7 +730,7 @@ def run_reference(args):
     probe_n = 8
     t0 = time.perf_counter()
     runner.run(runner.x_block(0, probe_n))
-    per_step_budget = max(0.5, 150.0 / max(1, args.steps + args.warmup))
+    per_step_budget = max(0.05, args.ref_seconds / max(1, args.steps + args.warmup))
     dt = time.perf_counter() - t0
     n = int(max(4, min(cfg["T"], probe_n * per_step_budget / max(dt, 1e-3))))
     cursor = 0

@@ -93,6 +93,12 @@ def check_routing(cfg, r, gpu_idx, gpu_w):
         assert ok, f"top-k differs beyond the near-tie band at token {bad}"
     w_ref = oracle.topk_weights(gpu_idx, r["logits"], r["g"], cfg["gate"], cfg["norm_topk_prob"],
                                 cfg["alpha"], cfg["eps"])
+    if cfg["norm_topk_prob"] and gpu_w.size:
+        # the renormalised weights of a token sum to alpha * S / (S + eps) (sigmoid; the GLM-4.5
+        # note's g-bar) or to alpha (softmax over the selected experts), in fp32 to ~1e-6
+        target = w_ref.sum(axis=1)
+        err_sum = np.abs(np.asarray(gpu_w, np.float64).sum(axis=1) - target).max()
+        assert err_sum <= 1e-6 * max(1.0, cfg["alpha"]) * cfg["k"], f"weight sum off by {err_sum}"
     err = np.abs(gpu_w - w_ref).max() if gpu_w.size else 0.0
     assert err <= W_ABS * max(1.0, cfg["alpha"]), f"gate weights off by {err}"
     return w_ref, ndiff

@@ -294,3 +294,35 @@ def test_bad_row_token_is_reported_not_faulted(B):
     keep[bad] = False
     assert torch.equal(out_perm[keep].view(torch.int32), ref[keep].view(torch.int32))
     assert torch.isfinite(out_perm[bad]).all()
+
+
+def test_zero_routed_scale_leaves_the_shared_expert(B):
+    """With routed_scaling_factor 0 every routed term is an exact zero, so y is
+    the shared expert's output alone ("Shared Expert" GLM-4.5 note: E_sh reads
+    the pre-routing x), bit for bit the standalone moe_shared_expert."""
+    cfg = ms.get_config("glm_small_bf16", alpha=0.0)
+    inp = gpu_inputs(cfg)
+    layer, y, _ = run_forward(B, cfg, inp)
+    d = layer.desc
+    y_sh = torch.empty_like(inp["x"])
+    wsh = torch.zeros(B.moe_shared_expert_workspace_size(d) + 256, dtype=torch.uint8, device="cuda")
+    B.moe_shared_expert(d, layer.weights, inp["x"].data_ptr(), y_sh.data_ptr(), wsh.data_ptr(), wsh.numel(),
+                        torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), y_sh.view(torch.int16))
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_random_shapes(B, seed):
+    """Seeded random layers inside the library's limits: widths, expert
+    counts, k, router and expert kinds, token counts with ragged tails."""
+    rng = np.random.default_rng(100 + seed)
+    swiglu = bool(rng.integers(0, 2))
+    M = int(rng.choice([2, 5, 8, 12, 16, 24, 40, 64]))
+    k = int(rng.integers(1, min(M, 8) + 1))
+    over = dict(T=int(rng.integers(1, 700)), D=int(16 * rng.integers(2, 24)),
+                I=int(16 * rng.integers(1, 24)), M=M, k=k, seed=seed)
+    name = "glm_small_bf16" if swiglu else "glam_small_bf16"
+    if swiglu:
+        over["I_sh"] = int(16 * rng.integers(0, 12))
+    check_layer(B, ms.get_config(name, **over), all_tokens=True)

@@ -32,7 +32,7 @@ listed in the design notes):
     layer output alone; ``expert_load`` reports the load statistic itself:
     the tokens each expert receives and their coefficient of variation.
 
-Pins: tests/oracle_pins.py checks every gradient here against central finite
+Pins: tests/oracle_pins_backward.py checks every gradient here against central finite
 differences of the pinned forward oracle (an independent derivative), on
 tiny layers of every router and expert variant, plus the shift invariance of
 the renormalised softmax weights.
@@ -115,7 +115,12 @@ def router_backward(idx, dw, logits, g, gate, norm_topk_prob, alpha, eps):
       for every i.
     sigmoid_bias: w_j = alpha g_j / (G + eps) with G = sum_S g (or alpha
       g_j), so dg_i = alpha (dw_i / (G + eps) - sum_j dw_j g_j / (G + eps)^2)
-      for i in S_t (alpha dw_i), and dl_i = dg_i g_i (1 - g_i).
+      for i in S_t (alpha dw_i), and dl_i = dg_i g_i (1 - g_i).  The
+      normalised form is evaluated centred, as
+      alpha / (G + eps) * (dw_i - sum_j gbar_j dw_j) with gbar = g / (G + eps),
+      the same value; with one chosen expert gbar is 1 to within eps, and
+      the gradient (which is eps-small) comes out as 0 instead of the
+      rounding residue of two equal terms.
     Chosen-expert indices equal to M (the sentinel) carry no weight."""
     idx = np.asarray(idx, dtype=np.int64)
     dw = _f64(dw)
@@ -144,7 +149,8 @@ def router_backward(idx, dw, logits, g, gate, norm_topk_prob, alpha, eps):
             gt = _f64(g)[t, es]
             if norm_topk_prob:
                 den = gt.sum() + eps
-                dg = alpha * (dw[t, js] / den - np.dot(dw[t, js], gt) / den ** 2)
+                gbar = gt / den
+                dg = alpha / den * (dw[t, js] - np.dot(gbar, dw[t, js]))
             else:
                 dg = alpha * dw[t, js]
             dl[t, es] = dg * gt * (1.0 - gt)

@@ -162,8 +162,22 @@ def pin_dense_backward(B):
     assert np.allclose(g["db2"][0], d["db2"], rtol=1e-12, atol=1e-13)
 
 
+def pin_single_choice_sigmoid_router(B):
+    """With one chosen expert the renormalised sigmoid weight is
+    alpha g / (g + eps), constant to within eps ("Shared Expert" GLM-4.5
+    note, eq. g-bar with k = 1), so the router gets no gradient: dlogits and
+    dW_r are zero, and dx is that of the experts alone."""
+    cfg = dict(T=7, D=5, M=4, k=1, gate="sigmoid_bias", act="swiglu", I=3,
+               norm_topk_prob=1, alpha=2.5, eps=1e-20, I_sh=2)
+    inp = tiny_inputs(cfg, 130)
+    dy = np.random.default_rng(131).standard_normal((cfg["T"], cfg["D"]))
+    g = B.moe_backward(cfg, inp, dy)
+    assert np.abs(g["dl"]).max() <= 1e-12 and np.abs(g["dw_r"]).max() <= 1e-12
+    assert np.abs(g["dw"]).max() > 1e-3
+
+
 BWD_PINS = [
     pin_fd_glam, pin_fd_glm_shared, pin_fd_softmax_unnormalised, pin_fd_sigmoid_unnormalised,
     pin_fd_grouped, pin_softmax_shift_invariance, pin_activation_derivatives, pin_expert_load,
-    pin_dense_backward,
+    pin_dense_backward, pin_single_choice_sigmoid_router,
 ]

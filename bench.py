@@ -58,6 +58,8 @@ def parse_args():
                     help="target run time of the whole --impl reference run")
     ap.add_argument("--T", type=int, default=None, help="override tokens per GPU (profiling runs)")
     ap.add_argument("--M", type=int, default=None, help="override routed experts (profiling runs)")
+    ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward"],
+                    help="backward: time moe_backward (all gradients of the layer) instead of the forward")
     return ap.parse_args()
 
 
@@ -765,10 +767,134 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def backward_cpu_baseline(cfg, inp, dy, idx, target_s, max_experts=16):
+    """The fp64 backward oracle on the first tokens of the workload, each
+    with only the experts it chose (its gradients do not depend on the
+    others); the sample grows while its experts fit in host memory."""
+    import oracle
+
+    f64 = lambda t: t.detach().to(torch.float64).cpu().numpy()  # noqa: E731
+    n = 1
+    while True:
+        used = np.unique(idx[:n])
+        pos = {int(e): i for i, e in enumerate(used)}
+        sel = torch.as_tensor(used, device=inp["w1"].device)
+        sub = {"x": f64(inp["x"][:n]), "w_r": f64(inp["w_r"][:, sel])}
+        for k in ("e_bias", "w1", "w2", "b1", "b2"):
+            sub[k] = None if inp.get(k) is None else f64(inp[k][sel])
+        for k in ("sh_w1", "sh_w2"):
+            sub[k] = None if inp.get(k) is None else f64(inp[k])
+        sub_idx = np.vectorize(lambda e: pos[int(e)])(idx[:n])
+        sub_cfg = dict(cfg, T=n, M=len(used), n_group=1, topk_group=1)
+        dyh = f64(dy[:n])
+        t0 = time.perf_counter()
+        oracle.moe_backward.moe_backward(sub_cfg, sub, dyh, idx=sub_idx)
+        dt = time.perf_counter() - t0
+        n2 = min(cfg["T"], 2 * n)
+        if dt >= target_s * 0.3 or n2 == n or len(np.unique(idx[:n2])) > max_experts:
+            break
+        n = n2
+    cores, api = _blas_threads()
+    return {"value": n / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {n} tokens of the workload with the {len(used)} experts they chose, fp64 NumPy "
+                      f"backward oracle ({api} BLAS); weights widened outside the timed run",
+            "seconds": dt}
+
+
+def run_backward(args):
+    """One step = moe_backward over the workload's tokens: the routing and
+    the experts' forward values recomputed, then every gradient of the layer."""
+    import sparse_mixture_experts_logits_b200 as B
+
+    rank, local_rank, world = dist_env()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = dist_init(world, local_rank)
+    cfg = workload_config(args)
+    T, D = cfg["T"], cfg["D"]
+    inp = ms.layer_inputs(dict(cfg, T=1), dev)
+    r0, r1 = token_rows(rank, T)
+    rows = torch.arange(r0, r1, device=dev)
+    inp["x"] = ms.normal_rows(rows, D, 1.0, ms._key(cfg, "x"), ms.act_dtype(cfg))
+    dy = ms.normal_rows(rows, D, 1.0, ms._key(cfg, "dy"), ms.act_dtype(cfg))
+    layer = B.MoELayer(cfg, inp)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    grads = layer.backward(inp["x"], dy)
+    for _ in range(max(3, args.warmup) - 1):
+        layer.backward(inp["x"], dy, grads=grads)
+    torch.cuda.synchronize()
+    if layer.backward_status() != 0:
+        raise RuntimeError("device status flag set during warm-up")
+    counts = layer.backward_view("counts").cpu().numpy()
+    idx = layer.backward_view("topk_idx").cpu().numpy()
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    for i in range(K):
+        flush.zero_()
+        starts[i].record(stream)
+        layer.backward(inp["x"], dy, grads=grads)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    if dist is not None:
+        dist.barrier()
+    ms_step = max_over_ranks(dist, sum(starts[i].elapsed_time(ends[i]) for i in range(K)) / K, dev)
+    if layer.backward_status() != 0:
+        raise RuntimeError("device status flag set during the timed steps")
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+    peaks, peak_src = load_peaks()
+    fwd_flops, _ = B.moe_algorithmic_work(layer.desc, counts)
+    # every GEMM of the layer has two in the backward (input and weight gradient)
+    flops = 2.0 * fwd_flops
+    peak_tf = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    achieved = flops / (ms_step / 1e3) / 1e12
+    # the CUDA-core fp32 FMA rate: 148 SMs x 128 lanes x 2 FLOP at the 1965 MHz clock ceiling
+    simt_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+    out = {
+        "metric": "MoE layer backward throughput (all gradients; routing and expert forward recomputed)",
+        "value": world * T / (ms_step / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": cfg["dtype"] + " in, fp32 sums and gradients",
+        "data": "synthetic (seeded counter-based generator; random-init weights)",
+        "config": {"workload": args.config, "T_per_gpu": T, "D": D, "M": cfg["M"], "k": cfg["k"],
+                   "I": cfg["I"], "I_sh": cfg.get("I_sh", 0),
+                   "l2": "flushed between steps (256 MiB write outside the timed events)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": achieved / peak_tf, "traffic": None,
+                     "kernel": "the whole step (bwd_gemm_kernel launches hold most of it; see the launch list)",
+                     "peak_source": f"{peak_src}: bf16_tflops_sustained",
+                     "algorithmic": {"flops": flops, "note": "2 x forward FLOPs; the recompute is not counted"},
+                     "frac_of_fp32_simt_peak": achieved / simt_peak},
+        "e2e": None,
+        "gpu_launches": B.moe_backward_launch_count(layer.desc) * K,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = backward_cpu_baseline(cfg, inp, dy, idx, args.cpu_seconds)
+    print(json.dumps(out), flush=True)
+    del layer
+    if dist is not None:
+        dist.destroy_process_group()
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.which == "backward":
+        run_backward(args)
     elif is_dense(workload_config(args)):
         run_dense(args)
     else:

@@ -332,6 +332,55 @@ moe_status_t moe_dense_ffn_profiled(const moe_dense_desc_t* d, const void* w1, c
                                     const void* addend, void* y, void* ws, size_t ws_bytes,
                                     void* stream, void* const* events, int n_events);
 
+/* ---- backward of the layer (training) ---------------------------------
+ * The chain rule through each forward step above.  The pages describe
+ * training only in prose (the GLaM notes: the router is trained with a
+ * penalty on uneven expert load); this is the gradient of the layer output
+ * itself.  The top-k choice is piecewise constant, so the gradient reaches
+ * the router only through the weights w of the chosen experts, and e_bias
+ * (which enters the choice only) has none. */
+
+/* Gradients written by moe_backward (device pointers, caller-owned; every
+ * one is overwritten, not accumulated). */
+typedef struct {
+  void* dx;      /* [T, D] dtype: dL/dx (routed experts + shared expert + router) */
+  float* dw_r;   /* [D, M] fp32 */
+  float* dw1;    /* [M, H or 2I, D] fp32 (layout of w1) */
+  float* db1;    /* [M, H] fp32; required iff act = GELU_TANH and has_bias, else ignored */
+  float* dw2;    /* [M, D, H or I] fp32 (layout of w2) */
+  float* db2;    /* [M, D] fp32; as db1 */
+  float* dsh_w1; /* [2 I_sh, D] fp32; required iff I_sh > 0, else ignored */
+  float* dsh_w2; /* [D, I_sh] fp32; as dsh_w1 */
+} moe_grads_t;
+
+/* Workspace of moe_backward.  It begins with the forward's layout
+ * (moe_workspace_layout: after the call the routing fields hold this
+ * backward's routing); the rest holds fp32 intermediates of every
+ * dispatched row (pre-activations, activations, expert outputs and their
+ * gradients).  0 if the descriptor is invalid. */
+size_t moe_backward_workspace_size(const moe_layer_desc_t* d);
+
+/* Given x [T, D] and dy = dL/dy [T, D] (both dtype) of y = MoE-FFN(x), write
+ * every gradient of L: the routing is recomputed (the same route and
+ * dispatch order as moe_forward), the experts' forward values are recomputed
+ * in fp32 from the dtype inputs, and every GEMM of the backward sums in fp32
+ * in a fixed order (bitwise repeatable).  Per chosen pair (t, j) with expert
+ * e and weight w:
+ *   dw[t,j]   = <dy_t, E_e(x_t)>,     dE = w dy_t  through the expert;
+ *   dlogits   from dw through the weight formula of the gate;
+ *   dx_t      = sum_j dx of the pair + shared expert's dx + dlogits_t W_r^T;
+ *   dW_r      = x^T dlogits.
+ * The expert and shared weights get the sums over their rows of the usual
+ * FFN weight gradients.  x, dy and the gradients must not overlap.  Errors
+ * as moe_forward; required gradient pointers that are NULL give
+ * MOE_ERR_INVALID_ARG.  T = 0 zero-fills the parameter gradients. */
+moe_status_t moe_backward(const moe_layer_desc_t* d, const moe_weights_t* w, const void* x,
+                          const void* dy, const moe_grads_t* grads, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/* Number of kernels one moe_backward call with this descriptor launches. */
+int moe_backward_launch_count(const moe_layer_desc_t* d);
+
 #ifdef __cplusplus
 }
 #endif

@@ -222,6 +222,11 @@ def addend_tokens(cfg, device="cpu") -> torch.Tensor:
     return normal((cfg["T"], cfg["D"]), 1.0, _key(cfg, "addend"), device, act_dtype(cfg))
 
 
+def upstream_grad(cfg, device="cpu") -> torch.Tensor:
+    """dL/dy of a backward pass, [T, D], N(0, 1) in the layer's dtype."""
+    return normal((cfg["T"], cfg["D"]), 1.0, _key(cfg, "dy"), device, act_dtype(cfg))
+
+
 def dense_inputs(cfg, device="cpu") -> dict:
     """Every input of one dense FFN layer call (the layer's weights are drawn
     like one expert's, under the name "dense")."""

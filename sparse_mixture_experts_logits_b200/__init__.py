@@ -1,4 +1,4 @@
-"""Sparse MoE FFN layer forward on NVIDIA B200 (sm_100a).
+"""Sparse MoE FFN layer forward and backward on NVIDIA B200 (sm_100a).
 
 The compute path is the C-ABI library ``libmoe_b200.so`` (declared in
 ``include/moe_b200.h``); this package is its Python binding: ctypes
@@ -18,6 +18,7 @@ from .abi import (  # noqa: F401
     moe_forward_profiled, moe_forward_launch_count, NUM_STAGE_EVENTS, STAGE_NAMES,
     moe_algorithmic_work, EXPORTED_SYMBOLS, moe_forward_add,
     DenseDesc, moe_dense_ffn_workspace_size, moe_dense_ffn, moe_dense_ffn_profiled, NUM_DENSE_EVENTS,
+    Grads, moe_backward_workspace_size, moe_backward, moe_backward_launch_count,
     DTYPE_F32, DTYPE_BF16, GATE_SOFTMAX, GATE_SIGMOID_BIAS, ACT_GELU_TANH, ACT_SWIGLU,
     DEVERR_NONE, DEVERR_BAD_EXPERT_INDEX, DEVERR_TIMEOUT, DEVERR_BAD_ROW_TOKEN,
 )

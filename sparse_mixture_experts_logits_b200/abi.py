@@ -27,6 +27,7 @@ EXPORTED_SYMBOLS = [
     "moe_combine", "moe_workspace_size", "moe_workspace_layout", "moe_forward",
     "moe_forward_profiled", "moe_forward_launch_count", "moe_algorithmic_work",
     "moe_forward_add", "moe_dense_ffn_workspace_size", "moe_dense_ffn", "moe_dense_ffn_profiled",
+    "moe_backward_workspace_size", "moe_backward", "moe_backward_launch_count",
 ]
 NUM_STAGE_EVENTS = 9
 NUM_DENSE_EVENTS = 3
@@ -57,6 +58,11 @@ class DenseDesc(ctypes.Structure):
 class Weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("w_r", "e_bias", "w1", "b1", "w2", "b2", "sh_w1", "sh_w2")]
+
+
+class Grads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("dx", "dw_r", "dw1", "db1", "dw2", "db2", "dsh_w1", "dsh_w2")]
 
 
 class WsLayout(ctypes.Structure):
@@ -111,6 +117,9 @@ _decl("moe_dense_ffn_workspace_size", _sz, [_P(DenseDesc)])
 _decl("moe_dense_ffn", _i, [_P(DenseDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
 _decl("moe_dense_ffn_profiled", _i, [_P(DenseDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp,
                                      _P(_vp), _i])
+_decl("moe_backward_workspace_size", _sz, [_P(LayerDesc)])
+_decl("moe_backward", _i, [_P(LayerDesc), _P(Weights), _vp, _vp, _P(Grads), _vp, _sz, _vp])
+_decl("moe_backward_launch_count", _i, [_P(LayerDesc)])
 
 
 def _status_name(s: int) -> str:
@@ -245,3 +254,16 @@ def moe_dense_ffn_profiled(desc, w1, b1, w2, b2, x, addend, y, ws, ws_bytes, str
     arr = (ctypes.c_void_p * len(events))(*events)
     _check("moe_dense_ffn_profiled", lib.moe_dense_ffn_profiled(
         ctypes.byref(desc), w1, b1, w2, b2, x, addend, y, ws, ws_bytes, stream, arr, len(events)))
+
+
+def moe_backward_workspace_size(desc: LayerDesc) -> int:
+    return lib.moe_backward_workspace_size(ctypes.byref(desc))
+
+
+def moe_backward(desc, weights, x, dy, grads, ws, ws_bytes, stream=None):
+    _check("moe_backward", lib.moe_backward(ctypes.byref(desc), ctypes.byref(weights), x, dy,
+                                            ctypes.byref(grads), ws, ws_bytes, stream))
+
+
+def moe_backward_launch_count(desc) -> int:
+    return lib.moe_backward_launch_count(ctypes.byref(desc))

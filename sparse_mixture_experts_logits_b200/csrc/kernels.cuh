@@ -101,4 +101,42 @@ struct SimtLaunch {
 };
 cudaError_t launch_simt_gemm(const SimtLaunch& L, cudaStream_t s);
 
+// backward.cu: C (+)= A B^T on the CUDA cores, fp32 sums, with strided
+// operands: A(m, k) = A[m * a_sm + k * a_sk], B(n, k) = B[g * b_gstride +
+// n * b_sn + k * b_sk], C(m, n) = C[g * c_gstride + m * ldc + n] (+ bias[g *
+// bias_gstride + n], bias of B's type).  Groups g come from offsets [G+1]:
+// mode 0 splits the rows m (absolute row indices, c_gstride unused), mode 1
+// splits the contraction k (absolute k indices; rows = M extent); without
+// offsets there is one group over [0, rows) or [0, K).  An empty group of
+// mode 1 writes zeros.
+struct BwdGemmLaunch {
+  const void* A; long long a_sm, a_sk; bool a_bf16;
+  const void* B; long long b_sn, b_sk, b_gstride; bool b_bf16;
+  const void* bias; long long bias_gstride;
+  float* C; long long ldc, c_gstride;
+  int mode;
+  const int32_t* offsets;
+  int G;
+  long long rows, K;
+  int N;
+  int accumulate;
+};
+cudaError_t launch_bwd_gemm(const BwdGemmLaunch& L, cudaStream_t s);
+// a = GELU(h) or SiLU(gate) * up for rows < min(rows, *n_rows) (n_rows may be null).
+cudaError_t launch_bwd_act(const float* h, float* a, const int32_t* n_rows, long long rows, int Ha, bool swiglu,
+                           cudaStream_t s);
+// h := dL/dh from da = dL/da, in place.
+cudaError_t launch_bwd_act_grad(const float* da, float* h, const int32_t* n_rows, long long rows, int Ha,
+                                bool swiglu, cudaStream_t s);
+// dw[t, j] = <dy_t, o[slot]>, dO[slot] = topk_w[t, j] dy_t.
+cudaError_t launch_bwd_pairs(int dtype, const void* dy, const float* o, const int32_t* slot_of,
+                             const float* topk_w, float* dw, float* dO, int T, int k, int D, long long rows_cap,
+                             cudaStream_t s);
+// out[g, :] = column sums of Y over the rows of group g.
+cudaError_t launch_bwd_colsum(const float* Y, long long ldy, const int32_t* offsets, int G, long long rows_cap,
+                              int N, float* out, cudaStream_t s);
+// dL/dlogits [T, M] from dL/dw [T, k].
+cudaError_t launch_bwd_router(const float* logits, const int32_t* idx, const float* dw, int T, int M, int k,
+                              int gate, int norm, float alpha, float eps, float* dl, cudaStream_t s);
+
 }  // namespace moe

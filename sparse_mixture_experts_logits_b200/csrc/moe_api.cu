@@ -828,3 +828,222 @@ void moe_algorithmic_work(const moe_layer_desc_t* d, const int32_t* counts_host,
 }
 
 }  // extern "C"
+
+// =========================================================== backward
+namespace {
+
+// The forward's layout first (route, dispatch order, out_perm = the experts'
+// recomputed outputs), then the backward's fp32 rows.
+struct BwdWs {
+  FwdWs f;
+  size_t xp, hpre, act, dO, da, dxp, dwp, dl, hs, as, das, dxs, total;
+};
+
+BwdWs backward_layout(const moe_layer_desc_t* d) {
+  BwdWs L;
+  L.f = forward_layout(d);
+  Carve c;
+  c.off = L.f.pub.total;
+  const size_t pairs = static_cast<size_t>(d->T) * d->k;
+  const size_t n1 = d->act == MOE_ACT_SWIGLU ? 2ull * d->I : static_cast<size_t>(d->I);
+  const size_t Ha = d->I, T = d->T, Is = d->I_sh;
+  L.xp = c.take(pairs * d->D * esize(d->dtype));
+  L.hpre = c.take(pairs * n1 * 4);  // pre-activations, then their gradient in place
+  L.act = c.take(pairs * Ha * 4);
+  L.dO = c.take(pairs * d->D * 4);
+  L.da = c.take(pairs * Ha * 4);
+  L.dxp = c.take(pairs * d->D * 4);
+  L.dwp = c.take(pairs * 4);
+  L.dl = c.take(T * d->M * 4);
+  L.hs = c.take(T * 2 * Is * 4);
+  L.as = c.take(T * Is * 4);
+  L.das = c.take(T * Is * 4);
+  L.dxs = c.take(T * d->D * 4);
+  L.total = c.off;
+  return L;
+}
+
+// C = A B^T with A(m, k) = A[m a_sm + k a_sk] and B(n, k) = B[g b_gstride + n b_sn + k b_sk].
+BwdGemmLaunch bwd_gemm(const void* A, long long a_sm, long long a_sk, bool a_bf16, const void* B, long long b_sn,
+                       long long b_sk, long long b_gstride, bool b_bf16, float* C, long long ldc, long long rows,
+                       long long K, int N) {
+  BwdGemmLaunch L{};
+  L.A = A; L.a_sm = a_sm; L.a_sk = a_sk; L.a_bf16 = a_bf16;
+  L.B = B; L.b_sn = b_sn; L.b_sk = b_sk; L.b_gstride = b_gstride; L.b_bf16 = b_bf16;
+  L.C = C; L.ldc = ldc;
+  L.rows = rows; L.K = K; L.N = N;
+  return L;
+}
+
+moe_status_t zero_param_grads(const moe_layer_desc_t* d, const moe_grads_t* g, cudaStream_t s) {
+  const bool swiglu = d->act == MOE_ACT_SWIGLU;
+  const size_t n1 = swiglu ? 2ull * d->I : static_cast<size_t>(d->I);
+  const size_t D = d->D, M = d->M, Ha = d->I, Is = d->I_sh;
+  MOE_CUDA(cudaMemsetAsync(g->dw_r, 0, D * M * 4, s));
+  MOE_CUDA(cudaMemsetAsync(g->dw1, 0, M * n1 * D * 4, s));
+  MOE_CUDA(cudaMemsetAsync(g->dw2, 0, M * D * Ha * 4, s));
+  if (!swiglu && d->has_bias) {
+    MOE_CUDA(cudaMemsetAsync(g->db1, 0, M * Ha * 4, s));
+    MOE_CUDA(cudaMemsetAsync(g->db2, 0, M * D * 4, s));
+  }
+  if (Is > 0) {
+    MOE_CUDA(cudaMemsetAsync(g->dsh_w1, 0, 2 * Is * D * 4, s));
+    MOE_CUDA(cudaMemsetAsync(g->dsh_w2, 0, D * Is * 4, s));
+  }
+  return MOE_OK;
+}
+
+moe_status_t backward_impl(const moe_layer_desc_t* d, const moe_weights_t* w, const void* x, const void* dy,
+                           const moe_grads_t* g, void* ws, size_t ws_bytes, cudaStream_t s) {
+  MOE_TRY(check_desc(d));
+  MOE_TRY(check_weights(d, w, true, true));
+  if (w->w_r == nullptr || g == nullptr) return MOE_ERR_INVALID_ARG;
+  const bool swiglu = d->act == MOE_ACT_SWIGLU;
+  const bool biases = !swiglu && d->has_bias;
+  if (!g->dw_r || !g->dw1 || !g->dw2) return MOE_ERR_INVALID_ARG;
+  if (biases && (!g->db1 || !g->db2)) return MOE_ERR_INVALID_ARG;
+  if (d->I_sh > 0 && (!g->dsh_w1 || !g->dsh_w2)) return MOE_ERR_INVALID_ARG;
+  if (d->T == 0) {
+    MOE_TRY(check_device());
+    return zero_param_grads(d, g, s);
+  }
+  if (!x || !dy || !g->dx || !ws || !aligned_ws(ws)) return MOE_ERR_INVALID_ARG;
+  const BwdWs L = backward_layout(d);
+  if (ws_bytes < L.total) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_device());
+  const bool bf = d->dtype == MOE_DTYPE_BF16;
+  const int T = d->T, D = d->D, M = d->M, k = d->k, Ha = d->I, Is = d->I_sh;
+  const int n1 = swiglu ? 2 * d->I : d->I;
+  const long long pairs = static_cast<long long>(T) * k;
+  int* status = at<int*>(ws, L.f.pub.status);
+  int32_t* idx = at<int32_t*>(ws, L.f.pub.topk_idx);
+  float* tw = at<float*>(ws, L.f.pub.topk_w);
+  int32_t* counts = at<int32_t*>(ws, L.f.pub.counts);
+  int32_t* offsets = at<int32_t*>(ws, L.f.pub.offsets);
+  int32_t* slot_of = at<int32_t*>(ws, L.f.pub.slot_of);
+  int32_t* row_token = at<int32_t*>(ws, L.f.pub.row_token);
+  float* row_w = at<float*>(ws, L.f.pub.row_w);
+  float* logits = at<float*>(ws, L.f.logits);
+  float* o = at<float*>(ws, L.f.pub.out_perm);
+  void* xp = at<void*>(ws, L.xp);
+  float* hpre = at<float*>(ws, L.hpre);
+  float* act = at<float*>(ws, L.act);
+  float* dO = at<float*>(ws, L.dO);
+  float* da = at<float*>(ws, L.da);
+  float* dxp = at<float*>(ws, L.dxp);
+  float* dwp = at<float*>(ws, L.dwp);
+  float* dl = at<float*>(ws, L.dl);
+  float* dxs = at<float*>(ws, L.dxs);
+  const int32_t* n_rows = offsets + M;  // pairs dispatched
+  Range whole("moe_backward");
+  MOE_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
+  {
+    Range r("moe.route");
+    MOE_TRY(run_route(x, w->w_r, w->e_bias, T, D, M, k, d->dtype, d->gate, d->norm_topk_prob,
+                      d->routed_scaling_factor, d->eps, d->n_group, d->topk_group, idx, tw, logits,
+                      at<void*>(ws, L.f.wrT), status, s));
+  }
+  {
+    Range r("moe.dispatch");
+    MOE_CUDA(launch_permute(idx, tw, T, k, M, counts, offsets, slot_of, row_token, row_w,
+                            at<int32_t*>(ws, L.f.chunk_counts), at<int32_t*>(ws, L.f.chunk_base), status, s));
+    MOE_CUDA(launch_gather_rows(x, row_token, n_rows, xp, static_cast<int>(pairs), T, D,
+                                static_cast<int>(esize(d->dtype)), status, s));
+  }
+  {
+    Range r("moe.experts_backward");
+    // forward values: h = x W1^T (+ b1), a = act(h), o = a W2^T (+ b2), per expert segment
+    BwdGemmLaunch g1 = bwd_gemm(xp, D, 1, bf, w->w1, D, 1, 1ll * n1 * D, bf, hpre, n1, pairs, D, n1);
+    g1.offsets = offsets; g1.G = M;
+    g1.bias = biases ? w->b1 : nullptr; g1.bias_gstride = Ha;
+    MOE_CUDA(launch_bwd_gemm(g1, s));
+    MOE_CUDA(launch_bwd_act(hpre, act, n_rows, pairs, Ha, swiglu, s));
+    BwdGemmLaunch g2 = bwd_gemm(act, Ha, 1, false, w->w2, Ha, 1, 1ll * D * Ha, bf, o, D, pairs, Ha, D);
+    g2.offsets = offsets; g2.G = M;
+    g2.bias = biases ? w->b2 : nullptr; g2.bias_gstride = D;
+    MOE_CUDA(launch_bwd_gemm(g2, s));
+    // dw of every pair and dO = w dy at its row
+    MOE_CUDA(launch_bwd_pairs(d->dtype, dy, o, slot_of, tw, dwp, dO, T, k, D, pairs, s));
+    // da = dO W2, dh = da * act'(h) (in place over h), dx rows = dh W1
+    BwdGemmLaunch g3 = bwd_gemm(dO, D, 1, false, w->w2, 1, Ha, 1ll * D * Ha, bf, da, Ha, pairs, D, Ha);
+    g3.offsets = offsets; g3.G = M;
+    MOE_CUDA(launch_bwd_gemm(g3, s));
+    MOE_CUDA(launch_bwd_act_grad(da, hpre, n_rows, pairs, Ha, swiglu, s));
+    BwdGemmLaunch g4 = bwd_gemm(hpre, n1, 1, false, w->w1, 1, D, 1ll * n1 * D, bf, dxp, D, pairs, n1, D);
+    g4.offsets = offsets; g4.G = M;
+    MOE_CUDA(launch_bwd_gemm(g4, s));
+    // weight gradients: sums over each expert's rows (the contraction split by expert)
+    BwdGemmLaunch g5 = bwd_gemm(dO, 1, D, false, act, 1, Ha, 0, false, g->dw2, Ha, D, pairs, Ha);
+    g5.mode = 1; g5.offsets = offsets; g5.G = M; g5.c_gstride = 1ll * D * Ha;
+    MOE_CUDA(launch_bwd_gemm(g5, s));
+    BwdGemmLaunch g6 = bwd_gemm(hpre, 1, n1, false, xp, 1, D, 0, bf, g->dw1, D, n1, pairs, D);
+    g6.mode = 1; g6.offsets = offsets; g6.G = M; g6.c_gstride = 1ll * n1 * D;
+    MOE_CUDA(launch_bwd_gemm(g6, s));
+    if (biases) {
+      MOE_CUDA(launch_bwd_colsum(dO, D, offsets, M, pairs, D, g->db2, s));
+      MOE_CUDA(launch_bwd_colsum(hpre, n1, offsets, M, pairs, Ha, g->db1, s));
+    }
+  }
+  if (Is > 0) {
+    Range r("moe.shared_expert_backward");
+    float* hs = at<float*>(ws, L.hs);
+    float* as = at<float*>(ws, L.as);
+    float* das = at<float*>(ws, L.das);
+    MOE_CUDA(launch_bwd_gemm(bwd_gemm(x, D, 1, bf, w->sh_w1, D, 1, 0, bf, hs, 2 * Is, T, D, 2 * Is), s));
+    MOE_CUDA(launch_bwd_act(hs, as, nullptr, T, Is, true, s));
+    MOE_CUDA(launch_bwd_gemm(bwd_gemm(dy, D, 1, bf, w->sh_w2, 1, Is, 0, bf, das, Is, T, D, Is), s));
+    MOE_CUDA(launch_bwd_act_grad(das, hs, nullptr, T, Is, true, s));
+    MOE_CUDA(launch_bwd_gemm(bwd_gemm(hs, 2 * Is, 1, false, w->sh_w1, 1, D, 0, bf, dxs, D, T, 2 * Is, D), s));
+    BwdGemmLaunch w2g = bwd_gemm(dy, 1, D, bf, as, 1, Is, 0, false, g->dsh_w2, Is, D, T, Is);
+    w2g.mode = 1;
+    MOE_CUDA(launch_bwd_gemm(w2g, s));
+    BwdGemmLaunch w1g = bwd_gemm(hs, 1, 2 * Is, false, x, 1, D, 0, bf, g->dsh_w1, D, 2 * Is, T, D);
+    w1g.mode = 1;
+    MOE_CUDA(launch_bwd_gemm(w1g, s));
+  }
+  {
+    Range r("moe.router_backward");
+    MOE_CUDA(launch_bwd_router(logits, idx, dwp, T, M, k, d->gate, d->norm_topk_prob, d->routed_scaling_factor,
+                               d->eps, dl, s));
+    BwdGemmLaunch wr = bwd_gemm(x, 1, D, bf, dl, 1, M, 0, false, g->dw_r, M, D, T, M);
+    wr.mode = 1;
+    MOE_CUDA(launch_bwd_gemm(wr, s));
+    BwdGemmLaunch xr = bwd_gemm(dl, M, 1, false, w->w_r, M, 1, 0, bf, dxs, D, T, M, D);
+    xr.accumulate = Is > 0 ? 1 : 0;  // onto the shared expert's dx
+    MOE_CUDA(launch_bwd_gemm(xr, s));
+  }
+  {
+    Range r("moe.combine_backward");
+    MOE_CUDA(launch_combine(d->dtype, dxp, slot_of, dxs, true, nullptr, g->dx, T, D, k, s));
+  }
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_backward_workspace_size(const moe_layer_desc_t* d) {
+  if (check_desc(d) != MOE_OK) return 0;
+  return backward_layout(d).total;
+}
+
+moe_status_t moe_backward(const moe_layer_desc_t* d, const moe_weights_t* w, const void* x, const void* dy,
+                          const moe_grads_t* grads, void* ws, size_t ws_bytes, void* stream) {
+  return backward_impl(d, w, x, dy, grads, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int moe_backward_launch_count(const moe_layer_desc_t* d) {
+  if (check_desc(d) != MOE_OK || d->T == 0) return 0;
+  int n = d->dtype == MOE_DTYPE_BF16 ? 3 : 2;                        // router logits + top-k
+  n += static_cast<long long>(d->T) * d->k <= 2048 ? 1 : 3;          // counting sort
+  n += 1;                                                            // gather
+  n += 9;                                                            // 6 expert GEMMs, act, pairs, act grad
+  if (d->act == MOE_ACT_GELU_TANH && d->has_bias) n += 2;            // bias gradients
+  if (d->I_sh > 0) n += 7;                                           // shared expert
+  n += 3;                                                            // router backward, dW_r, router dx
+  n += 1;                                                            // dx combine
+  return n;
+}
+
+}  // extern "C"

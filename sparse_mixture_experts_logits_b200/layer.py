@@ -75,6 +75,7 @@ class MoELayer:
         base = self.ws.data_ptr()
         self._ws_off = (-base) % 256
         self.layout = abi.moe_workspace_layout(self.desc)
+        self._bws = None
 
     @property
     def ws_ptr(self) -> int:
@@ -96,7 +97,50 @@ class MoELayer:
     def device_status(self, stream=None) -> int:
         return abi.moe_device_status(self.ws_ptr, _stream_handle(stream))
 
-    def view(self, name: str, dtype=None) -> torch.Tensor:
+    def grad_shapes(self) -> dict:
+        """Shapes of the gradients moe_backward writes (None: not written)."""
+        d = self.desc
+        swiglu = d.act == abi.ACT_SWIGLU
+        n1 = 2 * d.I if swiglu else d.I
+        biases = (not swiglu) and bool(d.has_bias)
+        return {
+            "dx": (d.T, d.D), "dw_r": (d.D, d.M), "dw1": (d.M, n1, d.D), "dw2": (d.M, d.D, d.I),
+            "db1": (d.M, d.I) if biases else None, "db2": (d.M, d.D) if biases else None,
+            "dsh_w1": (2 * d.I_sh, d.D) if d.I_sh else None, "dsh_w2": (d.D, d.I_sh) if d.I_sh else None,
+        }
+
+    def backward(self, x: torch.Tensor, dy: torch.Tensor, grads: dict | None = None, stream=None) -> dict:
+        """Gradients of L = sum(dy * MoE-FFN(x)) (moe_backward): dx in the
+        layer's dtype, every parameter gradient in fp32.  The backward has its
+        own workspace (allocated on first use); ``backward_view`` reads the
+        routing it recomputed."""
+        if self._bws is None:
+            self.bws_bytes = abi.moe_backward_workspace_size(self.desc)
+            if self.bws_bytes == 0:
+                raise abi.MoEError("moe_backward_workspace_size", abi.MOE_ERR_INVALID_ARG)
+            self._bws = torch.zeros(self.bws_bytes + 256, dtype=torch.uint8, device=self.device)
+            self._bws_off = (-self._bws.data_ptr()) % 256
+        if grads is None:
+            grads = {}
+            for name, shape in self.grad_shapes().items():
+                if shape is not None:
+                    dt = x.dtype if name == "dx" else torch.float32
+                    grads[name] = torch.empty(shape, dtype=dt, device=self.device)
+        g = abi.Grads()
+        for name in abi.Grads._fields_:
+            setattr(g, name[0], _ptr(grads.get(name[0])))
+        abi.moe_backward(self.desc, self.weights, x.data_ptr(), dy.data_ptr(), g,
+                         self._bws.data_ptr() + self._bws_off, self.bws_bytes, _stream_handle(stream))
+        return grads
+
+    def backward_status(self, stream=None) -> int:
+        return abi.moe_device_status(self._bws.data_ptr() + self._bws_off, _stream_handle(stream))
+
+    def backward_view(self, name: str) -> torch.Tensor:
+        """The routing intermediate ``name`` of the last backward."""
+        return self.view(name, ws=(self._bws, self._bws_off))
+
+    def view(self, name: str, dtype=None, ws=None) -> torch.Tensor:
         """The intermediate ``name`` of the last forward, as a tensor view."""
         d = self.desc
         pairs = d.T * d.k
@@ -108,12 +152,13 @@ class MoELayer:
             "out_perm": ((pairs, d.D), torch.float32),
         }
         shape, dt = shapes[name]
-        off = self._ws_off + getattr(self.layout, name)
+        buf, base = (self.ws, self._ws_off) if ws is None else ws
+        off = base + getattr(self.layout, name)
         n = 1
         for s in shape:
             n *= s
         nbytes = n * torch.empty((), dtype=dt).element_size()
-        return self.ws[off:off + nbytes].view(dt).view(*shape)
+        return buf[off:off + nbytes].view(dt).view(*shape)
 
 
 class DenseLayer:

@@ -171,3 +171,37 @@ def test_algorithmic_work_closed_form(B):
     d5 = B.desc_from_config(cfg5)
     f5, b5 = B.moe_algorithmic_work(d5, np.zeros(cfg5["M"], np.int32))
     assert b5 == 37748736 * 2 + 6144 * 256 * 2 + 4 * 256 + 2 * cfg5["T"] * 6144 * 2
+
+
+def test_backward_host_checks(B):
+    """moe_backward validates its descriptor and every required gradient
+    pointer before touching the device."""
+    for name in ms.all_config_names():
+        d = _desc(B, name)
+        assert B.moe_backward_workspace_size(d) > B.moe_workspace_size(d)
+        assert B.moe_backward_launch_count(d) > B.moe_forward_launch_count(d)
+    d = _desc(B, "glm_small_bf16")
+    w = B.Weights()
+    w.w_r, w.w1, w.w2, w.sh_w1, w.sh_w2 = 256, 256, 256, 256, 256
+    full = dict(dx=256, dw_r=256, dw1=256, dw2=256, dsh_w1=256, dsh_w2=256)
+    need = B.moe_backward_workspace_size(d)
+    for missing in ("dw_r", "dw1", "dw2", "dsh_w1", "dsh_w2"):
+        g = B.Grads(**{k: v for k, v in full.items() if k != missing})
+        with pytest.raises(B.MoEError) as e:
+            B.moe_backward(d, w, 256, 256, g, 256, need)
+        assert e.value.status == 1, missing
+    g = B.Grads(**full)
+    with pytest.raises(B.MoEError) as e:     # workspace one byte short
+        B.moe_backward(d, w, 256, 256, g, 256, need - 1)
+    assert e.value.status == 1
+    # GELU with biases needs db1 and db2
+    dg = _desc(B, "glam_small_bf16")
+    wg = B.Weights()
+    wg.w_r, wg.w1, wg.w2, wg.b1, wg.b2 = 256, 256, 256, 256, 256
+    with pytest.raises(B.MoEError) as e:
+        B.moe_backward(dg, wg, 256, 256, B.Grads(dx=256, dw_r=256, dw1=256, dw2=256, db1=256), 256,
+                       B.moe_backward_workspace_size(dg))
+    assert e.value.status == 1
+    bad = _desc(B, "glm_small_bf16")
+    bad.k = 0
+    assert B.moe_backward_workspace_size(bad) == 0 and B.moe_backward_launch_count(bad) == 0

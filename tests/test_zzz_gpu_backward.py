@@ -1,0 +1,196 @@
+"""Parity of the layer backward (moe_backward) with the fp64 CPU backward
+oracle, through the C ABI, on identical seeded inputs.
+
+The GPU recomputes the routing; where its top-k differs from the oracle's
+only at a near-tie, the oracle takes the GPU's choice (as in the forward
+tests).  Every gradient of the GPU is fp32 sums of the layer-dtype inputs
+with fp32 intermediates, so against the fp64 oracle the parameter
+gradients agree to a few fp32 ulps times the length of the sums; the bound
+below leaves two orders of magnitude of room.  dx of a bf16 layer is
+rounded to bf16 once and is held to the forward's output tolerance.
+
+Collected after every forward suite (test_zzz_*), so that a run stopping at
+the first failure has already checked the forward path."""
+import numpy as np
+import pytest
+import torch
+
+import moe_synth as ms
+import oracle
+from gpu_common import check_routing, check_y, gpu_inputs, np64, oracle_route
+
+pytestmark = pytest.mark.gpu
+
+GRAD_MAX_OVER_RMS = 1e-3   # max |g - g_ref| <= 1e-3 * rms(g_ref)
+GRAD_MEAN_REL = 1e-4       # sum |g - g_ref| / sum |g_ref| <= 1e-4
+PARAM_GRADS = ("dw_r", "dw1", "dw2", "db1", "db2", "dsh_w1", "dsh_w2")
+
+
+@pytest.fixture(scope="module")
+def B():
+    import sparse_mixture_experts_logits_b200 as B
+    return B
+
+
+def host(inp, rows=None):
+    out = {}
+    for k, v in inp.items():
+        if v is None:
+            out[k] = None
+        elif k == "x" and rows is not None:
+            out[k] = np64(v[torch.as_tensor(rows, device=v.device)])
+        else:
+            out[k] = np64(v)
+    return out
+
+
+def run(B, cfg):
+    inp = gpu_inputs(cfg)
+    dy = ms.upstream_grad(cfg, "cuda")
+    layer = B.MoELayer(cfg, inp)
+    g = layer.backward(inp["x"], dy)
+    torch.cuda.synchronize()
+    assert layer.backward_status() == 0
+    idx = layer.backward_view("topk_idx").cpu().numpy()
+    w = layer.backward_view("topk_w").cpu().numpy()
+    w_ref, _ = check_routing(cfg, oracle_route(cfg, inp), idx, w)
+    return inp, dy, layer, g, idx, w_ref
+
+
+def compact(cfg, inp, rows, idx):
+    """The layer restricted to tokens ``rows`` and to the experts they chose
+    (renumbered 0..m-1), as fp64 host arrays.  With the choice given, a
+    token's weights depend only on its chosen experts' scores (renormalised
+    softmax, sigmoid), so the restricted layer's dx of those tokens is the
+    full layer's."""
+    assert cfg["gate"] == "sigmoid_bias" or cfg["norm_topk_prob"]
+    used = np.unique(idx[rows])
+    pos = {int(e): i for i, e in enumerate(used)}
+    sel = torch.as_tensor(used, device=inp["w1"].device)
+    sub = {"x": np64(inp["x"][torch.as_tensor(rows, device=inp["x"].device)]),
+           "w_r": np64(inp["w_r"][:, sel])}
+    for k in ("e_bias", "w1", "w2", "b1", "b2"):
+        sub[k] = None if inp.get(k) is None else np64(inp[k][sel])
+    for k in ("sh_w1", "sh_w2"):
+        sub[k] = None if inp.get(k) is None else np64(inp[k])
+    sub_idx = np.vectorize(lambda e: pos[int(e)])(idx[rows])
+    return dict(cfg, T=len(rows), M=len(used), n_group=1, topk_group=1), sub, sub_idx
+
+
+def check_one_expert(cfg, inp, dy, idx, w_ref, g, e):
+    """Every gradient of expert e: its FFN backward over exactly the rows
+    routed to it, each scaled by its gate weight."""
+    tt, jj = np.nonzero(idx == e)
+    dyh = np64(dy[torch.as_tensor(tt, device=dy.device)])
+    b1, b2 = inp.get("b1"), inp.get("b2")
+    ref = oracle.moe_backward.expert_ffn_backward(
+        np64(inp["x"][torch.as_tensor(tt, device=dy.device)]), cfg["act"], np64(inp["w1"][e]),
+        np64(inp["w2"][e]), None if b1 is None else np64(b1[e]), None if b2 is None else np64(b2[e]),
+        w_ref[tt, jj][:, None] * dyh)
+    for name in ("dw1", "dw2", "db1", "db2"):
+        if ref[name] is not None:
+            check_grad(name, np64(g[name][e]), ref[name])
+
+
+def check_grad(name, got, ref):
+    m = oracle.error_metrics(got, ref)
+    assert m["max_over_rms"] <= GRAD_MAX_OVER_RMS and m["mean_rel"] <= GRAD_MEAN_REL, (name, m)
+
+
+def check_dx(cfg, got, ref):
+    if cfg["dtype"] == "f32":
+        check_grad("dx", got, ref)
+    else:
+        check_y(dict(cfg, named=False), got, ref)
+
+
+def check_all(cfg, g, ref):
+    check_dx(cfg, np64(g["dx"]), ref["dx"])
+    for name in PARAM_GRADS:
+        if ref[name] is None:
+            assert name not in g
+            continue
+        check_grad(name, np64(g[name]), ref[name])
+
+
+SMALL = ["glam_tiny_f32", "glam_small_bf16", "glm_small_bf16", "glm_small_f32", "glm_grouped_bf16",
+         "glm_grouped_f32", "glam_nonorm_f32"]
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_backward_matches_oracle(B, name):
+    cfg = ms.get_config(name)
+    inp, dy, _, g, idx, _ = run(B, cfg)
+    ref = oracle.moe_backward.moe_backward(cfg, host(inp), np64(dy), idx=idx)
+    check_all(cfg, g, ref)
+
+
+@pytest.mark.parametrize("name,over", [("glm_small_bf16", dict(T=1)), ("glm_small_bf16", dict(T=65)),
+                                       ("glm_small_bf16", dict(T=129, k=1)), ("glm_small_bf16", dict(k=16)),
+                                       ("glam_small_bf16", dict(M=1, k=1)), ("glm_small_f32", dict(T=200))])
+def test_backward_edge_shapes(B, name, over):
+    """A single token, ragged tiles, k = 1, k = M, one expert (softmax: its
+    weight is exactly 1, so the router gradient is exactly 0)."""
+    cfg = ms.get_config(name, **over)
+    inp, dy, _, g, idx, _ = run(B, cfg)
+    ref = oracle.moe_backward.moe_backward(cfg, host(inp), np64(dy), idx=idx)
+    check_all(cfg, g, ref)
+
+
+def test_backward_decode_full_size_sampled(B):
+    """GLM-4.5 decode (T = 32, D = 5120, 160 experts, k = 8, shared
+    expert): dx of two tokens, every gradient of one expert, and the shared
+    expert's gradients (a sum over all 32 tokens)."""
+    cfg = ms.get_config("glm45_decode_bf16")
+    inp, dy, _, g, idx, w_ref = run(B, cfg)
+    toks = np.array([0, cfg["T"] - 1])
+    sub_cfg, sub, sub_idx = compact(cfg, inp, toks, idx)
+    ref = oracle.moe_backward.moe_backward(sub_cfg, sub, np64(dy)[toks], idx=sub_idx)
+    check_dx(cfg, np64(g["dx"][torch.as_tensor(toks, device=dy.device)]), ref["dx"])
+    check_one_expert(cfg, inp, dy, idx, w_ref, g, int(idx[0, 0]))
+    sh = oracle.moe_backward.expert_ffn_backward(np64(inp["x"]), "swiglu", np64(inp["sh_w1"]),
+                                                 np64(inp["sh_w2"]), None, None, np64(dy))
+    check_grad("dsh_w1", np64(g["dsh_w1"]), sh["dw1"])
+    check_grad("dsh_w2", np64(g["dsh_w2"]), sh["dw2"])
+
+
+def test_backward_glam_full_size_sampled(B):
+    """The GLaM layer (T = 8192, D = 2048, 64 experts of H = 8192, top-2)
+    in the launch configuration the benchmark times: dx of sampled tokens
+    and every gradient of two experts; an expert no token chose has exactly
+    zero gradient."""
+    cfg = ms.get_config("glam_prefill_bf16")
+    inp, dy, layer, g, idx, w_ref = run(B, cfg)
+    toks = np.array([0, 1, 4095, 5000, 8190, 8191])
+    sub_cfg, sub, sub_idx = compact(cfg, inp, toks, idx)
+    ref = oracle.moe_backward.moe_backward(sub_cfg, sub, np64(dy)[toks], idx=sub_idx)
+    check_dx(cfg, np64(g["dx"][torch.as_tensor(toks, device=dy.device)]), ref["dx"])
+    counts = layer.backward_view("counts").cpu().numpy()
+    busy = np.nonzero(counts > 0)[0]
+    for e in (int(busy[np.argmin(counts[busy])]), int(np.argmax(counts))):
+        check_one_expert(cfg, inp, dy, idx, w_ref, g, e)
+    for z in np.nonzero(counts == 0)[0][:2]:
+        assert float(g["dw1"][int(z)].abs().max()) == 0.0
+
+
+def test_backward_deterministic(B):
+    cfg = ms.get_config("glm_small_bf16")
+    inp, dy, layer, g1, _, _ = run(B, cfg)
+    g2 = layer.backward(inp["x"], dy)
+    torch.cuda.synchronize()
+    for name, t in g1.items():
+        assert torch.equal(t.view(torch.int16) if t.dtype == torch.bfloat16 else t.view(torch.int32),
+                           g2[name].view(torch.int16) if t.dtype == torch.bfloat16 else g2[name].view(torch.int32))
+
+
+def test_backward_zero_tokens_zero_fill(B):
+    cfg = ms.get_config("glm_small_bf16")
+    inp = gpu_inputs(cfg)
+    layer = B.MoELayer(cfg, inp, T=0)
+    grads = {n: torch.full(s, 7.0, device="cuda") for n, s in layer.grad_shapes().items()
+             if s is not None and n != "dx"}
+    grads["dx"] = torch.empty((0, cfg["D"]), dtype=torch.bfloat16, device="cuda")
+    layer.backward(inp["x"][:0], inp["x"][:0], grads=grads)
+    torch.cuda.synchronize()
+    for n, t in grads.items():
+        assert t.numel() == 0 or float(t.abs().max()) == 0.0, n

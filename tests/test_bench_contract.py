@@ -41,3 +41,25 @@ def test_reference_arm_line(config):
 def test_reference_arm_other_ranks_print_nothing():
     assert run_bench("--impl", "reference", "--config", "glam_small_bf16", "--steps", "1", "--warmup", "1",
                      "--ref-seconds", "1", env={"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
+
+
+@pytest.mark.parametrize("config", ["glam_small_bf16", "glm_small_bf16"])
+def test_backward_cpu_baseline_sample(config):
+    """The backward leg's CPU baseline (the fp64 backward oracle on the first
+    tokens, restricted to the experts they chose) runs on host tensors."""
+    sys.path.insert(0, ROOT)
+    import torch
+
+    import bench
+    import moe_synth as ms
+    import oracle
+
+    cfg = ms.get_config(config)
+    inp = ms.layer_inputs(cfg, "cpu")
+    dy = ms.upstream_grad(cfg, "cpu")
+    f64 = lambda t: None if t is None else t.to(torch.float64).numpy()  # noqa: E731
+    r = oracle.route(f64(inp["x"]), f64(inp["w_r"]), f64(inp["e_bias"]), cfg["k"], cfg["gate"],
+                     cfg["norm_topk_prob"], cfg["alpha"], cfg["eps"])
+    cb = bench.backward_cpu_baseline(cfg, inp, dy, r["idx"], target_s=0.05, max_experts=6)
+    assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["unit"] == "tokens/s" and cb["cores"] >= 1
+    assert "experts they chose" in cb["sample"]

@@ -203,6 +203,16 @@ moe_status_t moe_permute_static_scratch(const int32_t* topk_idx, const float* to
                                         int32_t* row_token, float* row_w, int32_t* device_status,
                                         void* stream);
 
+/* x_perm[s, :] = x[row_token[s], :] for s < min(rows, *n_rows) (n_rows a
+ * device int32, e.g. offsets + M, or NULL for all `rows`): the tokens'
+ * rows in dispatch order, contiguous, e.g. to send each expert owner its
+ * rows in one piece (expert parallelism).  x and x_perm in dtype; a
+ * row_token outside [0, T) gives a zero row and sets MOE_DEVERR_BAD_ROW_TOKEN
+ * in *device_status (a device int32, may be NULL). */
+moe_status_t moe_gather_rows(const void* x, const int32_t* row_token, const int32_t* n_rows,
+                             void* x_perm, int rows, int T, int D, int dtype,
+                             int32_t* device_status, void* stream);
+
 /* ---- experts: "GLaM" eq. FFN; GLM-5 GlmMoeDsaExperts.forward ----------- */
 
 size_t moe_expert_ffn_workspace_size(const moe_layer_desc_t* d);

@@ -27,7 +27,7 @@ EXPORTED_SYMBOLS = [
     "moe_combine", "moe_workspace_size", "moe_workspace_layout", "moe_forward",
     "moe_forward_profiled", "moe_forward_launch_count", "moe_algorithmic_work",
     "moe_forward_add", "moe_dense_ffn_workspace_size", "moe_dense_ffn", "moe_dense_ffn_profiled",
-    "moe_backward_workspace_size", "moe_backward", "moe_backward_launch_count",
+    "moe_backward_workspace_size", "moe_backward", "moe_backward_launch_count", "moe_gather_rows",
 ]
 NUM_STAGE_EVENTS = 9
 NUM_DENSE_EVENTS = 3
@@ -117,6 +117,7 @@ _decl("moe_dense_ffn_workspace_size", _sz, [_P(DenseDesc)])
 _decl("moe_dense_ffn", _i, [_P(DenseDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
 _decl("moe_dense_ffn_profiled", _i, [_P(DenseDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp,
                                      _P(_vp), _i])
+_decl("moe_gather_rows", _i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp])
 _decl("moe_backward_workspace_size", _sz, [_P(LayerDesc)])
 _decl("moe_backward", _i, [_P(LayerDesc), _P(Weights), _vp, _vp, _P(Grads), _vp, _sz, _vp])
 _decl("moe_backward_launch_count", _i, [_P(LayerDesc)])
@@ -267,3 +268,8 @@ def moe_backward(desc, weights, x, dy, grads, ws, ws_bytes, stream=None):
 
 def moe_backward_launch_count(desc) -> int:
     return lib.moe_backward_launch_count(ctypes.byref(desc))
+
+
+def moe_gather_rows(x, row_token, n_rows, x_perm, rows, T, D, dtype, device_status=None, stream=None):
+    _check("moe_gather_rows", lib.moe_gather_rows(x, row_token, n_rows, x_perm, rows, T, D, dtype, device_status,
+                                                  stream))

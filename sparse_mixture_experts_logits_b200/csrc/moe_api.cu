@@ -502,6 +502,17 @@ moe_status_t moe_permute(const int32_t* topk_idx, const float* topk_w, int T, in
   return MOE_OK;
 }
 
+moe_status_t moe_gather_rows(const void* x, const int32_t* row_token, const int32_t* n_rows, void* x_perm,
+                             int rows, int T, int D, int dtype, int32_t* device_status, void* stream) {
+  if (rows < 0 || T < 0 || D < 1) return MOE_ERR_INVALID_ARG;
+  if (dtype != MOE_DTYPE_F32 && dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (rows == 0) return MOE_OK;
+  if (!x || !row_token || !x_perm) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_device());
+  return cuda_status(launch_gather_rows(x, row_token, n_rows, x_perm, rows, T, D, static_cast<int>(esize(dtype)),
+                                        device_status, static_cast<cudaStream_t>(stream)));
+}
+
 size_t moe_expert_ffn_workspace_size(const moe_layer_desc_t* d) {
   if (check_desc(d) != MOE_OK) return 0;
   return ffn_layout(d).total;

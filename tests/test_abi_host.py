@@ -205,3 +205,16 @@ def test_backward_host_checks(B):
     bad = _desc(B, "glm_small_bf16")
     bad.k = 0
     assert B.moe_backward_workspace_size(bad) == 0 and B.moe_backward_launch_count(bad) == 0
+
+
+def test_gather_rows_host_checks(B):
+    with pytest.raises(B.MoEError) as e:
+        B.moe_gather_rows(256, 256, None, 256, -1, 4, 8, 1)
+    assert e.value.status == 1
+    with pytest.raises(B.MoEError) as e:
+        B.moe_gather_rows(256, 256, None, 256, 4, 4, 8, 7)
+    assert e.value.status == 2
+    with pytest.raises(B.MoEError) as e:
+        B.moe_gather_rows(None, 256, None, 256, 4, 4, 8, 1)
+    assert e.value.status == 1
+    B.moe_gather_rows(None, None, None, None, 0, 4, 8, 1)   # zero rows: nothing to do

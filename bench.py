@@ -865,10 +865,11 @@ def run_backward(args):
         "metric": "MoE layer backward throughput (all gradients; routing and expert forward recomputed)",
         "value": world * T / (ms_step / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": cfg["dtype"] + " in, fp32 sums and gradients",
+        "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded counter-based generator; random-init weights)",
         "config": {"workload": args.config, "T_per_gpu": T, "D": D, "M": cfg["M"], "k": cfg["k"],
-                   "I": cfg["I"], "I_sh": cfg.get("I_sh", 0),
+                   "I": cfg["I"], "I_sh": cfg.get("I_sh", 0), "inputs": cfg["dtype"],
+                   "arithmetic": "fp32 on the CUDA cores (inputs widened from the layer dtype)",
                    "l2": "flushed between steps (256 MiB write outside the timed events)",
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",

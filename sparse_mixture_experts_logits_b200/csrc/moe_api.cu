@@ -30,18 +30,18 @@ inline size_t esize(int dtype) { return dtype == MOE_DTYPE_BF16 ? 2 : 4; }
 
 // Every entry point runs only on compute capability 10.0 (sm_100a code).
 moe_status_t check_device() {
-  static std::atomic<int> verdict[64];
+  static std::atomic<int> arch_ok[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
   if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
-  int v = verdict[dev].load();
+  int v = arch_ok[dev].load();
   if (v == 0) {
     int major = 0, minor = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
       return MOE_ERR_CUDA;
     v = (major == 10 && minor == 0) ? 1 : 2;
-    verdict[dev].store(v);
+    arch_ok[dev].store(v);
   }
   return v == 1 ? MOE_OK : MOE_ERR_UNSUPPORTED;
 }

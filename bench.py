@@ -60,6 +60,8 @@ def parse_args():
     ap.add_argument("--M", type=int, default=None, help="override routed experts (profiling runs)")
     ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward"],
                     help="backward: time moe_backward (all gradients of the layer) instead of the forward")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism: each of the N ranks owns M/N experts, rows exchanged by all-to-all")
     return ap.parse_args()
 
 
@@ -890,10 +892,83 @@ def run_backward(args):
         dist.destroy_process_group()
 
 
+def run_ep(args):
+    """One step = the expert-parallel forward (sparse_mixture_experts_logits_b200.ep) on
+    every rank's own T tokens: route, exchange, local experts, exchange back, combine."""
+    import sparse_mixture_experts_logits_b200 as B
+    from sparse_mixture_experts_logits_b200 import ep
+
+    rank, local_rank, world = dist_env()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = dist_init(world, local_rank)
+    cfg = workload_config(args)
+    T, D = cfg["T"], cfg["D"]
+    full = ms.layer_inputs(dict(cfg, T=1), dev)
+    mine = ep.local_expert_tensors(full, rank, world)
+    del full
+    r0, r1 = token_rows(rank, T)
+    x = ms.normal_rows(torch.arange(r0, r1, device=dev), D, 1.0, ms._key(cfg, "x"), ms.act_dtype(cfg))
+    layer = ep.ExpertParallelMoE(cfg, mine, rank, world)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(max(3, args.warmup)):
+        layer.forward(x)
+    torch.cuda.synchronize()
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    recv, launches = [], 0
+    for i in range(K):
+        flush.zero_()
+        starts[i].record(stream)
+        layer.forward(x)
+        ends[i].record(stream)
+        recv.append(layer.last_plan.rows_received)
+        launches += layer.launch_count(T, recv[-1])
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    if dist is not None:
+        dist.barrier()
+    ms_step = max_over_ranks(dist, sum(starts[i].elapsed_time(ends[i]) for i in range(K)) / K, dev)
+    if int(layer.status.item()) != 0:
+        raise RuntimeError("device status flag set during the timed steps")
+    if rank == 0:
+        rows_out = (world - 1) / max(1, world) * T * cfg["k"]  # rows that leave the rank, on average
+        out = {
+            "metric": "MoE layer forward throughput, expert-parallel (routed experts split over the ranks)",
+            "value": world * T / (ms_step / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": cfg["dtype"],
+            "data": "synthetic (seeded counter-based generator; random-init weights)",
+            "config": {"workload": args.config, "T_per_gpu": T, "D": D, "M": cfg["M"], "k": cfg["k"],
+                       "I": cfg["I"], "I_sh": cfg.get("I_sh", 0), "parallelism": f"ep{world}",
+                       "l2": "flushed between steps (256 MiB write outside the timed events)"},
+            "exchange": {"rows_received_rank0_mean": float(np.mean(recv)),
+                         "rows_leaving_each_rank_expected": rows_out,
+                         "bytes_out_per_rank_expected": rows_out * D * (2 if cfg["dtype"] == "bf16" else 4)
+                         + rows_out * 4 + rows_out * D * 4},
+            "e2e": None, "gpu_launches": launches, "gpu_launches_note": "rank 0's own kernels; NCCL's not counted",
+            "clocks": clocks,
+        }
+        print(json.dumps(out), flush=True)
+    del layer
+    if dist is not None:
+        dist.destroy_process_group()
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.ep:
+        run_ep(args)
     elif args.which == "backward":
         run_backward(args)
     elif is_dense(workload_config(args)):

@@ -152,6 +152,21 @@ class ExpertParallelMoE:
         self.w_shared = abi.Weights()
         self.w_shared.sh_w1, self.w_shared.sh_w2 = _ptr(tensors.get("sh_w1")), _ptr(tensors.get("sh_w2"))
 
+    def launch_count(self, T: int, rows_received: int) -> int:
+        """Kernels of the library one forward on this rank launches (the
+        collectives' own kernels not counted)."""
+        bf16 = self.cfg["dtype"] == "bf16"
+        k = self.cfg["k"]
+        n = 3 if bf16 else 2                                  # router logits + top-k
+        n += 1 if T * k <= 2048 else 3                        # dispatch order
+        n += 1                                                # rows into dispatch order
+        if rows_received > 0:
+            n += 1 if rows_received <= 2048 else 3            # received rows by local expert
+            n += 3 if bf16 else 2                             # [gather,] the expert GEMMs
+            n += 1                                            # back to arrival order
+        n += 2 if self.cfg.get("I_sh") else 0                 # shared expert
+        return n + 1                                          # combine
+
     def _desc(self, T, M=None, k=None, dtype=None):
         d = desc_from_config(self.cfg, T)
         if M is not None:

@@ -37,6 +37,9 @@ design notes):
     selection scores (its only score when a group holds one expert); the
     topk_group best groups (ties to the lower group index) stay eligible and
     every other expert is excluded from the top-k.  n_group = 1 is no mask.
+  * Expert capacity (no page gives a rule): expert e keeps the first
+    ceil(factor T k / M) of its pairs in the dispatch order above and the
+    rest become the sentinel below; weights are not renormalised.
   * Expert index M (one past the last expert) is the "no expert" sentinel of
     the quoted GlmMoeDsaExperts.forward (one_hot over M + 1 classes, class M
     skipped): such a (token, slot) pair is dispatched nowhere and adds
@@ -54,7 +57,8 @@ import numpy as np
 
 __all__ = [
     "gelu_tanh", "silu", "sigmoid", "router_logits", "selection_scores",
-    "topk_select", "group_limit", "topk_weights", "route", "permute", "expert_ffn",
+    "topk_select", "group_limit", "topk_weights", "route", "permute", "expert_capacity", "capacity_drop",
+    "expert_ffn",
     "shared_expert", "moe_tokens", "moe_forward", "dense_layer", "adopt_topk",
     "param_count", "error_metrics",
 ]
@@ -255,6 +259,33 @@ def permute(idx, w, M):
         row_w = _f64(w).T.reshape(-1)[order]
     return {"counts": counts, "offsets": offsets, "slot_of": slot_of,
             "row_token": row_token, "row_w": row_w}
+
+
+def expert_capacity(factor, T, k, M):
+    """Pairs an expert may take: ceil(factor * T * k / M) (reading r23: the
+    pages name no capacity rule; a capacity factor of 1 lets every expert
+    take exactly its even share of the T k pairs)."""
+    if factor < 0 or M < 1:
+        raise ValueError("bad capacity")
+    return int(np.ceil(factor * T * k / M - 1e-12)) if T * k > 0 else 0
+
+
+def capacity_drop(idx, M, capacity):
+    """Expert capacity over the dispatch order of ``permute`` (reading r23):
+    expert e keeps the first ``capacity`` of its pairs in (slot j, then token
+    t) order, so every token's first choice ranks before any second choice;
+    each later pair becomes the sentinel M, which [GLM5-SE]
+    GlmMoeDsaExperts.forward skips.  Weights are left as they are: a dropped
+    pair adds nothing, and the token's other terms keep their weights."""
+    idx = np.asarray(idx, dtype=np.int64)
+    if capacity < 0:
+        raise ValueError("capacity < 0")
+    p = permute(idx, None, M)
+    out = idx.copy()
+    kept = idx < M
+    rank = p["slot_of"] - p["offsets"][np.where(kept, idx, 0)]
+    out[kept & (rank >= capacity)] = M
+    return out
 
 
 # ---------------------------------------------------------------------------

@@ -470,9 +470,42 @@ def pin_adopt_topk(O):
     assert not ok
 
 
+def pin_capacity_drop(O):
+    """Expert capacity against a scalar loop over the (slot, token) order:
+    a per-expert counter admits a pair while it is below the capacity.
+    Invariants: kept counts never exceed it, an ample capacity drops nothing,
+    a zero capacity drops everything, sentinels in the input stay."""
+    rng = np.random.default_rng(21)
+    for T, k, M in ((40, 2, 5), (33, 4, 8), (7, 3, 3)):
+        idx = np.stack([rng.choice(M, size=k, replace=False) for _ in range(T)])
+        idx[rng.random(idx.shape) < 0.1] = M
+        for cap in (0, 1, 3, (T * k) // M, T * k):
+            ref = idx.copy()
+            seen = [0] * M
+            for j in range(k):
+                for t in range(T):
+                    e = int(idx[t, j])
+                    if e == M:
+                        continue
+                    if seen[e] >= cap:
+                        ref[t, j] = M
+                    else:
+                        seen[e] += 1
+            got = O.capacity_drop(idx, M, cap)
+            assert np.array_equal(got, ref), (T, k, M, cap)
+            kept = got[got < M]
+            assert (np.bincount(kept, minlength=M) <= cap).all()
+        assert np.array_equal(O.capacity_drop(idx, M, T * k), idx)
+        assert (O.capacity_drop(idx, M, 0) == M).all()
+    assert O.expert_capacity(1.0, 8192, 2, 64) == 256
+    assert O.expert_capacity(1.25, 300, 4, 16) == 94
+    assert O.expert_capacity(0.0, 300, 4, 16) == 0
+
+
 ALL_PINS = [
     pin_gelu, pin_silu_sigmoid, pin_topk_bruteforce, pin_softmax_top2_closed_form,
     pin_sigmoid_router, pin_bias_selects_only, pin_group_limit, pin_permute, pin_sentinel, pin_bruteforce_forward,
     pin_single_expert_is_dense_ffn, pin_k_equals_m, pin_shared_branch,
     pin_sum_no_residual, pin_dense_layer, pin_param_counts, pin_error_metrics, pin_adopt_topk,
+    pin_capacity_drop,
 ]

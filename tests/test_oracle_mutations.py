@@ -156,11 +156,32 @@ def m_dense_no_b2(O):
                                                                                 addend)
 
 
+def m_capacity_token_major(O):
+    def drop(idx, M, capacity):
+        idx = np.asarray(idx, np.int64)
+        out = idx.copy()
+        seen = np.zeros(M, np.int64)
+        for t in range(idx.shape[0]):          # token first: a later token's first choice loses
+            for j in range(idx.shape[1]):
+                e = idx[t, j]
+                if e < M:
+                    if seen[e] >= capacity:
+                        out[t, j] = M
+                    seen[e] += 1
+        return out
+    O.capacity_drop = drop
+
+
+def m_capacity_off_by_one(O):
+    orig = O.capacity_drop
+    O.capacity_drop = lambda idx, M, capacity: orig(idx, M, capacity + 1)
+
+
 MUTANTS = [m_swap_gate_up, m_drop_b2, m_bias_in_weights, m_tie_to_higher_index,
            m_no_renorm, m_no_alpha, m_token_major_dispatch, m_gelu_erf,
            m_shared_missing, m_transposed_router, m_wrong_param_count, m_group_score_max,
            m_group_score_all, m_group_mask_zero, m_group_tie_high, m_dense_drops_addend, m_dense_no_b2,
-           m_block_drops_addend]
+           m_block_drops_addend, m_capacity_token_major, m_capacity_off_by_one]
 
 
 @pytest.mark.parametrize("mutant", MUTANTS, ids=lambda f: f.__name__)

@@ -203,6 +203,22 @@ moe_status_t moe_permute_static_scratch(const int32_t* topk_idx, const float* to
                                         int32_t* row_token, float* row_w, int32_t* device_status,
                                         void* stream);
 
+/* Expert capacity (the pages give no capacity rule; this is the plain one):
+ * an expert takes at most `capacity` pairs, the first ones in moe_permute's
+ * dispatch order (slot j, then token t: every first choice before any
+ * second choice), and every later pair's index becomes the sentinel M, which
+ * the dispatch and the combine skip.  Gate weights are left as they are (a
+ * dropped pair adds nothing).  topk_idx [T, k] is rewritten in place;
+ * slot_of and offsets are what moe_permute produced for it.  Run
+ * moe_permute again afterwards to get the dispatch of the kept pairs.
+ * capacity >= 0; 0 < M <= 1024; T = 0 launches nothing. */
+moe_status_t moe_capacity_drop(int32_t* topk_idx, const int32_t* slot_of, const int32_t* offsets,
+                               int T, int k, int M, int capacity, void* stream);
+
+/* ceil(factor * T * k / M): with factor 1 every expert may take exactly its
+ * even share of the T k pairs.  -1 for factor < 0, M < 1, T < 0 or k < 1. */
+int moe_expert_capacity(double factor, int T, int k, int M);
+
 /* x_perm[s, :] = x[row_token[s], :] for s < min(rows, *n_rows) (n_rows a
  * device int32, e.g. offsets + M, or NULL for all `rows`): the tokens'
  * rows in dispatch order, contiguous, e.g. to send each expert owner its

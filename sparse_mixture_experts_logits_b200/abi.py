@@ -28,6 +28,7 @@ EXPORTED_SYMBOLS = [
     "moe_forward_profiled", "moe_forward_launch_count", "moe_algorithmic_work",
     "moe_forward_add", "moe_dense_ffn_workspace_size", "moe_dense_ffn", "moe_dense_ffn_profiled",
     "moe_backward_workspace_size", "moe_backward", "moe_backward_launch_count", "moe_gather_rows",
+    "moe_capacity_drop", "moe_expert_capacity",
 ]
 NUM_STAGE_EVENTS = 9
 NUM_DENSE_EVENTS = 3
@@ -118,6 +119,8 @@ _decl("moe_dense_ffn", _i, [_P(DenseDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _v
 _decl("moe_dense_ffn_profiled", _i, [_P(DenseDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp,
                                      _P(_vp), _i])
 _decl("moe_gather_rows", _i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp])
+_decl("moe_capacity_drop", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp])
+_decl("moe_expert_capacity", _i, [ctypes.c_double, _i, _i, _i])
 _decl("moe_backward_workspace_size", _sz, [_P(LayerDesc)])
 _decl("moe_backward", _i, [_P(LayerDesc), _P(Weights), _vp, _vp, _P(Grads), _vp, _sz, _vp])
 _decl("moe_backward_launch_count", _i, [_P(LayerDesc)])
@@ -273,3 +276,11 @@ def moe_backward_launch_count(desc) -> int:
 def moe_gather_rows(x, row_token, n_rows, x_perm, rows, T, D, dtype, device_status=None, stream=None):
     _check("moe_gather_rows", lib.moe_gather_rows(x, row_token, n_rows, x_perm, rows, T, D, dtype, device_status,
                                                   stream))
+
+
+def moe_capacity_drop(topk_idx, slot_of, offsets, T, k, M, capacity, stream=None):
+    _check("moe_capacity_drop", lib.moe_capacity_drop(topk_idx, slot_of, offsets, T, k, M, capacity, stream))
+
+
+def moe_expert_capacity(factor, T, k, M) -> int:
+    return lib.moe_expert_capacity(float(factor), T, k, M)

@@ -31,6 +31,10 @@ cudaError_t launch_permute(const int32_t* topk_idx, const float* topk_w, int T, 
                            float* row_w, int32_t* chunk_counts, int32_t* chunk_base, int* status,
                            cudaStream_t s);
 
+// capacity.cu: idx[p] := M where slot_of[p] - offsets[idx[p]] >= capacity (in place).
+cudaError_t launch_capacity_drop(int32_t* idx, const int32_t* slot_of, const int32_t* offsets, int T, int k, int M,
+                                 int capacity, cudaStream_t s);
+
 // misc.cu
 // bf16 rows of x into dispatch order by token: x_perm[slot_of[t, j]] = x[t] (D % 8 == 0).
 cudaError_t launch_scatter_rows(const void* x, const int32_t* slot_of, void* x_perm, int T, int k, int D,

@@ -1,6 +1,7 @@
 // C ABI of the MoE layer forward: argument checks, workspace layouts and
 // the sequence of kernel launches of every entry point (see moe_b200.h).
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <cstring>
 
@@ -500,6 +501,23 @@ moe_status_t moe_permute(const int32_t* topk_idx, const float* topk_w, int T, in
   MOE_CUDA(launch_permute(topk_idx, topk_w, T, k, M, counts, offsets, slot_of, row_token, row_w,
                           at<int32_t*>(ws, L.chunk_counts), at<int32_t*>(ws, L.chunk_base), status, s));
   return MOE_OK;
+}
+
+moe_status_t moe_capacity_drop(int32_t* topk_idx, const int32_t* slot_of, const int32_t* offsets, int T, int k,
+                               int M, int capacity, void* stream) {
+  if (T < 0 || k < 1 || M < 1 || capacity < 0) return MOE_ERR_INVALID_ARG;
+  if (M > kMaxExperts || static_cast<long long>(T) * k >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!topk_idx || !slot_of || !offsets) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_device());
+  return cuda_status(launch_capacity_drop(topk_idx, slot_of, offsets, T, k, M, capacity,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+int moe_expert_capacity(double factor, int T, int k, int M) {
+  if (!(factor >= 0.0) || M < 1 || T < 0 || k < 1) return -1;
+  const double c = std::ceil(factor * static_cast<double>(T) * k / M - 1e-12);
+  return c > 2147483647.0 ? 2147483647 : static_cast<int>(c);
 }
 
 moe_status_t moe_gather_rows(const void* x, const int32_t* row_token, const int32_t* n_rows, void* x_perm,

@@ -218,3 +218,17 @@ def test_gather_rows_host_checks(B):
         B.moe_gather_rows(None, 256, None, 256, 4, 4, 8, 1)
     assert e.value.status == 1
     B.moe_gather_rows(None, None, None, None, 0, 4, 8, 1)   # zero rows: nothing to do
+
+
+def test_capacity_host_checks(B):
+    import oracle
+    for factor, T, k, M in ((1.0, 8192, 2, 64), (1.25, 300, 4, 16), (0.5, 333, 2, 8), (0.0, 10, 2, 4),
+                            (2.0, 1, 8, 160), (1.0, 0, 2, 8)):
+        assert B.moe_expert_capacity(factor, T, k, M) == oracle.expert_capacity(factor, T, k, M)
+    assert B.moe_expert_capacity(-1.0, 10, 2, 4) == -1 and B.moe_expert_capacity(1.0, 10, 2, 0) == -1
+    for args, status in [((256, 256, 256, 10, 2, 8, -1), 1), ((256, 256, 256, 10, 0, 8, 4), 1),
+                         ((None, 256, 256, 10, 2, 8, 4), 1), ((256, 256, 256, 10, 2, 2000, 4), 2)]:
+        with pytest.raises(B.MoEError) as e:
+            B.moe_capacity_drop(*args)
+        assert e.value.status == status
+    B.moe_capacity_drop(None, None, None, 0, 2, 8, 4)   # T = 0: nothing to do

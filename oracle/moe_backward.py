@@ -17,8 +17,7 @@ the chain rule applied to one forward step, in the forward's notation:
              g-bar_i, E_sh, eq. y.
   [GLM5-SE]  "GLM-5 - Shared expert", section "All 5 steps" (SwiGLU).
 
-Readings (the pages describe training only in prose; each reading is also
-listed in the design notes):
+Readings (the pages describe training only in prose):
   * The top-k choice S_t is a discrete function of the scores: its
     derivative is zero wherever it is defined, so the gradient flows only
     through the weights w_{t,j} of the experts already chosen and through

@@ -17,8 +17,7 @@ passage of the source pages, cited by page title and section/equation:
              "Exact per-instance accounting" and the quoted
              GlmMoeDsaExperts / GlmMoeDsaMoE / GlmMoeDsaMLP forward excerpts.
 
-Readings taken where the pages leave a step open (each is also listed in the
-design notes):
+Readings taken where the pages leave a step open:
   * GLaM's "normalized gate weight": the softmax probabilities of the k
     selected experts renormalised to sum to one; because the full softmax
     denominator cancels, alpha_j = exp(l_j - l_max) / sum_S exp(l - l_max).
@@ -262,21 +261,21 @@ def permute(idx, w, M):
 
 
 def expert_capacity(factor, T, k, M):
-    """Pairs an expert may take: ceil(factor * T * k / M) (reading r23: the
-    pages name no capacity rule; a capacity factor of 1 lets every expert
-    take exactly its even share of the T k pairs)."""
+    """Pairs an expert may take: ceil(factor * T * k / M).  The pages name no
+    capacity rule; this is the plain one, under which a capacity factor of 1
+    lets every expert take exactly its even share of the T k pairs."""
     if factor < 0 or M < 1:
         raise ValueError("bad capacity")
     return int(np.ceil(factor * T * k / M - 1e-12)) if T * k > 0 else 0
 
 
 def capacity_drop(idx, M, capacity):
-    """Expert capacity over the dispatch order of ``permute`` (reading r23):
-    expert e keeps the first ``capacity`` of its pairs in (slot j, then token
-    t) order, so every token's first choice ranks before any second choice;
-    each later pair becomes the sentinel M, which [GLM5-SE]
-    GlmMoeDsaExperts.forward skips.  Weights are left as they are: a dropped
-    pair adds nothing, and the token's other terms keep their weights."""
+    """Expert capacity over the dispatch order of ``permute`` (a reading: the
+    pages give no rule).  Expert e keeps the first ``capacity`` of its pairs
+    in (slot j, then token t) order, so every token's first choice ranks
+    before any second choice; each later pair becomes the sentinel M, which
+    [GLM5-SE] GlmMoeDsaExperts.forward skips.  Weights are left as they are:
+    a dropped pair adds nothing, and the token's other terms keep theirs."""
     idx = np.asarray(idx, dtype=np.int64)
     if capacity < 0:
         raise ValueError("capacity < 0")

@@ -780,7 +780,7 @@ def backward_cpu_baseline(cfg, inp, dy, idx, target_s, max_experts=16):
     while True:
         used = np.unique(idx[:n])
         pos = {int(e): i for i, e in enumerate(used)}
-        sel = torch.as_tensor(used, device=inp["w1"].device)
+        sel = torch.as_tensor(used.astype(np.int64), device=inp["w1"].device)
         sub = {"x": f64(inp["x"][:n]), "w_r": f64(inp["w_r"][:, sel])}
         for k in ("e_bias", "w1", "w2", "b1", "b2"):
             sub[k] = None if inp.get(k) is None else f64(inp[k][sel])

@@ -66,7 +66,7 @@ def compact(cfg, inp, rows, idx):
     assert cfg["gate"] == "sigmoid_bias" or cfg["norm_topk_prob"]
     used = np.unique(idx[rows])
     pos = {int(e): i for i, e in enumerate(used)}
-    sel = torch.as_tensor(used, device=inp["w1"].device)
+    sel = torch.as_tensor(used.astype(np.int64), device=inp["w1"].device)
     sub = {"x": np64(inp["x"][torch.as_tensor(rows, device=inp["x"].device)]),
            "w_r": np64(inp["w_r"][:, sel])}
     for k in ("e_bias", "w1", "w2", "b1", "b2"):

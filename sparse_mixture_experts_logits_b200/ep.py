@@ -137,6 +137,8 @@ class ExpertParallelMoE:
     (w1/w2/b1/b2 with E = M / world rows each, see local_expert_tensors) and
     the shared expert, all on this rank's device."""
 
+    out_dtype = torch.float32  # the experts' outputs as they travel back (moe_expert_ffn's fp32 rows)
+
     def __init__(self, cfg: dict, tensors: dict, rank: int, world: int, group=None):
         self.cfg = cfg
         self.rank, self.world, self.group = rank, world, group
@@ -182,71 +184,104 @@ class ExpertParallelMoE:
         buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
         return buf, buf.data_ptr() + (-buf.data_ptr()) % 256
 
-    def forward(self, x: torch.Tensor, stream=None) -> torch.Tensor:
-        cfg, dev = self.cfg, self.device
+    # ---- the library's kernels, one method per step (tensors in, tensors out) ----
+
+    def _route(self, x):
+        """topk_idx [T, k] int32 and topk_w [T, k] fp32 (moe_route_topk)."""
         T, D = x.shape
-        M, k = self.M, cfg["k"]
-        s = _stream_handle(stream)
+        M, k = self.M, self.cfg["k"]
         d = self._desc(T)
-        i32 = dict(dtype=torch.int32, device=dev)
-        f32 = dict(dtype=torch.float32, device=dev)
-        status = torch.zeros(1, **i32)
-        # 1. route and dispatch this rank's tokens
-        idx = torch.empty((T, k), **i32)
-        tw = torch.empty((T, k), **f32)
-        rbuf, rws = self._ws(abi.moe_route_workspace_size(T, D, M, d.dtype), dev)
+        idx = torch.empty((T, k), dtype=torch.int32, device=self.device)
+        tw = torch.empty((T, k), dtype=torch.float32, device=self.device)
+        buf, ws = self._ws(abi.moe_route_workspace_size(T, D, M, d.dtype), self.device)
         abi.moe_route_topk(x.data_ptr(), _ptr(self.t["w_r"]), _ptr(self.t.get("e_bias")), T, D, M, k, d.dtype,
                            d.gate, d.norm_topk_prob, d.routed_scaling_factor, d.eps, d.n_group, d.topk_group,
-                           idx.data_ptr(), tw.data_ptr(), rws, rbuf.numel() - 256, s)
-        counts = torch.empty(M, **i32)
-        offsets = torch.empty(M + 1, **i32)
-        slot_of = torch.empty((T, k), **i32)
-        row_token = torch.empty(T * k, **i32)
-        row_w = torch.empty(T * k, **f32)
-        pbuf, pws = self._ws(abi.moe_permute_workspace_size(T, k, M), dev)
-        abi.moe_permute(idx.data_ptr(), tw.data_ptr(), T, k, M, counts.data_ptr(), offsets.data_ptr(),
-                        slot_of.data_ptr(), row_token.data_ptr(), row_w.data_ptr(), pws, pbuf.numel() - 256, s)
-        x_perm = torch.empty((T * k, D), dtype=x.dtype, device=dev)
-        abi.moe_gather_rows(x.data_ptr(), row_token.data_ptr(), offsets[M:].data_ptr(), x_perm.data_ptr(), T * k,
-                            T, D, d.dtype, status.data_ptr(), s)
+                           idx.data_ptr(), tw.data_ptr(), ws, buf.numel() - 256, self._s)
+        return idx, tw
+
+    def _dispatch(self, idx, tw, M):
+        """The dispatch order of (idx, tw) over M experts (moe_permute)."""
+        T, k = idx.shape
+        i32 = dict(dtype=torch.int32, device=self.device)
+        p = {"counts": torch.empty(M, **i32), "offsets": torch.empty(M + 1, **i32),
+             "slot_of": torch.empty((T, k), **i32), "row_token": torch.empty(T * k, **i32),
+             "row_w": torch.empty(T * k, dtype=torch.float32, device=self.device)}
+        buf, ws = self._ws(abi.moe_permute_workspace_size(T, k, M), self.device)
+        abi.moe_permute(idx.data_ptr(), tw.data_ptr(), T, k, M, p["counts"].data_ptr(), p["offsets"].data_ptr(),
+                        p["slot_of"].data_ptr(), p["row_token"].data_ptr(), p["row_w"].data_ptr(), ws,
+                        buf.numel() - 256, self._s)
+        return p
+
+    def _gather(self, x, p):
+        """x's rows in dispatch order (moe_gather_rows)."""
+        T, D = x.shape
+        rows = p["row_token"].numel()
+        out = torch.empty((rows, D), dtype=x.dtype, device=self.device)
+        abi.moe_gather_rows(x.data_ptr(), p["row_token"].data_ptr(), p["offsets"][self.M:].data_ptr(),
+                            out.data_ptr(), rows, T, D, self._desc(T).dtype, self.status.data_ptr(), self._s)
+        return out
+
+    def _local_experts(self, x_recv, ids, w_recv):
+        """w * E_e(x) (fp32) of every received row, in arrival order: the rows
+        ordered by local expert (moe_permute, k = 1), the experts
+        (moe_expert_ffn), and back to arrival order (moe_combine, k = 1, fp32)."""
+        R, D = x_recv.shape
+        out_arr = torch.empty((R, D), dtype=torch.float32, device=self.device)
+        ids_d = torch.as_tensor(ids, device=self.device).view(R, 1)
+        p = self._dispatch(ids_d, w_recv.view(R, 1), self.E)
+        d_loc = self._desc(R, M=self.E, k=1)
+        out_perm = torch.empty((R, D), dtype=torch.float32, device=self.device)
+        buf, ws = self._ws(abi.moe_expert_ffn_workspace_size(d_loc), self.device)
+        abi.moe_expert_ffn(d_loc, self.w_local, x_recv.data_ptr(), p["offsets"].data_ptr(),
+                           p["row_token"].data_ptr(), p["row_w"].data_ptr(), out_perm.data_ptr(), ws,
+                           buf.numel() - 256, self._s)
+        # row r is the only slot of "token" r
+        abi.moe_combine(self._desc(R, M=self.E, k=1, dtype=abi.DTYPE_F32), out_perm.data_ptr(),
+                        p["slot_of"].data_ptr(), None, None, out_arr.data_ptr(), self._s)
+        return out_arr
+
+    def _shared(self, x):
+        """The shared expert's output in the layer dtype, or None."""
+        if not self.cfg.get("I_sh"):
+            return None
+        d = self._desc(x.shape[0])
+        y_sh = torch.empty_like(x)
+        buf, ws = self._ws(abi.moe_shared_expert_workspace_size(d), self.device)
+        abi.moe_shared_expert(d, self.w_shared, x.data_ptr(), y_sh.data_ptr(), ws, buf.numel() - 256, self._s)
+        return y_sh
+
+    def _combine(self, out_rows, slot_of, y_sh, x):
+        """y[t] = sum_j out_rows[slot_of[t, j]] (+ y_sh[t]) (moe_combine)."""
+        y = torch.empty_like(x)
+        abi.moe_combine(self._desc(x.shape[0]), out_rows.data_ptr(), slot_of.data_ptr(), _ptr(y_sh), None,
+                        y.data_ptr(), self._s)
+        return y
+
+    # ---- one forward ----
+
+    def forward(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+        T = x.shape[0]
+        k = self.cfg["k"]
+        self._s = _stream_handle(stream) if x.is_cuda else None
+        self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
+        # 1. route and dispatch this rank's tokens; its rows in dispatch order
+        idx, tw = self._route(x)
+        p = self._dispatch(idx, tw, self.M)
+        x_perm = self._gather(x, p)
         # 2. the exchange plan and the rows out
-        recv_counts = exchange_counts(counts, self.world, self.group)
-        plan = make_plan(counts.cpu().numpy(), recv_counts.cpu().numpy(), self.world)
+        recv_counts = exchange_counts(p["counts"], self.world, self.group)
+        plan = make_plan(p["counts"].cpu().numpy(), recv_counts.cpu().numpy(), self.world)
+        # the router never picks the sentinel, so all T k pairs go out and come back
+        assert plan.rows_sent == T * k
         x_recv = send_rows(x_perm, plan, self.group)
-        w_recv = send_rows(row_w, plan, self.group)
+        w_recv = send_rows(p["row_w"], plan, self.group)
         # 3. this rank's experts over the rows it received
-        R = plan.rows_received
-        out_arr = torch.empty((R, D), **f32)
-        if R > 0:
-            ids = torch.as_tensor(arrival_expert_ids(plan), device=dev).view(R, 1)
-            l_counts = torch.empty(self.E, **i32)
-            l_offsets = torch.empty(self.E + 1, **i32)
-            l_slot = torch.empty((R, 1), **i32)
-            l_token = torch.empty(R, **i32)
-            l_w = torch.empty(R, **f32)
-            lbuf, lws = self._ws(abi.moe_permute_workspace_size(R, 1, self.E), dev)
-            abi.moe_permute(ids.data_ptr(), w_recv.data_ptr(), R, 1, self.E, l_counts.data_ptr(),
-                            l_offsets.data_ptr(), l_slot.data_ptr(), l_token.data_ptr(), l_w.data_ptr(), lws,
-                            lbuf.numel() - 256, s)
-            d_loc = self._desc(R, M=self.E, k=1)
-            out_perm = torch.empty((R, D), **f32)
-            fbuf, fws = self._ws(abi.moe_expert_ffn_workspace_size(d_loc), dev)
-            abi.moe_expert_ffn(d_loc, self.w_local, x_recv.data_ptr(), l_offsets.data_ptr(), l_token.data_ptr(),
-                               l_w.data_ptr(), out_perm.data_ptr(), fws, fbuf.numel() - 256, s)
-            # back to arrival order: row r is the (only) slot of "token" r
-            abi.moe_combine(self._desc(R, M=self.E, k=1, dtype=abi.DTYPE_F32), out_perm.data_ptr(),
-                            l_slot.data_ptr(), None, None, out_arr.data_ptr(), s)
+        if plan.rows_received > 0:
+            out_arr = self._local_experts(x_recv, arrival_expert_ids(plan), w_recv)
+        else:
+            out_arr = torch.empty((0, x.shape[1]), dtype=self.out_dtype, device=self.device)
         # 4. results home, then this rank's combine with its shared expert
         out_back = return_rows(out_arr, plan, self.group)
-        y_sh = None
-        if cfg.get("I_sh"):
-            y_sh = torch.empty_like(x)
-            sbuf, sws = self._ws(abi.moe_shared_expert_workspace_size(d), dev)
-            abi.moe_shared_expert(d, self.w_shared, x.data_ptr(), y_sh.data_ptr(), sws, sbuf.numel() - 256, s)
-        # the router never picks the sentinel, so every one of the T k pairs went out and came back
-        assert plan.rows_sent == T * k
-        y = torch.empty_like(x)
-        abi.moe_combine(d, out_back.data_ptr(), slot_of.data_ptr(), _ptr(y_sh), None, y.data_ptr(), s)
+        y = self._combine(out_back, p["slot_of"], self._shared(x), x)
         self.last_plan = plan
-        self.status = status
         return y

@@ -1,13 +1,12 @@
-"""Expert parallelism's exchange on CPU gloo ranks: every rank routes its own
-tokens, sends each row to the owner of its expert with the plan of
-sparse_mixture_experts_logits_b200.ep, the owner computes its experts over
-the rows it received, the results come back, and each rank's combine must
-equal the oracle's single-process layer on that rank's tokens.
-
-The compute steps run here in the fp64 oracle (the library's kernels need a
-GPU); what is under test is the plan and the exchange: split sizes, the
-arrival order and the local expert of every received row, and the way back
-to each rank's dispatch order."""
+"""Expert parallelism on CPU gloo ranks: ExpertParallelMoE.forward (the
+product's orchestration, exchange plan and collectives) with each kernel step
+done by the fp64 oracle, since the library's kernels need a GPU.  Every rank
+routes its own tokens, sends each row to the owner of its expert, the owner
+runs its experts over the rows it received, the results come back, and each
+rank's output must equal the oracle's single-process layer on its tokens.
+What is under test is the plan and the exchange: split sizes, the arrival
+order and the local expert of every received row, and the way back to each
+rank's dispatch order."""
 import os
 import socket
 import sys
@@ -28,12 +27,6 @@ def _free_port():
     return port
 
 
-def _layer_inputs(cfg):
-    import moe_synth as ms
-    f64 = lambda t: None if t is None else t.double().numpy()  # noqa: E731
-    return {k: f64(v) for k, v in ms.layer_inputs(cfg).items()}
-
-
 def _forced_idx(T, k, M, world, rank):
     """A routing that leaves the experts of the last rank without rows and
     sends nothing from rank 0 to rank 1: every token picks k distinct experts
@@ -42,6 +35,65 @@ def _forced_idx(T, k, M, world, rank):
     allowed = list(range(E)) if rank == 0 else [e for e in range(M) if e // E not in (1, world - 1)]
     rng = np.random.default_rng(rank)
     return np.stack([rng.choice(allowed, size=k, replace=False) for _ in range(T)]).astype(np.int64)
+
+
+def _oracle_layer_class():
+    """ExpertParallelMoE with each kernel step done by the fp64 oracle on host
+    tensors; forward(), the exchange plan and the collectives are the
+    product's own."""
+    import oracle
+    from sparse_mixture_experts_logits_b200 import ep
+
+    class OracleEP(ep.ExpertParallelMoE):
+        forced = None
+        out_dtype = torch.float64
+
+        def _route(self, x):
+            c = self.cfg
+            xs, w_r = x.numpy(), self.t["w_r"].numpy()
+            if self.forced is not None:
+                idx = self.forced
+                logits = xs @ w_r
+                w = oracle.topk_weights(idx, logits, oracle.sigmoid(logits), c["gate"], c["norm_topk_prob"],
+                                        c["alpha"], c["eps"])
+            else:
+                bias = self.t.get("e_bias")
+                r = oracle.route(xs, w_r, None if bias is None else bias.numpy(), c["k"], c["gate"],
+                                 c["norm_topk_prob"], c["alpha"], c["eps"])
+                idx, w = r["idx"], r["w"]
+            return torch.as_tensor(idx, dtype=torch.int32), torch.as_tensor(w)
+
+        def _dispatch(self, idx, tw, M):
+            p = oracle.permute(idx.numpy(), tw.numpy(), M)
+            return {k: torch.as_tensor(v) for k, v in p.items()}
+
+        def _gather(self, x, p):
+            return x[p["row_token"]]
+
+        def _local_experts(self, x_recv, ids, w_recv):
+            out = torch.zeros(x_recv.shape, dtype=torch.float64)
+            for le in np.unique(ids):
+                sel = np.nonzero(ids == le)[0]
+                b1, b2 = self.t.get("b1"), self.t.get("b2")
+                e = oracle.expert_ffn(x_recv.numpy()[sel], self.cfg["act"], self.t["w1"][le].numpy(),
+                                      self.t["w2"][le].numpy(), None if b1 is None else b1[le].numpy(),
+                                      None if b2 is None else b2[le].numpy())
+                out[sel] = torch.as_tensor(w_recv.numpy()[sel, None] * e)
+            return out
+
+        def _shared(self, x):
+            if not self.cfg.get("I_sh"):
+                return None
+            sh = oracle.shared_expert(x.numpy(), self.t["sh_w1"].numpy(), self.t["sh_w2"].numpy())
+            return torch.as_tensor(sh)
+
+        def _combine(self, out_rows, slot_of, y_sh, x):
+            y = torch.zeros(x.shape, dtype=torch.float64)
+            for j in range(slot_of.shape[1]):
+                y += out_rows[slot_of[:, j].long()]
+            return y if y_sh is None else y + y_sh
+
+    return OracleEP
 
 
 def _worker(rank, world, port, name, T_total, forced, out_dir):
@@ -55,54 +107,21 @@ def _worker(rank, world, port, name, T_total, forced, out_dir):
         from sparse_mixture_experts_logits_b200 import ep
 
         cfg = ms.get_config(name, T=T_total)
-        inp = _layer_inputs(cfg)
-        M, k, D = cfg["M"], cfg["k"], cfg["D"]
-        E = ep.experts_per_rank(M, world)
+        full = {k: None if v is None else v.double() for k, v in ms.layer_inputs(cfg).items()}
         per = T_total // world
-        rows = slice(rank * per, (rank + 1) * per)
-        mine = dict(inp, x=inp["x"][rows])
-        local_cfg = dict(cfg, T=per)
-        # 1. this rank's routing and dispatch order
+        x = full["x"][rank * per:(rank + 1) * per].contiguous()
+        layer = _oracle_layer_class()(cfg, ep.local_expert_tensors(full, rank, world), rank, world)
         if forced:
-            idx = _forced_idx(per, k, M, world, rank)
-            w = oracle.topk_weights(idx, mine["x"] @ inp["w_r"], oracle.sigmoid(mine["x"] @ inp["w_r"]),
-                                    cfg["gate"], cfg["norm_topk_prob"], cfg["alpha"], cfg["eps"])
-        else:
-            r = oracle.route(mine["x"], inp["w_r"], inp.get("e_bias"), k, cfg["gate"], cfg["norm_topk_prob"],
-                             cfg["alpha"], cfg["eps"])
-            idx, w = r["idx"], r["w"]
-        p = oracle.permute(idx, w, M)
-        x_perm = torch.from_numpy(mine["x"][p["row_token"]])
-        # 2. the plan and the rows out
-        recv_counts = ep.exchange_counts(torch.as_tensor(p["counts"], dtype=torch.int32), world)
-        plan = ep.make_plan(p["counts"], recv_counts.numpy(), world)
-        assert plan.rows_sent == per * k
-        x_recv = ep.send_rows(x_perm, plan)
-        w_recv = ep.send_rows(torch.from_numpy(p["row_w"]), plan)
-        assert x_recv.shape == (plan.rows_received, D) and w_recv.shape == (plan.rows_received,)
-        # 3. this rank's experts (global ids rank*E + local) over the rows it received
-        ids = ep.arrival_expert_ids(plan)
-        out_arr = np.zeros((plan.rows_received, D))
-        for le in np.unique(ids):
-            sel = np.nonzero(ids == le)[0]
-            g = rank * E + int(le)
-            b1 = None if inp.get("b1") is None else inp["b1"][g]
-            b2 = None if inp.get("b2") is None else inp["b2"][g]
-            out = oracle.expert_ffn(x_recv.numpy()[sel], cfg["act"], inp["w1"][g], inp["w2"][g], b1, b2)
-            out_arr[sel] = w_recv.numpy()[sel, None] * out
-        # 4. results home, combine with the shared expert
-        out_back = ep.return_rows(torch.from_numpy(out_arr), plan).numpy()
-        y = np.zeros((per, D))
-        for j in range(k):
-            y += out_back[p["slot_of"][:, j]]
-        if cfg.get("I_sh"):
-            y += oracle.shared_expert(mine["x"], inp["sh_w1"], inp["sh_w2"])
-        ref = oracle.moe_forward(local_cfg, mine, idx=idx)["y"]
-        ok = np.allclose(y, ref, rtol=1e-12, atol=1e-12)
+            layer.forced = _forced_idx(per, cfg["k"], cfg["M"], world, rank)
+        y = layer.forward(x).numpy()
+        mine = {k: (None if v is None else v.numpy()) for k, v in full.items()}
+        mine["x"] = x.numpy()
+        ref = oracle.moe_forward(dict(cfg, T=per), mine, idx=layer.forced)["y"]
+        plan = layer.last_plan
         total_recv = torch.tensor([plan.rows_received])
         dist.all_reduce(total_recv)
-        torch.save({"ok": bool(ok), "err": float(np.abs(y - ref).max()), "recv": plan.rows_received,
-                    "send": plan.send_splits, "total_recv": int(total_recv)},
+        torch.save({"ok": bool(np.allclose(y, ref, rtol=1e-12, atol=1e-12)), "err": float(np.abs(y - ref).max()),
+                    "recv": plan.rows_received, "send": plan.send_splits, "total_recv": int(total_recv)},
                    os.path.join(out_dir, f"rank{rank}.pt"))
     finally:
         dist.destroy_process_group()

@@ -232,3 +232,37 @@ def test_capacity_host_checks(B):
             B.moe_capacity_drop(*args)
         assert e.value.status == status
     B.moe_capacity_drop(None, None, None, 0, 2, 8, 4)   # T = 0: nothing to do
+
+
+def _header_signatures():
+    """name -> list of parameter declarations, from include/moe_b200.h."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    sigs = {}
+    for m in re.finditer(r"\b(moe_[a-z_0-9]+)\s*\(([^;{]*?)\)\s*;", src, flags=re.S):
+        params = " ".join(m.group(2).split())
+        sigs[m.group(1)] = [] if params in ("", "void") else [p.strip() for p in params.split(",")]
+    return sigs
+
+
+def test_binding_arity_and_kinds_match_the_header(B):
+    """ctypes does not check a call against the C declaration: every
+    binding's argtypes must have the header's parameter count, with pointers
+    where the header has pointers and numbers where it has numbers."""
+    import ctypes
+    sigs = _header_signatures()
+    assert set(sigs) == set(B.EXPORTED_SYMBOLS)
+    lib = B.lib
+    for name, params in sigs.items():
+        argtypes = getattr(lib, name).argtypes
+        assert argtypes is not None, name
+        assert len(argtypes) == len(params), (name, len(argtypes), params)
+        for p, a in zip(params, argtypes):
+            is_ptr = "*" in p
+            ptr_like = a is ctypes.c_void_p or a is ctypes.c_char_p or hasattr(a, "_type_") and \
+                isinstance(a, type(ctypes.POINTER(ctypes.c_int)))
+            assert is_ptr == bool(ptr_like), (name, p, a)
+            if not is_ptr:
+                ctype = p.split()[0]
+                expect = {"int": ctypes.c_int, "float": ctypes.c_float, "double": ctypes.c_double,
+                          "size_t": ctypes.c_size_t, "moe_status_t": ctypes.c_int}[ctype]
+                assert a is expect, (name, p, a)

@@ -266,3 +266,38 @@ def test_binding_arity_and_kinds_match_the_header(B):
                 expect = {"int": ctypes.c_int, "float": ctypes.c_float, "double": ctypes.c_double,
                           "size_t": ctypes.c_size_t, "moe_status_t": ctypes.c_int}[ctype]
                 assert a is expect, (name, p, a)
+
+
+def test_struct_fields_match_the_header(B):
+    """Every ctypes struct lists the header struct's fields, in order, with
+    the header's types (int, float, size_t, pointer)."""
+    import ctypes
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    structs = {}
+    for m in re.finditer(r"typedef struct \{(.*?)\}\s*(moe_[a-z_]+_t)\s*;", src, flags=re.S):
+        fields = []
+        for decl in m.group(1).split(";"):
+            decl = " ".join(decl.split())
+            if not decl:
+                continue
+            for name in decl.split(",") if "*" not in decl else [decl]:
+                fields.append(name)
+        structs[m.group(2)] = fields
+    pairs = {"moe_layer_desc_t": B.LayerDesc, "moe_weights_t": B.Weights, "moe_ws_layout_t": B.WsLayout,
+             "moe_dense_desc_t": B.DenseDesc, "moe_grads_t": B.Grads}
+    assert set(pairs) == set(structs)
+    for cname, cls in pairs.items():
+        expanded = []
+        for decl in structs[cname]:
+            parts = decl.replace("*", " * ").split()
+            if "*" in parts:
+                expanded.append((parts[-1], "ptr"))
+            else:
+                ctype = parts[0]
+                for i, tok in enumerate(parts[1:]):
+                    expanded.append((tok.strip(), ctype))
+        names = [f[0] for f in cls._fields_]
+        assert names == [n for n, _ in expanded], (cname, names, expanded)
+        kinds = {"int": ctypes.c_int, "float": ctypes.c_float, "size_t": ctypes.c_size_t, "ptr": ctypes.c_void_p}
+        for (n, t), (fname, ftype) in zip(expanded, cls._fields_):
+            assert ftype is kinds[t], (cname, n, t, ftype)

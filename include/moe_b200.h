@@ -69,7 +69,7 @@ typedef enum { MOE_ACT_GELU_TANH = 0, MOE_ACT_SWIGLU = 1 } moe_act_t;
 
 /* Device-side error codes written to the workspace flag. */
 #define MOE_DEVERR_NONE 0
-#define MOE_DEVERR_BAD_EXPERT_INDEX 1 /* topk_idx entry outside [0, M) */
+#define MOE_DEVERR_BAD_EXPERT_INDEX 1 /* topk_idx entry outside [0, M] (M: the sentinel) */
 #define MOE_DEVERR_TIMEOUT 2          /* a bounded wait inside a kernel gave up */
 #define MOE_DEVERR_BAD_ROW_TOKEN 3    /* row_token entry outside [0, T) (row zero-filled) */
 

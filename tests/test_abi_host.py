@@ -301,3 +301,16 @@ def test_struct_fields_match_the_header(B):
         kinds = {"int": ctypes.c_int, "float": ctypes.c_float, "size_t": ctypes.c_size_t, "ptr": ctypes.c_void_p}
         for (n, t), (fname, ftype) in zip(expanded, cls._fields_):
             assert ftype is kinds[t], (cname, n, t, ftype)
+
+
+def test_constants_match_the_header(B):
+    """Status codes, enum values, device error codes and event counts of the
+    binding equal the header's."""
+    from sparse_mixture_experts_logits_b200 import abi
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    values = {m.group(1): int(m.group(2)) for m in re.finditer(r"\b(MOE_[A-Z_0-9]+)\s*=\s*(\d+)", src)}
+    values.update({m.group(1): int(m.group(2)) for m in re.finditer(r"#define (MOE_[A-Z_0-9]+) (\d+)", src)})
+    assert len(values) >= 17
+    for name, v in values.items():
+        attr = name if name.startswith(("MOE_OK", "MOE_ERR_")) else name[len("MOE_"):]
+        assert getattr(abi, attr) == v, (name, v)

@@ -192,11 +192,13 @@ moe_status_t moe_permute(const int32_t* topk_idx, const float* topk_w, int T, in
  *   M * ceil(T*k / 512) <= 524288; larger requests return
  *   MOE_ERR_UNSUPPORTED without launching.  No cudaMalloc/cudaFree.
  *   device_status: optional int32 device word, cleared by the call, set to
- *   MOE_DEVERR_BAD_EXPERT_INDEX if topk_idx holds an index outside [0, M).
+ *   MOE_DEVERR_BAD_EXPERT_INDEX if topk_idx holds an index outside [0, M]
+ *   (M itself is the sentinel, dispatched nowhere).
  *   All calls on a device share the scratch array; calls whose kernels
  *   overlap on the GPU (unordered streams) race and may give wrong results.
- *   The first call on each device looks up the array's address with that
- *   device current; make it before any stream capture begins.
+ *   The first call on each device (and again after the device's context is
+ *   recreated, e.g. by cudaDeviceReset) looks up the array's address with
+ *   that device current; make it before any stream capture begins.
  * Other arguments and outputs: as moe_permute (bit-identical results). */
 moe_status_t moe_permute_static_scratch(const int32_t* topk_idx, const float* topk_w, int T, int k,
                                         int M, int32_t* counts, int32_t* offsets, int32_t* slot_of,
@@ -406,6 +408,23 @@ moe_status_t moe_backward(const moe_layer_desc_t* d, const moe_weights_t* w, con
 
 /* Number of kernels one moe_backward call with this descriptor launches. */
 int moe_backward_launch_count(const moe_layer_desc_t* d);
+
+/* ---- diagnostics (no counterpart on the source pages) ------------------- */
+
+/* Self-test of the bounded waits that every pipelined kernel of this library
+ * uses instead of unbounded spins.  One kernel of 64 threads waits on two
+ * shared-memory barriers that nothing ever arrives on: warp 0 with a limit
+ * of limit_ns, warp 1 with 4 x limit_ns.  Warp 0 gives up when its limit
+ * passes, records MOE_DEVERR_TIMEOUT in *device_status and raises the
+ * kernel's abort flag; warp 1 must then leave on that flag (as the other
+ * roles of a GEMM do), well before its own limit.  No fault, no hang: the
+ * context stays usable.
+ *   device_status: device int32, cleared by the call, MOE_DEVERR_TIMEOUT
+ *   afterwards.  elapsed_ns: NULL or device uint64 [2]: the nanoseconds
+ *   each warp waited, bit 63 set if its wait succeeded (it never should).
+ *   1000 <= limit_ns <= 2e9, else MOE_ERR_INVALID_ARG. */
+moe_status_t moe_selftest_wait_timeout(uint64_t limit_ns, int32_t* device_status,
+                                       uint64_t* elapsed_ns, void* stream);
 
 #ifdef __cplusplus
 }

@@ -353,13 +353,16 @@ def moe_tokens(x_rows, idx_rows, w_rows, act, get_expert, shared=None, sentinel=
     return y
 
 
-def moe_forward(cfg, inp, idx=None, addend=None):
+def moe_forward(cfg, inp, idx=None, addend=None, w=None):
     """Whole layer: route, dispatch order, experts, combine, shared add.
 
     ``cfg`` holds T, D, M, k, gate, act, norm_topk_prob, alpha, eps, I_sh;
     ``inp`` holds numpy arrays x, w_r, e_bias, w1, b1, w2, b2, sh_w1, sh_w2
     (w1/w2/b1/b2 indexable by expert).  ``idx`` overrides the selection
-    (used when the oracle adopts the GPU's choice at a near-tie).  With
+    (used when the oracle adopts the GPU's choice at a near-tie); it may hold
+    the sentinel M ("no expert", [GLM5-SE] one_hot over M + 1 classes), whose
+    pairs add nothing.  ``w`` overrides the gate weights and must be given
+    when ``idx`` holds the sentinel (a sentinel has no router score).  With
     ``addend`` the output is the sparse block sum of the "GLaM" note, section
     "Interleaving Dense and Sparse Layers": addend + MoE-FFN(x), addend
     standing for Attention(h)."""
@@ -368,8 +371,15 @@ def moe_forward(cfg, inp, idx=None, addend=None):
               cfg.get("topk_group", 1))
     if idx is not None:
         r["idx"] = np.asarray(idx, dtype=np.int64)
-        r["w"] = topk_weights(r["idx"], r["logits"], r["g"], cfg["gate"],
-                              cfg["norm_topk_prob"], cfg["alpha"], cfg["eps"])
+        if w is not None:
+            r["w"] = _f64(w)
+        elif (r["idx"] == cfg["M"]).any():
+            raise ValueError("an index holding the sentinel M needs its gate weights passed as w")
+        else:
+            r["w"] = topk_weights(r["idx"], r["logits"], r["g"], cfg["gate"],
+                                  cfg["norm_topk_prob"], cfg["alpha"], cfg["eps"])
+    elif w is not None:
+        r["w"] = _f64(w)
     p = permute(r["idx"], r["w"], cfg["M"])
 
     def get_expert(e):
@@ -381,7 +391,7 @@ def moe_forward(cfg, inp, idx=None, addend=None):
     shared = None
     if cfg.get("I_sh"):
         shared = (inp["sh_w1"], inp["sh_w2"])
-    y = moe_tokens(inp["x"], r["idx"], r["w"], cfg["act"], get_expert, shared)
+    y = moe_tokens(inp["x"], r["idx"], r["w"], cfg["act"], get_expert, shared, sentinel=cfg["M"])
     if addend is not None:
         y = _f64(addend) + y
     out = dict(r)

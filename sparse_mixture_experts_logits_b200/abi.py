@@ -28,7 +28,7 @@ EXPORTED_SYMBOLS = [
     "moe_forward_profiled", "moe_forward_launch_count", "moe_algorithmic_work",
     "moe_forward_add", "moe_dense_ffn_workspace_size", "moe_dense_ffn", "moe_dense_ffn_profiled",
     "moe_backward_workspace_size", "moe_backward", "moe_backward_launch_count", "moe_gather_rows",
-    "moe_capacity_drop", "moe_expert_capacity",
+    "moe_capacity_drop", "moe_expert_capacity", "moe_selftest_wait_timeout",
 ]
 NUM_STAGE_EVENTS = 9
 NUM_DENSE_EVENTS = 3
@@ -121,6 +121,7 @@ _decl("moe_dense_ffn_profiled", _i, [_P(DenseDesc), _vp, _vp, _vp, _vp, _vp, _vp
 _decl("moe_gather_rows", _i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp])
 _decl("moe_capacity_drop", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp])
 _decl("moe_expert_capacity", _i, [ctypes.c_double, _i, _i, _i])
+_decl("moe_selftest_wait_timeout", _i, [ctypes.c_uint64, _vp, _vp, _vp])
 _decl("moe_backward_workspace_size", _sz, [_P(LayerDesc)])
 _decl("moe_backward", _i, [_P(LayerDesc), _P(Weights), _vp, _vp, _P(Grads), _vp, _sz, _vp])
 _decl("moe_backward_launch_count", _i, [_P(LayerDesc)])
@@ -284,3 +285,8 @@ def moe_capacity_drop(topk_idx, slot_of, offsets, T, k, M, capacity, stream=None
 
 def moe_expert_capacity(factor, T, k, M) -> int:
     return lib.moe_expert_capacity(float(factor), T, k, M)
+
+
+def moe_selftest_wait_timeout(limit_ns, device_status, elapsed_ns=None, stream=None):
+    _check("moe_selftest_wait_timeout",
+           lib.moe_selftest_wait_timeout(int(limit_ns), device_status, elapsed_ns, stream))

@@ -98,17 +98,18 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase of parity `parity` of mbarrier `bar` to complete.
-// Gives up (returns false) when *abort becomes non-zero or after
-// kWaitTimeoutNs, in which case it records the timeout and raises *abort.
+// Gives up (returns false) when *abort becomes non-zero or after limit_ns
+// (kWaitTimeoutNs unless given), in which case it records the timeout and
+// raises *abort.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          int* status) {
+                                          int* status, uint64_t limit_ns = kWaitTimeoutNs) {
   if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((n & 31u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort = 1;
         set_status(status, MOE_DEVERR_TIMEOUT);
         return false;
@@ -121,8 +122,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // outcome (false when any lane saw the abort flag or the time limit).  Keeps
 // the caller's loop control warp-uniform.
 __device__ __forceinline__ bool mbar_wait_all(uint32_t bar, uint32_t parity, volatile int* abort,
-                                              int* status) {
-  const bool ok = mbar_wait(bar, parity, abort, status);
+                                              int* status, uint64_t limit_ns = kWaitTimeoutNs) {
+  const bool ok = mbar_wait(bar, parity, abort, status, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 

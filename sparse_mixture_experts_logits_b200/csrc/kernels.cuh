@@ -66,6 +66,9 @@ struct GemmLaunch {
 };
 cudaError_t launch_gemm_sm100(const GemmLaunch& L, cudaStream_t s);
 int num_sms();
+// MOE_OK when the current device is compute capability 10.0 (the only
+// target of this library's sm_100a code), MOE_ERR_UNSUPPORTED otherwise.
+moe_status_t check_device();
 
 // gemm_swap_sm100.cu: grouped bf16 GEMM with the token rows on the MMA's N
 // side (see gemm_swap_sm100.cuh).  `epi` is a GemmEpilogue.

@@ -12,22 +12,7 @@
 
 using namespace moe;
 
-namespace {
-
-constexpr size_t kAlign = 256;
-inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
-inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
-
-struct Carve {
-  size_t off = 0;
-  size_t take(size_t bytes) {
-    const size_t o = off;
-    off += align_up(bytes);
-    return o;
-  }
-};
-
-inline size_t esize(int dtype) { return dtype == MOE_DTYPE_BF16 ? 2 : 4; }
+namespace moe {
 
 // Every entry point runs only on compute capability 10.0 (sm_100a code).
 moe_status_t check_device() {
@@ -46,6 +31,25 @@ moe_status_t check_device() {
   }
   return v == 1 ? MOE_OK : MOE_ERR_UNSUPPORTED;
 }
+
+}  // namespace moe
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
+
+struct Carve {
+  size_t off = 0;
+  size_t take(size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes);
+    return o;
+  }
+};
+
+inline size_t esize(int dtype) { return dtype == MOE_DTYPE_BF16 ? 2 : 4; }
 
 inline moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 #define MOE_TRY(expr)                          \

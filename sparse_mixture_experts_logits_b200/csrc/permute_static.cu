@@ -26,8 +26,10 @@
 //     whose kernels overlap on the GPU (different streams without ordering
 //     between them) race on the array and may produce wrong results.
 //   * The first call on each device looks up the array's device address
-//     (cudaGetSymbolAddress) with that device current.  Make that first call
-//     before any stream capture begins.
+//     (cudaGetSymbolAddress) with that device current, and records it with
+//     the device's current context.  A later call in a different context
+//     (after cudaDeviceReset, for instance) looks it up again.  Make the
+//     first call on a device before any stream capture begins.
 #include <atomic>
 #include <mutex>
 
@@ -43,19 +45,48 @@ static __device__ __align__(256) int32_t g_perm_scratch[2 * kStaticPermScratchIn
 constexpr int kMaxDevices = 64;
 std::mutex g_addr_mutex;
 int32_t* g_addr[kMaxDevices] = {nullptr};
+CUcontext g_ctx[kMaxDevices] = {nullptr};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+// cuCtxGetCurrent through the runtime's driver entry-point table (the
+// library links no driver library directly).
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+CUcontext current_context() {
+  CUcontext c = nullptr;
+  const CtxGetCurrentFn fn = ctx_get_current();
+  if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
 
 // Device address of g_perm_scratch on the current device.  The host-side
 // symbol `g_perm_scratch` is only a stand-in, not a device address, so the
-// kernels get this pointer instead.
+// kernels get this pointer instead.  It is looked up once per device and
+// context: a context created anew (the module loaded again) may place the
+// array elsewhere.
 moe_status_t scratch_address(int32_t** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_addr_mutex);
-  if (g_addr[dev] == nullptr) {
+  CUcontext ctx = current_context();
+  if (g_addr[dev] == nullptr || ctx == nullptr || ctx != g_ctx[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_perm_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
     g_addr[dev] = static_cast<int32_t*>(p);
+    g_ctx[dev] = current_context();  // the lookup makes the device's context current
   }
   *out = g_addr[dev];
   return MOE_OK;
@@ -76,14 +107,10 @@ extern "C" moe_status_t moe_permute_static_scratch(const int32_t* topk_idx, cons
     return MOE_ERR_UNSUPPORTED;
   if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
   if (T > 0 && (!topk_idx || !topk_w || !slot_of || !row_token || !row_w)) return MOE_ERR_INVALID_ARG;
-  int major = 0, minor = 0, dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  if (major != 10 || minor != 0) return MOE_ERR_UNSUPPORTED;
+  moe_status_t st = check_device();
+  if (st != MOE_OK) return st;
   int32_t* scratch = nullptr;
-  moe_status_t st = scratch_address(&scratch);
+  st = scratch_address(&scratch);
   if (st != MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (device_status != nullptr && cudaMemsetAsync(device_status, 0, sizeof(int32_t), s) != cudaSuccess)

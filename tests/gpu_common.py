@@ -160,5 +160,36 @@ def sample_tokens(cfg, counts, row_token, offsets, n_random=6, seed=0):
     return np.array(sorted(t for t in toks if 0 <= t < T), dtype=np.int64)
 
 
+def swap_token_tiles(cnt, max_width=256):
+    """Token tiles of one expert segment of ``cnt`` rows as the library's
+    tokens-on-N expert GEMM cuts it: the fewest tiles of at most 256 rows,
+    all of one width rounded up to a multiple of 16, the last one ragged.
+    Returns (first row, rows) of each tile, relative to the segment."""
+    if cnt <= 0:
+        return []
+    n0 = -(-cnt // max_width)
+    width = (-(-cnt // n0) + 15) // 16 * 16
+    return [(r0, min(width, cnt - r0)) for r0 in range(0, cnt, width)]
+
+
+def tile_tokens(cfg, counts, row_token, offsets, seed=0):
+    """Tokens whose outputs together exercise every token tile of the
+    full-size expert GEMMs: for each expert segment and each of its token
+    tiles, the tokens of the tile's first row, last row and one row between;
+    for the shared expert (one segment of all T tokens) the first and last
+    token of each 256-token tile; plus the extremes of sample_tokens."""
+    rng = np.random.default_rng(seed)
+    toks = set(sample_tokens(cfg, counts, row_token, offsets).tolist())
+    for e in range(len(counts)):
+        base = int(offsets[e])
+        for r0, n in swap_token_tiles(int(counts[e])):
+            for r in {r0, r0 + n - 1, r0 + int(rng.integers(0, n))}:
+                toks.add(int(row_token[base + r]))
+    if cfg.get("I_sh"):
+        for r0, n in swap_token_tiles(cfg["T"]):
+            toks.update((r0, r0 + n - 1))
+    return np.array(sorted(toks), dtype=np.int64)
+
+
 def gpu_inputs(cfg):
     return ms.layer_inputs(cfg, "cuda")

@@ -224,6 +224,43 @@ def pin_sentinel(O):
     assert np.allclose(y_s, y_0, rtol=1e-13, atol=1e-13)
 
 
+def pin_forward_sentinel(O):
+    """The whole-layer oracle given a selection that holds the sentinel M:
+    each token's output is, by a per-pair loop over its kept pairs only,
+    sum_j w[t, j] E_idx[t, j](x_t) plus the shared expert; a token whose
+    pairs are all sentinels gets the shared expert alone."""
+    cfg = dict(TINY[2])
+    inp = tiny_inputs(cfg, 71)
+    r = O.route(inp["x"], inp["w_r"], inp["e_bias"], cfg["k"], cfg["gate"], 1, cfg["alpha"], cfg["eps"])
+    M = cfg["M"]
+    idx = r["idx"].copy()
+    idx[1::3, 0] = M
+    idx[4, :] = M
+    out = O.moe_forward(cfg, inp, idx=idx, w=r["w"])
+    assert out["offsets"][M] == (idx < M).sum()
+    for t in range(cfg["T"]):
+        ref = np.zeros(cfg["D"])
+        for j in range(cfg["k"]):
+            e = idx[t, j]
+            if e == M:
+                continue
+            h = inp["w1"][e] @ inp["x"][t]
+            I = h.shape[0] // 2
+            a = (h[:I] / (1.0 + np.exp(-h[:I]))) * h[I:]
+            ref += r["w"][t, j] * (inp["w2"][e] @ a)
+        if cfg.get("I_sh"):
+            hs = inp["sh_w1"] @ inp["x"][t]
+            Is = hs.shape[0] // 2
+            ref += inp["sh_w2"] @ ((hs[:Is] / (1.0 + np.exp(-hs[:Is]))) * hs[Is:])
+        assert np.allclose(out["y"][t], ref, rtol=1e-12, atol=1e-12), t
+    try:
+        O.moe_forward(cfg, inp, idx=idx)
+    except ValueError:
+        pass
+    else:
+        raise AssertionError("a sentinel selection without weights must be refused")
+
+
 def pin_permute(O):
     rng = np.random.default_rng(5)
     for T, k, M in [(37, 3, 7), (64, 8, 16), (1, 1, 1), (5, 4, 64)]:
@@ -504,7 +541,7 @@ def pin_capacity_drop(O):
 
 ALL_PINS = [
     pin_gelu, pin_silu_sigmoid, pin_topk_bruteforce, pin_softmax_top2_closed_form,
-    pin_sigmoid_router, pin_bias_selects_only, pin_group_limit, pin_permute, pin_sentinel, pin_bruteforce_forward,
+    pin_sigmoid_router, pin_bias_selects_only, pin_group_limit, pin_permute, pin_sentinel, pin_forward_sentinel, pin_bruteforce_forward,
     pin_single_expert_is_dense_ffn, pin_k_equals_m, pin_shared_branch,
     pin_sum_no_residual, pin_dense_layer, pin_param_counts, pin_error_metrics, pin_adopt_topk,
     pin_capacity_drop,

@@ -264,7 +264,8 @@ def test_binding_arity_and_kinds_match_the_header(B):
             if not is_ptr:
                 ctype = p.split()[0]
                 expect = {"int": ctypes.c_int, "float": ctypes.c_float, "double": ctypes.c_double,
-                          "size_t": ctypes.c_size_t, "moe_status_t": ctypes.c_int}[ctype]
+                          "size_t": ctypes.c_size_t, "moe_status_t": ctypes.c_int,
+                          "uint64_t": ctypes.c_uint64}[ctype]
                 assert a is expect, (name, p, a)
 
 

@@ -7,7 +7,7 @@ import torch
 import moe_synth as ms
 import oracle
 from gpu_common import (check_permutation, check_routing, check_y, gpu_inputs, np64, oracle_route,
-                        oracle_y, sample_tokens)
+                        oracle_y, sample_tokens, tile_tokens)
 
 pytestmark = pytest.mark.gpu
 
@@ -33,13 +33,18 @@ def run_forward(B, cfg, inp):
 
 
 def check_layer(B, cfg, all_tokens=True):
+    """all_tokens: True compares y on every token; "tiles" on the tokens of
+    the first, last and one middle row of every token tile of the expert and
+    shared GEMMs (so every tile is compared at full K); False on a sample."""
     inp = gpu_inputs(cfg)
     layer, y, v = run_forward(B, cfg, inp)
     r = oracle_route(cfg, inp)
     w_ref, ndiff = check_routing(cfg, r, v["topk_idx"], v["topk_w"])
     p = check_permutation(cfg, v["topk_idx"], v["topk_w"], v)
-    if all_tokens:
+    if all_tokens is True:
         tokens = np.arange(cfg["T"])
+    elif all_tokens == "tiles":
+        tokens = tile_tokens(cfg, p["counts"], p["row_token"], p["offsets"])
     else:
         tokens = sample_tokens(cfg, p["counts"], p["row_token"], p["offsets"])
     y_ref = oracle_y(cfg, inp, tokens, v["topk_idx"], w_ref)
@@ -52,17 +57,26 @@ def test_small_layer_all_tokens(B, name):
     check_layer(B, ms.get_config(name), all_tokens=True)
 
 
+# GLaM prefill and decode: y on every token; the GLM prefill layers: y on
+# the tokens of every token tile of every expert segment (first, last and a
+# middle row), which covers each tile of both expert GEMMs at full K.
+FULL_TOKENS = {"glam_prefill_bf16": True, "glm45_decode_bf16": True, "glm45_prefill_bf16": "tiles",
+               "glm5_skewed_prefill_bf16": "tiles"}
+
+
 @pytest.mark.parametrize("name", FULL)
-def test_full_size_layer_sampled(B, name):
+def test_full_size_layer(B, name):
     """Full-size workloads in the benchmark's launch configuration: routing
-    and dispatch checked on every token, y on a sample of tokens."""
-    check_layer(B, ms.get_config(name), all_tokens=False)
+    and dispatch checked on every token, y on every token or on every token
+    tile of the expert GEMMs, at the literal bound."""
+    _, _, _, _, m, _ = check_layer(B, ms.get_config(name), all_tokens=FULL_TOKENS[name])
+    print(name, m)
 
 
-def test_group_limited_full_size_sampled(B):
+def test_group_limited_full_size(B):
     """The GLM-5 skewed prefill layer with the router limited to the 4 best
-    of 8 expert groups (32 experts each)."""
-    check_layer(B, ms.get_config("glm5_skewed_prefill_bf16", n_group=8, topk_group=4), all_tokens=False)
+    of 8 expert groups (32 experts each), y on every token tile."""
+    check_layer(B, ms.get_config("glm5_skewed_prefill_bf16", n_group=8, topk_group=4), all_tokens="tiles")
 
 
 @pytest.mark.parametrize("name,over", [

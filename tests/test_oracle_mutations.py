@@ -147,7 +147,7 @@ def m_dense_drops_addend(O):
 
 def m_block_drops_addend(O):
     orig = O.moe_forward
-    O.moe_forward = lambda cfg, inp, idx=None, addend=None: orig(cfg, inp, idx)
+    O.moe_forward = lambda cfg, inp, idx=None, addend=None, w=None: orig(cfg, inp, idx, w=w)
 
 
 def m_dense_no_b2(O):

@@ -5,7 +5,7 @@ them no allocator).  It keeps its scratch in an array compiled into the
 library, so it must give exactly what moe_permute gives with a workspace,
 and a second call must not be disturbed by what the first left behind.
 
-This file is collected last on purpose (test_zz_*), so that a run stopping
+This file is collected last on purpose (test_zzzz_*), so that a run stopping
 at the first failure has already run every other test."""
 import numpy as np
 import pytest
@@ -61,6 +61,19 @@ def test_static_scratch_permute_matches_workspace_permute_twice():
         for a, b in zip(ref, got):
             assert torch.equal(a.view(torch.int32), b.view(torch.int32))
         assert int(got[1][-1]) == idx.numel()
+
+    # the call itself takes no device memory: free memory is unchanged across
+    # a further call (the outputs are allocated before the first reading)
+    outs = [torch.empty(n, dtype=dt, device=dev) for n, dt in
+            [(M, torch.int32), (M + 1, torch.int32), (T * k, torch.int32), (T * k, torch.int32),
+             (T * k, torch.float32)]]
+    s = torch.cuda.current_stream().cuda_stream
+    torch.cuda.synchronize()
+    free_before, _ = torch.cuda.mem_get_info()
+    B.moe_permute_static_scratch(idx1.data_ptr(), w1.data_ptr(), T, k, M, *[o.data_ptr() for o in outs], None, s)
+    torch.cuda.synchronize()
+    free_after, _ = torch.cuda.mem_get_info()
+    assert free_after == free_before
 
 
 def test_static_scratch_limits_and_errors():

@@ -865,20 +865,24 @@ def run_backward(args):
     achieved = flops / (ms_step / 1e3) / 1e12
     # the CUDA-core fp32 FMA rate: 148 SMs x 128 lanes x 2 FLOP at the 1965 MHz clock ceiling
     simt_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+    tc = cfg["dtype"] == "bf16"
     out = {
         "metric": "MoE layer backward throughput (all gradients; routing and expert forward recomputed)",
         "value": world * T / (ms_step / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32",
+        "vs_baseline": None, "dtype": "bf16" if tc else "f32",
         "data": "synthetic (seeded counter-based generator; random-init weights)",
         "config": {"workload": args.config, "T_per_gpu": T, "D": D, "M": cfg["M"], "k": cfg["k"],
                    "I": cfg["I"], "I_sh": cfg.get("I_sh", 0), "inputs": cfg["dtype"],
-                   "arithmetic": "fp32 on the CUDA cores (inputs widened from the layer dtype)",
+                   "arithmetic": ("bf16 operands on tcgen05, fp32 accumulation (moe_gemm_swap_kernel: forward, "
+                                  "input-gradient and grouped-K weight-gradient layouts)") if tc else
+                   "fp32 on the CUDA cores",
                    "l2": "flushed between steps (256 MiB write outside the timed events)",
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": achieved / peak_tf, "traffic": None,
-                     "kernel": "the whole step (bwd_gemm_kernel launches hold most of it; see the launch list)",
+                     "kernel": ("the whole step (moe_gemm_swap_kernel launches hold most of it; see the launch list)"
+                                if tc else "the whole step (bwd_gemm_kernel launches hold most of it)"),
                      "peak_source": f"{peak_src}: bf16_tflops (burst)",
                      "algorithmic": {"flops": flops, "note": "2 x forward FLOPs; the recompute is not counted"},
                      "frac_of_fp32_simt_peak": achieved / simt_peak},

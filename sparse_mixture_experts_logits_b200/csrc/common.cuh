@@ -293,6 +293,23 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory matrix descriptor of an MN-major bf16 tile with the 128-byte
+// swizzle (the layout a TMA load with CU_TENSOR_MAP_SWIZZLE_128B writes for
+// a box of 64 MN-consecutive elements by K rows): each K row is 128 bytes
+// holding 64 MN-consecutive elements, groups of 8 K rows are 1024 bytes
+// apart (stride offset), and the next 64 MN elements start `mn_group_bytes`
+// later (leading offset).  A K = 16 slice spans 16 rows, i.e. 2048 bytes.
+// The tile must start 1024-byte aligned.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t saddr, uint32_t mn_group_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);                  // start address (16 B units)
+  d |= static_cast<uint64_t>((mn_group_bytes >> 4) & 0x3FFFu) << 16;    // leading offset: next 64 MN
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;                          // stride offset: next 8 K rows
+  d |= static_cast<uint64_t>(1) << 46;                                  // descriptor version
+  d |= static_cast<uint64_t>(2) << 61;                                  // 128-byte swizzle
+  return d;
+}
+
 // Instruction descriptor: bf16 A and B (K-major), fp32 accumulator, M x N.
 __host__ __device__ constexpr uint32_t umma_idesc_bf16(int m, int n) {
   return (1u << 4)                                 // D format: f32
@@ -300,6 +317,12 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int m, int n) {
          | (1u << 10)                              // B format: bf16
          | (static_cast<uint32_t>(n >> 3) << 17)   // N / 8
          | (static_cast<uint32_t>(m >> 4) << 24);  // M / 16
+}
+// Same with the major-ness of each operand: a_mn / b_mn = 1 for an MN-major
+// (transposed) operand in shared memory.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16_major(int m, int n, int a_mn, int b_mn) {
+  return umma_idesc_bf16(m, n) | (static_cast<uint32_t>(a_mn & 1) << 15) |
+         (static_cast<uint32_t>(b_mn & 1) << 16);
 }
 
 #define MOE_TMEM_LD32(taddr, r)                                                                   \

@@ -25,12 +25,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// bf16 [rows, K] row-major, box = box_rows x 64, 128-byte swizzle; rows past the end read as zero.
-bool tmap_bf16(CUtensorMap* map, const void* base, long long rows, int K, int box_rows) {
+// bf16 [rows, cols] row-major, box = box_rows x 64 columns, 128-byte swizzle;
+// rows and columns past the end read as zero.
+bool tmap_bf16(CUtensorMap* map, const void* base, long long rows, int cols, int box_rows) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
@@ -38,14 +39,14 @@ bool tmap_bf16(CUtensorMap* map, const void* base, long long rows, int K, int bo
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EPI>
+template <int EPI, int LAYOUT = kSwFwd>
 cudaError_t launch_swap_epi(const CUtensorMap& tw, const CUtensorMap& tx, const SwapArgs& args,
                             long long tiles_ub, cudaStream_t s) {
   static std::atomic<unsigned> configured{0};
   static std::atomic<int> max_clusters[32];
   int dev = 0;
   cudaGetDevice(&dev);
-  auto kernel = moe_gemm_swap_kernel<EPI>;
+  auto kernel = moe_gemm_swap_kernel<EPI, LAYOUT>;
   const unsigned bit = 1u << (dev & 31);
   if (!(configured.load() & bit)) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSwDynSmem);
@@ -87,9 +88,16 @@ cudaError_t launch_swap_epi(const CUtensorMap& tw, const CUtensorMap& tx, const 
 
 cudaError_t launch_gemm_swap(const SwapLaunch& L, cudaStream_t s) {
   CUtensorMap tw, tx;
-  if (!tmap_bf16(&tw, L.W, L.w_rows, L.K, 64)) return cudaErrorInvalidValue;
-  if (!tmap_bf16(&tx, L.X, L.x_rows, L.K, 128)) return cudaErrorInvalidValue;
-  SwapArgs a;
+  // A: K-major weight rows, or (backward) an MN-major [rows, a_cols] matrix;
+  // B: K-major token rows (128-row boxes), or (weight gradients) MN-major.
+  const int a_inner = L.layout == kSwFwd ? L.K : L.a_cols;
+  if (!tmap_bf16(&tw, L.W, L.w_rows, a_inner, 64)) return cudaErrorInvalidValue;
+  if (L.layout == kSwWgrad) {
+    if (!tmap_bf16(&tx, L.X, L.x_rows, L.b_cols, 64)) return cudaErrorInvalidValue;
+  } else if (!tmap_bf16(&tx, L.X, L.x_rows, L.K, 128)) {
+    return cudaErrorInvalidValue;
+  }
+  SwapArgs a = {};
   a.num_groups = L.num_groups;
   a.offsets = L.offsets;
   a.rows = static_cast<int>(L.rows);
@@ -107,11 +115,39 @@ cudaError_t launch_gemm_swap(const SwapLaunch& L, cudaStream_t s) {
   a.bias = static_cast<const __nv_bfloat16*>(L.bias);
   a.addend = static_cast<const __nv_bfloat16*>(L.addend);
   a.status = L.status;
+  a.k_rows_per_group = L.k_rows_per_group;
+  a.b_tiles = L.b_tiles;
+  a.b_cols = L.b_cols;
+  a.out_gstride = L.out_gstride;
+  a.out2 = static_cast<__nv_bfloat16*>(L.out2);
+  a.out3 = static_cast<__nv_bfloat16*>(L.out3);
+  a.ldo2 = L.ldo2;
+  a.aux = static_cast<const __nv_bfloat16*>(L.aux);
+  a.ld_aux = L.ld_aux;
+  a.parts = L.parts;
+  a.ld_parts = L.ld_parts;
+  a.half_cols = L.half_cols;
+  a.counts = L.counts;
+  if (L.layout == kSwWgrad) {
+    const long long tiles_ub = static_cast<long long>(L.num_groups) * L.w_tiles * L.b_tiles;
+    if (L.epi != EPI_STORE_F32) return cudaErrorInvalidValue;
+    return launch_swap_epi<EPI_STORE_F32, kSwWgrad>(tw, tx, a, tiles_ub, s);
+  }
   // token tiles of a segment: ceil(rows_g / 256) at most, so the total is at most rows/256 + #groups
   const long long tt_ub = L.offsets ? L.rows / kSwMaxTile + std::min<long long>(L.num_groups, L.rows)
                                     : (L.rows + kSwMaxTile - 1) / kSwMaxTile;
   const long long tiles_ub = tt_ub * L.w_tiles;
+  if (L.layout == kSwDgrad) {
+    switch (L.epi) {
+      case EPI_STORE_F32: return launch_swap_epi<EPI_STORE_F32, kSwDgrad>(tw, tx, a, tiles_ub, s);
+      case EPI_BWD_GELU_DACT: return launch_swap_epi<EPI_BWD_GELU_DACT, kSwDgrad>(tw, tx, a, tiles_ub, s);
+      case EPI_BWD_SWIGLU_DACT: return launch_swap_epi<EPI_BWD_SWIGLU_DACT, kSwDgrad>(tw, tx, a, tiles_ub, s);
+    }
+    return cudaErrorInvalidValue;
+  }
   switch (L.epi) {
+    case EPI_BWD_GELU_SAVE: return launch_swap_epi<EPI_BWD_GELU_SAVE>(tw, tx, a, tiles_ub, s);
+    case EPI_BWD_SWIGLU_SAVE: return launch_swap_epi<EPI_BWD_SWIGLU_SAVE>(tw, tx, a, tiles_ub, s);
     case EPI_GELU_BIAS: return launch_swap_epi<EPI_GELU_BIAS>(tw, tx, a, tiles_ub, s);
     case EPI_SWIGLU: return launch_swap_epi<EPI_SWIGLU>(tw, tx, a, tiles_ub, s);
     case EPI_SCALE_BIAS: return launch_swap_epi<EPI_SCALE_BIAS>(tw, tx, a, tiles_ub, s);

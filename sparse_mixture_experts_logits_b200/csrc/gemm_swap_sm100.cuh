@@ -32,6 +32,21 @@
 // allocator and (first CTA) MMA issuer, warps 2..9 epilogue.  Every wait is
 // bounded (kWaitTimeoutNs) and reports MOE_DEVERR_TIMEOUT through the status
 // word instead of hanging.
+//
+// Three operand layouts (template LAYOUT), all with the same tiles, TMEM
+// accumulator and epilogue geometry (a TMEM lane is an A index, a column a B
+// index):
+//   kSwFwd    A = weight rows, K-major ([rows, K], the forward GEMMs);
+//             B = token rows, K-major; groups split the token rows.
+//   kSwDgrad  A = a weight stack read MN-major: group g's K rows are
+//             g * k_rows_per_group + k of a [G * K, A_cols] matrix (W2 or
+//             W1 of the nn.Linear layout contracted over its out index, the
+//             input gradients of the backward); B and groups as kSwFwd.
+//   kSwWgrad  A and B both MN-major activations [rows, cols] and the groups
+//             split the contraction (the rows): group g (segment offsets[g]
+//             .. offsets[g+1], a multiple of 64 rows whose padding rows are
+//             zero) gives out[g] = A_g^T B_g, the weight gradients of the
+//             backward.  Every output tile covers 256 A columns x 256 B columns.
 #pragma once
 
 #include "gemm_sm100.cuh"
@@ -71,6 +86,27 @@ struct SwapArgs {
   const __nv_bfloat16* bias;   // EPI_GELU_BIAS / EPI_SCALE_BIAS / EPI_BIAS_ADD: [G, out_cols] or nullptr
   const __nv_bfloat16* addend; // EPI_BIAS_ADD: [rows, ldo] or nullptr
   int* status;
+  // kSwDgrad: K rows of A per group.  kSwWgrad: B tiles per group, valid B
+  // columns (output rows) and output elements per group.
+  int k_rows_per_group;
+  int b_tiles;
+  int b_cols;
+  long long out_gstride;
+  // backward epilogues: second and third bf16 outputs [rows, ldo2] (SAVE),
+  // the saved pre-activations aux [rows, ld_aux] and the per-32-column partial
+  // dot products parts [rows, ld_parts] (DACT), and I, the offset of the up
+  // half in the SwiGLU outputs.
+  __nv_bfloat16* out2;
+  __nv_bfloat16* out3;
+  int ldo2;
+  const __nv_bfloat16* aux;
+  int ld_aux;
+  float* parts;
+  int ld_parts;
+  int half_cols;
+  // optional [G]: rows of group g's segment to compute (the segment starts
+  // at offsets[g] and may be longer: zero padding that no tile covers)
+  const int* counts;
 };
 
 // Token tiles of a segment of `cnt` rows: ceil(cnt / 256) tiles of equal
@@ -84,10 +120,23 @@ __device__ __forceinline__ void token_tiling(int cnt, int& width, int& ntiles) {
 
 struct SwapTile {
   int g, wt, tok0, nrows, n;  // group, weight tile, first token, rows, MMA N
+  int nkb;                    // k-blocks of this tile (kSwWgrad: the group's rows / 64)
 };
 
-__device__ __forceinline__ SwapTile swap_decode(int tile, int G, const int* s_tstart, const int* s_off,
-                                                int w_tiles) {
+// Tiles of one group: token tiles x weight tiles, or (kSwWgrad) the fixed
+// 256 x 256 output tiles of a group that has rows.
+template <int LAYOUT>
+__device__ __forceinline__ int swap_group_tiles(int cnt, const SwapArgs& a) {
+  if constexpr (LAYOUT == kSwWgrad) return cnt > 0 ? a.w_tiles * a.b_tiles : 0;
+  int width, ntt;
+  token_tiling(cnt, width, ntt);
+  return ntt * a.w_tiles;
+}
+
+template <int LAYOUT>
+__device__ __forceinline__ SwapTile swap_decode(int tile, int G, const int* s_tstart, const int* s_cnt,
+                                                const SwapArgs& a, int num_kb) {
+  const int w_tiles = a.w_tiles;
   int lo = 0, hi = G - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -95,7 +144,18 @@ __device__ __forceinline__ SwapTile swap_decode(int tile, int G, const int* s_ts
   }
   SwapTile t;
   t.g = lo;
-  const int cnt = s_off[lo + 1] - s_off[lo];
+  const int cnt = s_cnt[lo];
+  if constexpr (LAYOUT == kSwWgrad) {
+    const int local = tile - s_tstart[lo];
+    t.wt = local % w_tiles;
+    const int bt = local / w_tiles;
+    t.tok0 = bt * kSwMaxTile;
+    t.nrows = min(kSwMaxTile, a.b_cols - t.tok0);
+    t.n = kSwMaxTile;
+    t.nkb = (cnt + kBK - 1) / kBK;
+    return t;
+  }
+  t.nkb = num_kb;
   int width, ntt;
   token_tiling(cnt, width, ntt);
   const int local = tile - s_tstart[lo];
@@ -119,15 +179,54 @@ __device__ __forceinline__ void swap_store(const SwapArgs& a, size_t row, int co
   else
     static_cast<__nv_bfloat16*>(a.out)[row * a.ldo + col] = __float2bfloat16_rn(v);
 }
-
+// Same at an element offset `base` (a group's own output block).
 template <int EPI>
+__device__ __forceinline__ void swap_store(const SwapArgs& a, size_t base, int col, float v, size_t row) {
+  if constexpr (EPI == EPI_SCALE_BIAS || EPI == EPI_STORE_F32)
+    static_cast<float*>(a.out)[base + row * a.ldo + col] = v;
+  else
+    static_cast<__nv_bfloat16*>(a.out)[base + row * a.ldo + col] = __float2bfloat16_rn(v);
+}
+
+// d/dv of the GELU tanh form 0.5 v (1 + tanh(u)), u = c (v + 0.044715 v^3):
+// 0.5 (1 + tanh u) + 0.5 v (1 - tanh^2 u) c (1 + 3 * 0.044715 v^2), with
+// tanh u = 1 - 2 / (1 + e^{2u}).
+__device__ __forceinline__ float gelu_tanh_grad_fast(float v) {
+  const float c = 0.7978845608028654f;
+  const float u = c * fmaf(0.044715f * v, v * v, v);
+  const float th = 1.0f - __fdividef(2.0f, 1.0f + __expf(2.0f * u));
+  return 0.5f * (1.0f + th) + 0.5f * v * (1.0f - th * th) * c * fmaf(3.0f * 0.044715f, v * v, 1.0f);
+}
+
+// Sum over the warp's 32 lanes of v[i] for every i, in 31 shuffles: after
+// the five halving rounds lane L holds the sum of v[L] over all lanes (the
+// butterfly transpose-reduction).  Exact order fixed, so repeatable.
+__device__ __forceinline__ float warp_transpose_sum(float (&v)[32], int lane) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < off; ++i) {
+      const float send = upper ? v[i] : v[i + off];
+      const float keep = upper ? v[i + off] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  return v[0];
+}
+
+template <int EPI, int LAYOUT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     moe_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmap_w,
                          const __grid_constant__ CUtensorMap tmap_x, const SwapArgs args) {
   constexpr int S = kSwStages;
-  constexpr bool kSwiglu = EPI == EPI_SWIGLU;
+  constexpr bool kSwiglu = EPI == EPI_SWIGLU || EPI == EPI_BWD_SWIGLU_SAVE;
+  constexpr bool kAMn = LAYOUT != kSwFwd;
+  constexpr bool kBMn = LAYOUT == kSwWgrad;
+  static_assert(!(kSwiglu && LAYOUT != kSwFwd), "the gate/up pairing reads K-major weight rows");
   extern __shared__ uint8_t dyn_smem[];
   __shared__ int s_off[kMaxExperts + 1];
+  __shared__ int s_cnt[kMaxExperts];
   __shared__ int s_tstart[kMaxExperts + 1];
   __shared__ __align__(8) uint64_t s_full[S];
   __shared__ __align__(8) uint64_t s_empty[S];
@@ -158,16 +257,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     s_off[i] = static_cast<int>(o < 0 ? 0 : (o > args.rows ? args.rows : o));
   }
   __syncthreads();
+  for (int i = threadIdx.x; i < G; i += blockDim.x) {
+    const int seg = max(0, s_off[i + 1] - s_off[i]);
+    s_cnt[i] = args.counts != nullptr ? max(0, min(args.counts[i], seg)) : seg;
+  }
+  __syncthreads();
   if (warp == 0) {
     int carry = 0;
     for (int base = 0; base < G; base += 32) {
       const int g = base + lane;
       int v = 0;
-      if (g < G) {
-        int width, ntt;
-        token_tiling(s_off[g + 1] - s_off[g], width, ntt);
-        v = ntt * args.w_tiles;
-      }
+      if (g < G) v = swap_group_tiles<LAYOUT>(s_cnt[g], args);
       int incl = v;
 #pragma unroll
       for (int d = 1; d < 32; d <<= 1) {
@@ -223,12 +323,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // both CTAs' bytes of one k-block: weight rows + 128 token rows each
     constexpr uint32_t kb_bytes = 2u * (kSwATileBytes + kSwBTileBytes);
     for (int tile = unit; ok && tile < total; tile += units) {
-      const SwapTile t = swap_decode(tile, G, s_tstart, s_off, args.w_tiles);
+      const SwapTile t = swap_decode<LAYOUT>(tile, G, s_tstart, s_cnt, args, num_kb);
+      // kSwFwd / kSwDgrad: B = this CTA's half of the token tile, K-major rows.
+      // kSwWgrad: B = this CTA's 128 of the tile's 256 B columns, rows of the segment.
       const int x_row = s_off[t.g] + t.tok0 + static_cast<int>(rank) * (t.n >> 1);
-      const int w_base = t.g * args.w_rows_per_group + t.wt * args.w_tile_step +
+      const int b_col = t.tok0 + static_cast<int>(rank) * (kSwMaxTile >> 1);
+      // A: kSwFwd weight rows; otherwise the first of this CTA's 128 A columns
+      const int w_base = (LAYOUT == kSwFwd ? t.g * args.w_rows_per_group : 0) + t.wt * args.w_tile_step +
                          static_cast<int>(rank) * args.w_cta_step;
-      for (int kb0 = 0; kb0 < num_kb; kb0 += kSwKB) {
-        const int nk = min(kSwKB, num_kb - kb0);
+      const int k_row0 = LAYOUT == kSwDgrad ? t.g * args.k_rows_per_group : s_off[t.g];
+      for (int kb0 = 0; kb0 < t.nkb; kb0 += kSwKB) {
+        const int nk = min(kSwKB, t.nkb - kb0);
         if (!mbar_wait_all(smem_addr(&s_empty[s]), ph ^ 1u, abort_flag, args.status)) { ok = false; break; }
         if (lane == 0) {
           const uint32_t sa = smem_base + s * kSwStageBytes;
@@ -238,9 +343,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int i = 0; i < nk; ++i) {
             const int kc = (kb0 + i) * kBK;
             const uint32_t ai = sa + i * kSwATileBytes;
-            tma_load_2d_pair(ai, &tmap_w, full_leader, kc, w_base);
-            tma_load_2d_pair(ai + 64 * kBK * 2, &tmap_w, full_leader, kc, w_base + args.w_hi_offset);
-            tma_load_2d_pair(sb + i * kSwBTileBytes, &tmap_x, full_leader, kc, x_row);
+            const uint32_t bi = sb + i * kSwBTileBytes;
+            if constexpr (!kAMn) {
+              tma_load_2d_pair(ai, &tmap_w, full_leader, kc, w_base);
+              tma_load_2d_pair(ai + 64 * kBK * 2, &tmap_w, full_leader, kc, w_base + args.w_hi_offset);
+            } else {
+              // two boxes of 64 A columns x 64 K rows (8 KB each, 8 KB apart)
+              tma_load_2d_pair(ai, &tmap_w, full_leader, w_base, k_row0 + kc);
+              tma_load_2d_pair(ai + 64 * kBK * 2, &tmap_w, full_leader, w_base + args.w_hi_offset, k_row0 + kc);
+            }
+            if constexpr (!kBMn) {
+              tma_load_2d_pair(bi, &tmap_x, full_leader, kc, x_row);
+            } else {
+              tma_load_2d_pair(bi, &tmap_x, full_leader, b_col, k_row0 + kc);
+              tma_load_2d_pair(bi + 64 * kBK * 2, &tmap_x, full_leader, b_col + 64, k_row0 + kc);
+            }
           }
         }
         __syncwarp();
@@ -252,20 +369,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // -------------------------------------------------------- MMA issuer
       uint32_t it = 0, s = 0, ph = 0;
       bool ok = true;
-      // descriptors of stage 0; stage s and k-slice kk add s * stage/16 and 2 * kk
-      // to the 14-bit start-address field, which never carries (smem < 256 KB)
-      const uint64_t da0 = sw128_kmajor_desc(smem_base);
-      const uint64_t db0 = sw128_kmajor_desc(smem_base + kSwKB * kSwATileBytes);
+      // descriptors of stage 0; stage s and k-slice kk add s * stage/16 and
+      // kk * (slice bytes)/16 to the 14-bit start-address field, which never
+      // carries (smem < 256 KB).  A K = 16 slice is 32 bytes along a K-major
+      // row, or 16 rows of 128 bytes (2048 bytes) of an MN-major tile.
+      constexpr uint64_t kAStep = kAMn ? 128 : 2;
+      constexpr uint64_t kBStep = kBMn ? 128 : 2;
+      const uint64_t da0 = kAMn ? sw128_mnmajor_desc(smem_base, 64 * kBK * 2) : sw128_kmajor_desc(smem_base);
+      const uint64_t db0 = kBMn ? sw128_mnmajor_desc(smem_base + kSwKB * kSwATileBytes, 64 * kBK * 2)
+                                : sw128_kmajor_desc(smem_base + kSwKB * kSwATileBytes);
       for (int tile = unit; ok && tile < total; tile += units, ++it) {
-        const SwapTile t = swap_decode(tile, G, s_tstart, s_off, args.w_tiles);
-        const uint32_t idesc = umma_idesc_bf16(256, t.n);
+        const SwapTile t = swap_decode<LAYOUT>(tile, G, s_tstart, s_cnt, args, num_kb);
+        const uint32_t idesc = umma_idesc_bf16_major(256, t.n, kAMn ? 1 : 0, kBMn ? 1 : 0);
         const uint32_t buf = it & 1u;
         const uint32_t tph = (it >> 1) & 1u;
         if (!mbar_wait_all(smem_addr(&s_tempty[buf]), tph ^ 1u, abort_flag, args.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * 256u;
-        for (int kb0 = 0; kb0 < num_kb; kb0 += kSwKB) {
-          const int nk = min(kSwKB, num_kb - kb0);
+        for (int kb0 = 0; kb0 < t.nkb; kb0 += kSwKB) {
+          const int nk = min(kSwKB, t.nkb - kb0);
           if (!mbar_wait_all(smem_addr(&s_full[s]), ph, abort_flag, args.status)) { ok = false; break; }
           if (lane == 0) {
             const uint64_t off = static_cast<uint64_t>(s * (kSwStageBytes >> 4));
@@ -275,9 +397,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const uint64_t a = da0 + off + i * (kSwATileBytes >> 4);
                 const uint64_t b = db0 + off + i * (kSwBTileBytes >> 4);
                 umma_bf16_pair(d_tmem, a, b, idesc, (kb0 | i) != 0 ? 1u : 0u);
-                umma_bf16_pair(d_tmem, a + 2, b + 2, idesc, 1u);
-                umma_bf16_pair(d_tmem, a + 4, b + 4, idesc, 1u);
-                umma_bf16_pair(d_tmem, a + 6, b + 6, idesc, 1u);
+                umma_bf16_pair(d_tmem, a + kAStep, b + kBStep, idesc, 1u);
+                umma_bf16_pair(d_tmem, a + 2 * kAStep, b + 2 * kBStep, idesc, 1u);
+                umma_bf16_pair(d_tmem, a + 3 * kAStep, b + 3 * kBStep, idesc, 1u);
               }
             }
             umma_commit_pair(smem_addr(&s_empty[s]), 0x3);
@@ -308,7 +430,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t it = 0, xc = 0;
     bool ok = true;
     for (int tile = unit; ok && tile < total; tile += units, ++it) {
-      const SwapTile t = swap_decode(tile, G, s_tstart, s_off, args.w_tiles);
+      const SwapTile t = swap_decode<LAYOUT>(tile, G, s_tstart, s_cnt, args, num_kb);
       const uint32_t buf = it & 1u;
       const uint32_t tph = (it >> 1) & 1u;
       if (!mbar_wait(smem_addr(&s_tfull[buf]), tph, abort_flag, args.status)) break;
@@ -317,17 +439,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                               : t.wt * args.cols_per_tile + static_cast<int>(rank) * 128 + m;
       const bool col_ok = col < args.out_cols;
       float bias = 0.f;
-      if constexpr (EPI == EPI_GELU_BIAS || EPI == EPI_SCALE_BIAS || EPI == EPI_BIAS_ADD) {
+      if constexpr (EPI == EPI_GELU_BIAS || EPI == EPI_SCALE_BIAS || EPI == EPI_BIAS_ADD ||
+                    EPI == EPI_BWD_GELU_SAVE) {
         if (args.bias != nullptr && col_ok)
           bias = __bfloat162float(args.bias[static_cast<size_t>(t.g) * args.out_cols + col]);
       }
-      const size_t row0 = static_cast<size_t>(s_off[t.g]) + t.tok0;
+      // output row of the tile's first token (kSwWgrad: the first B column of
+      // the tile, in group g's own output block)
+      const size_t row0 = LAYOUT == kSwWgrad ? static_cast<size_t>(t.tok0)
+                                             : static_cast<size_t>(s_off[t.g]) + t.tok0;
+      const size_t gofs = LAYOUT == kSwWgrad ? static_cast<size_t>(t.g) * args.out_gstride : 0;
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * 256u;
+      constexpr bool kScaled = EPI == EPI_SCALE_BIAS || EPI == EPI_BWD_GELU_SAVE ||
+                               EPI == EPI_BWD_SWIGLU_SAVE || EPI == EPI_BWD_GELU_DACT ||
+                               EPI == EPI_BWD_SWIGLU_DACT;
       for (int c = 32 * part; c < t.n; c += 64) {
         uint32_t r[32];
         MOE_TMEM_LD32(tacc + c, r);
         tmem_ld_wait();
         const int nv = min(32, t.nrows - c);  // tokens of this chunk that exist
+        float rs = 1.f;                       // this lane's token's row scale (gate weight)
+        if constexpr (kScaled) {
+          if (lane < nv && args.row_scale != nullptr) rs = args.row_scale[row0 + c + lane];
+        }
         if constexpr (kSwiglu) {
           if (up_warp) {
             if (!mbar_wait(smem_addr(&s_xempty[pair]), (xc & 1u) ^ 1u, abort_flag, args.status)) { ok = false; break; }
@@ -336,22 +470,71 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_arrive(smem_addr(&s_xfull[pair]));
           } else {
             if (!mbar_wait(smem_addr(&s_xfull[pair]), xc & 1u, abort_flag, args.status)) { ok = false; break; }
-            float v[32];
+            if constexpr (EPI == EPI_SWIGLU) {
+              float v[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = silu_fast(__uint_as_float(r[i])) * xs[lane * kSwXPitch + i];
-            mbar_arrive(smem_addr(&s_xempty[pair]));
-            if (col_ok) {
+              for (int i = 0; i < 32; ++i) v[i] = silu_fast(__uint_as_float(r[i])) * xs[lane * kSwXPitch + i];
+              mbar_arrive(smem_addr(&s_xempty[pair]));
+              if (col_ok) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (i < nv) swap_store<EPI>(args, row0 + c + i, col, v[i]);
+                for (int i = 0; i < 32; ++i)
+                  if (i < nv) swap_store<EPI>(args, row0 + c + i, col, v[i]);
+              }
+            } else {  // EPI_BWD_SWIGLU_SAVE: g, u, a = SiLU(g) u, w a
+              float u[32];
+#pragma unroll
+              for (int i = 0; i < 32; ++i) u[i] = xs[lane * kSwXPitch + i];
+              mbar_arrive(smem_addr(&s_xempty[pair]));
+              __nv_bfloat16* hp = static_cast<__nv_bfloat16*>(args.out);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const float g = __uint_as_float(r[i]);
+                const float a = silu_fast(g) * u[i];
+                const float w = __shfl_sync(0xffffffffu, rs, i);
+                if (col_ok && i < nv) {
+                  const size_t row = row0 + c + i;
+                  hp[row * args.ldo + col] = __float2bfloat16_rn(g);
+                  hp[row * args.ldo + args.half_cols + col] = __float2bfloat16_rn(u[i]);
+                  args.out2[row * args.ldo2 + col] = __float2bfloat16_rn(a);
+                  if (args.out3 != nullptr) args.out3[row * args.ldo2 + col] = __float2bfloat16_rn(w * a);
+                }
+              }
             }
           }
           ++xc;
-        } else {
-          float rs = 1.f;
-          if constexpr (EPI == EPI_SCALE_BIAS) {
-            if (lane < nv) rs = args.row_scale[row0 + c + lane];
+        } else if constexpr (EPI == EPI_BWD_GELU_DACT || EPI == EPI_BWD_SWIGLU_DACT) {
+          // G = acc (the gradient reaching a, before the gate weight); dh out,
+          // and per token the partial <G, a> over this warp's 32 columns
+          float prod[32];
+          __nv_bfloat16* dh = static_cast<__nv_bfloat16*>(args.out);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float G = __uint_as_float(r[i]);
+            const float w = __shfl_sync(0xffffffffu, rs, i);
+            prod[i] = 0.f;
+            if (col_ok && i < nv) {
+              const size_t row = row0 + c + i;
+              if constexpr (EPI == EPI_BWD_GELU_DACT) {
+                const float h = __bfloat162float(args.aux[row * args.ld_aux + col]);
+                dh[row * args.ldo + col] = __float2bfloat16_rn(w * G * gelu_tanh_grad_fast(h));
+                prod[i] = G * gelu_tanh_fast(h);
+              } else {
+                const float g = __bfloat162float(args.aux[row * args.ld_aux + col]);
+                const float u = __bfloat162float(args.aux[row * args.ld_aux + args.half_cols + col]);
+                const float sg = __fdividef(1.0f, 1.0f + __expf(-g));
+                const float si = g * sg;
+                const float da = w * G;
+                dh[row * args.ldo + col] = __float2bfloat16_rn(da * u * sg * fmaf(g, 1.0f - sg, 1.0f));
+                dh[row * args.ldo + args.half_cols + col] = __float2bfloat16_rn(da * si);
+                prod[i] = G * si * u;
+              }
+            }
           }
+          const float tot = warp_transpose_sum(prod, lane);
+          // one partial per 32-column chunk that holds any valid column
+          if (args.parts != nullptr && lane < nv && col - lane < args.out_cols)
+            args.parts[(row0 + c + lane) * args.ld_parts + ((col - lane) >> 5)] = tot;
+        } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             float v = __uint_as_float(r[i]) + bias;
@@ -361,7 +544,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               if (args.addend != nullptr && col_ok && i < nv)
                 v += __bfloat162float(args.addend[(row0 + c + i) * args.ldo + col]);
             }
-            if (col_ok && i < nv) swap_store<EPI>(args, row0 + c + i, col, v);
+            if constexpr (EPI == EPI_BWD_GELU_SAVE) {
+              const float a = gelu_tanh_fast(v);
+              const float w = __shfl_sync(0xffffffffu, rs, i);
+              if (col_ok && i < nv) {
+                const size_t row = row0 + c + i;
+                static_cast<__nv_bfloat16*>(args.out)[row * args.ldo + col] = __float2bfloat16_rn(v);
+                args.out2[row * args.ldo2 + col] = __float2bfloat16_rn(a);
+                if (args.out3 != nullptr) args.out3[row * args.ldo2 + col] = __float2bfloat16_rn(w * a);
+              }
+            } else {
+              if (col_ok && i < nv) swap_store<EPI>(args, gofs, col, v, row0 + c + i);
+            }
           }
         }
       }

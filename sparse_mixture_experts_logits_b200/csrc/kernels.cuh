@@ -74,8 +74,9 @@ moe_status_t check_device();
 // side (see gemm_swap_sm100.cuh).  `epi` is a GemmEpilogue.
 struct SwapLaunch {
   int epi;
-  const void* W; long long w_rows;  // bf16 [w_rows, K] weight stack
-  const void* X; long long x_rows;  // bf16 [x_rows, K] token rows in dispatch order
+  int layout;                       // kSwFwd (0), kSwDgrad (1) or kSwWgrad (2) of gemm_swap_sm100.cuh
+  const void* W; long long w_rows;  // bf16 [w_rows, K] weight stack (kSwFwd), [w_rows, a_cols] otherwise
+  const void* X; long long x_rows;  // bf16 [x_rows, K] token rows in dispatch order ([x_rows, b_cols]: kSwWgrad)
   int K;
   int num_groups;
   const int* offsets;        // device [G+1] or nullptr (single group of `rows` rows)
@@ -87,6 +88,16 @@ struct SwapLaunch {
   const void* bias;
   const void* addend;        // EPI_BIAS_ADD: bf16 [rows, ldo] or nullptr
   int* status;
+  // backward layouts and epilogues (see SwapArgs)
+  int a_cols;                // columns of the MN-major A matrix
+  int k_rows_per_group;      // kSwDgrad
+  int b_tiles, b_cols;       // kSwWgrad
+  long long out_gstride;     // kSwWgrad
+  void* out2; void* out3; int ldo2;
+  const void* aux; int ld_aux;
+  float* parts; int ld_parts;
+  int half_cols;
+  const int* counts;         // optional [G]: rows computed per group (segments start at offsets)
 };
 cudaError_t launch_gemm_swap(const SwapLaunch& L, cudaStream_t s);
 
@@ -107,6 +118,22 @@ struct SimtLaunch {
   const float* addend;  // EPI_BIAS_ADD: [rows, ldo] or nullptr
 };
 cudaError_t launch_simt_gemm(const SimtLaunch& L, cudaStream_t s);
+
+// bwd_tc.cu: helpers of the tensor-core backward (bf16 layers), which keeps
+// its per-row tensors in a dispatch order padded per expert to 64 rows.
+cudaError_t launch_pad_dispatch(const int32_t* idx, const int32_t* slot_of, const float* topk_w,
+                                const int32_t* counts, const int32_t* offsets, int T, int k, int M,
+                                long long rows_cap, int32_t* offsets_pad, int32_t* slot_pad,
+                                int32_t* row_token_pad, float* row_w_pad, cudaStream_t s);
+cudaError_t launch_gather_pad(const void* src, const int32_t* row_token_pad, const int32_t* n_rows, void* dst,
+                              long long rows_cap, int T, int D, cudaStream_t s);
+cudaError_t launch_zero_pad_rows(const int32_t* counts, const int32_t* offsets_pad, int M, void* buf,
+                                 long long rows_cap, int cols_bf16, cudaStream_t s);
+cudaError_t launch_dw_finish(const float* parts, int nparts, const int32_t* slot_pad, const int32_t* idx,
+                             const void* dy, const void* b2, int D, int M, int T, int k, float* dw, cudaStream_t s);
+cudaError_t launch_colsum_bf16(const void* Y, long long ldy, const float* scale, const int32_t* offsets, int G,
+                               long long rows_cap, int N, float* out, cudaStream_t s);
+cudaError_t launch_zero_empty_groups(const int32_t* counts, int G, long long per_group, float* out, cudaStream_t s);
 
 // backward.cu: C (+)= A B^T on the CUDA cores, fp32 sums, with strided
 // operands: A(m, k) = A[m * a_sm + k * a_sk], B(n, k) = B[g * b_gstride +

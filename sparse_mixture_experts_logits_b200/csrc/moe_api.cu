@@ -870,10 +870,52 @@ namespace {
 struct BwdWs {
   FwdWs f;
   size_t xp, hpre, act, dO, da, dxp, dwp, dl, hs, as, das, dxs, total;
+  // tensor-core path (bf16): the padded dispatch order and its bf16 tensors
+  long long rows_pad;
+  size_t offp, slotp, rtp, rwp, xpp, dypp, hpb, ab, awb, dhb, dxpp, parts, hsb, asb, dhsb;
 };
 
+// Rows of the backward's padded dispatch order: every expert's segment is
+// rounded up to 64 rows, so at most T k + 63 M rows.
+long long padded_rows(const moe_layer_desc_t* d) {
+  return (static_cast<long long>(d->T) * d->k + 63ll * d->M + 63) / 64 * 64;
+}
+
+BwdWs backward_layout_tc(const moe_layer_desc_t* d) {
+  BwdWs L{};
+  L.f = forward_layout(d);
+  Carve c;
+  c.off = L.f.pub.total;
+  const size_t pairs = static_cast<size_t>(d->T) * d->k;
+  const size_t n1 = d->act == MOE_ACT_SWIGLU ? 2ull * d->I : static_cast<size_t>(d->I);
+  const size_t Ha = d->I, T = d->T, Is = d->I_sh, D = d->D;
+  const size_t P = static_cast<size_t>(padded_rows(d));
+  L.rows_pad = static_cast<long long>(P);
+  L.offp = c.take((d->M + 1) * 4);
+  L.slotp = c.take(pairs * 4);
+  L.rtp = c.take(P * 4);
+  L.rwp = c.take(P * 4);
+  L.xpp = c.take(P * D * 2);
+  L.dypp = c.take(P * D * 2);
+  L.hpb = c.take(P * n1 * 2);
+  L.ab = c.take(P * Ha * 2);
+  L.awb = c.take(P * Ha * 2);
+  L.dhb = c.take(P * n1 * 2);
+  L.dxpp = c.take(P * D * 4);
+  L.parts = c.take(P * ((Ha + 31) / 32) * 4);
+  L.dwp = c.take(pairs * 4);
+  L.dl = c.take(T * d->M * 4);
+  L.hsb = c.take(T * 2 * Is * 2);
+  L.asb = c.take(T * Is * 2);
+  L.dhsb = c.take(T * 2 * Is * 2);
+  L.dxs = c.take(T * D * 4);
+  L.total = c.off;
+  return L;
+}
+
 BwdWs backward_layout(const moe_layer_desc_t* d) {
-  BwdWs L;
+  if (d->dtype == MOE_DTYPE_BF16) return backward_layout_tc(d);
+  BwdWs L{};
   L.f = forward_layout(d);
   Carve c;
   c.off = L.f.pub.total;
@@ -926,6 +968,222 @@ moe_status_t zero_param_grads(const moe_layer_desc_t* d, const moe_grads_t* g, c
   return MOE_OK;
 }
 
+// A tokens-on-N GEMM of the backward: A is the weight stack (K-major for
+// the recomputed forward, MN-major for the input gradients) or an MN-major
+// activation (weight gradients), B the token rows.
+SwapLaunch bwd_swap(int epi, int layout, const void* A, long long a_rows, const void* B, long long b_rows, int K,
+                    int G, const int32_t* offsets, const int32_t* counts, long long rows, int out_cols, void* out,
+                    int ldo, int* status) {
+  SwapLaunch L{};
+  L.epi = epi;
+  L.layout = layout;
+  L.W = A;
+  L.w_rows = a_rows;
+  L.X = B;
+  L.x_rows = b_rows;
+  L.K = K;
+  L.num_groups = G;
+  L.offsets = offsets;
+  L.counts = counts;
+  L.rows = rows;
+  L.w_tiles = (out_cols + 255) / 256;
+  L.w_tile_step = 256;
+  L.w_hi_offset = 64;
+  L.w_cta_step = 128;
+  L.cols_per_tile = 256;
+  L.out_cols = out_cols;
+  L.a_cols = out_cols;
+  L.ldo = ldo;
+  L.out = out;
+  L.status = status;
+  return L;
+}
+
+// The backward of a bf16 layer on the tensor cores.  Per expert segment
+// (rows r of the padded dispatch order, token t(r), gate weight w_r):
+//   recompute  h = x W1^T (+ b1), a = act(h), aw = w a         (save epilogue)
+//   dgrad      G = dy W2;  dh = w G act'(h);  parts = <G, a>   (fused epilogue)
+//              dx_rows = dh W1                                  (fp32)
+//   wgrad      dW2 = dy^T aw,  dW1 = dh^T x  over the segment   (grouped-K GEMMs)
+//   dw[t, j]   = <G, a> + <dy_t, b2>  (the gradient reaching the gate weight)
+// then the shared expert the same way with w = 1, the router's backward, and
+// dx_t = sum_j dx_rows + shared dx + router dx, rounded once.
+moe_status_t backward_tc_impl(const moe_layer_desc_t* d, const moe_weights_t* w, const void* x, const void* dy,
+                              const moe_grads_t* g, void* ws, cudaStream_t s) {
+  const bool swiglu = d->act == MOE_ACT_SWIGLU;
+  const bool biases = !swiglu && d->has_bias;
+  const BwdWs L = backward_layout(d);
+  const int T = d->T, D = d->D, M = d->M, k = d->k, Ha = d->I, Is = d->I_sh;
+  const int n1 = swiglu ? 2 * d->I : d->I;
+  const long long pairs = static_cast<long long>(T) * k;
+  const long long P = L.rows_pad;
+  const int nparts = (Ha + 31) / 32;
+  int* status = at<int*>(ws, L.f.pub.status);
+  int32_t* idx = at<int32_t*>(ws, L.f.pub.topk_idx);
+  float* tw = at<float*>(ws, L.f.pub.topk_w);
+  int32_t* counts = at<int32_t*>(ws, L.f.pub.counts);
+  int32_t* offsets = at<int32_t*>(ws, L.f.pub.offsets);
+  int32_t* slot_of = at<int32_t*>(ws, L.f.pub.slot_of);
+  int32_t* row_token = at<int32_t*>(ws, L.f.pub.row_token);
+  float* row_w = at<float*>(ws, L.f.pub.row_w);
+  float* logits = at<float*>(ws, L.f.logits);
+  int32_t* offp = at<int32_t*>(ws, L.offp);
+  int32_t* slotp = at<int32_t*>(ws, L.slotp);
+  int32_t* rtp = at<int32_t*>(ws, L.rtp);
+  float* rwp = at<float*>(ws, L.rwp);
+  void* xpp = at<void*>(ws, L.xpp);
+  void* dypp = at<void*>(ws, L.dypp);
+  void* hpb = at<void*>(ws, L.hpb);
+  void* ab = at<void*>(ws, L.ab);
+  void* awb = at<void*>(ws, L.awb);
+  void* dhb = at<void*>(ws, L.dhb);
+  float* dxpp = at<float*>(ws, L.dxpp);
+  float* parts = at<float*>(ws, L.parts);
+  float* dwp = at<float*>(ws, L.dwp);
+  float* dl = at<float*>(ws, L.dl);
+  float* dxs = at<float*>(ws, L.dxs);
+  const int32_t* n_rows_pad = offp + M;
+  Range whole("moe_backward");
+  MOE_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
+  {
+    Range r("moe.route");
+    MOE_TRY(run_route(x, w->w_r, w->e_bias, T, D, M, k, d->dtype, d->gate, d->norm_topk_prob,
+                      d->routed_scaling_factor, d->eps, d->n_group, d->topk_group, idx, tw, logits,
+                      at<void*>(ws, L.f.wrT), status, s));
+  }
+  {
+    Range r("moe.dispatch");
+    MOE_CUDA(launch_permute(idx, tw, T, k, M, counts, offsets, slot_of, row_token, row_w,
+                            at<int32_t*>(ws, L.f.chunk_counts), at<int32_t*>(ws, L.f.chunk_base), status, s));
+    MOE_CUDA(launch_pad_dispatch(idx, slot_of, tw, counts, offsets, T, k, M, P, offp, slotp, rtp, rwp, s));
+    MOE_CUDA(launch_gather_pad(x, rtp, n_rows_pad, xpp, P, T, D, s));
+    MOE_CUDA(launch_gather_pad(dy, rtp, n_rows_pad, dypp, P, T, D, s));
+    // padding rows of the weight-gradient operands that no GEMM tile writes
+    MOE_CUDA(launch_zero_pad_rows(counts, offp, M, awb, P, Ha, s));
+    MOE_CUDA(launch_zero_pad_rows(counts, offp, M, dhb, P, n1, s));
+  }
+  {
+    Range r("moe.experts_backward");
+    // recompute: h (bf16), a = act(h), aw = w a
+    SwapLaunch ga{};
+    if (swiglu) {
+      ga = bwd_swap(EPI_BWD_SWIGLU_SAVE, kSwFwd, w->w1, 1ll * M * n1, xpp, P, D, M, offp, counts, P, Ha, hpb, n1,
+                    status);
+      ga.w_rows_per_group = n1;
+      ga.w_tiles = (Ha + 127) / 128;
+      ga.w_tile_step = 128;
+      ga.w_hi_offset = Ha;
+      ga.w_cta_step = 64;
+      ga.cols_per_tile = 128;
+      ga.half_cols = Ha;
+    } else {
+      ga = bwd_swap(EPI_BWD_GELU_SAVE, kSwFwd, w->w1, 1ll * M * Ha, xpp, P, D, M, offp, counts, P, Ha, hpb, Ha,
+                    status);
+      ga.w_rows_per_group = Ha;
+      ga.bias = biases ? w->b1 : nullptr;
+    }
+    ga.out2 = ab;
+    ga.out3 = awb;
+    ga.ldo2 = Ha;
+    ga.row_scale = rwp;
+    MOE_CUDA(launch_gemm_swap(ga, s));
+    // G = dy W2 (W2 read MN-major); dh = w G act'(h); per-32-column <G, a>
+    SwapLaunch gb = bwd_swap(swiglu ? EPI_BWD_SWIGLU_DACT : EPI_BWD_GELU_DACT, kSwDgrad, w->w2, 1ll * M * D, dypp,
+                             P, D, M, offp, counts, P, Ha, dhb, n1, status);
+    gb.k_rows_per_group = D;
+    gb.aux = hpb;
+    gb.ld_aux = n1;
+    gb.half_cols = Ha;
+    gb.row_scale = rwp;
+    gb.parts = parts;
+    gb.ld_parts = nparts;
+    MOE_CUDA(launch_gemm_swap(gb, s));
+    // dx rows = dh W1 (W1 read MN-major), fp32
+    SwapLaunch gc = bwd_swap(EPI_STORE_F32, kSwDgrad, w->w1, 1ll * M * n1, dhb, P, n1, M, offp, counts, P, D, dxpp,
+                             D, status);
+    gc.k_rows_per_group = n1;
+    MOE_CUDA(launch_gemm_swap(gc, s));
+    // weight gradients over each expert's padded segment
+    SwapLaunch gd = bwd_swap(EPI_STORE_F32, kSwWgrad, awb, P, dypp, P, 0, M, offp, nullptr, P, Ha, g->dw2, Ha,
+                             status);
+    gd.b_cols = D;
+    gd.b_tiles = (D + 255) / 256;
+    gd.out_gstride = 1ll * D * Ha;
+    MOE_CUDA(launch_gemm_swap(gd, s));
+    SwapLaunch ge = bwd_swap(EPI_STORE_F32, kSwWgrad, xpp, P, dhb, P, 0, M, offp, nullptr, P, D, g->dw1, D,
+                             status);
+    ge.b_cols = n1;
+    ge.b_tiles = (n1 + 255) / 256;
+    ge.out_gstride = 1ll * n1 * D;
+    MOE_CUDA(launch_gemm_swap(ge, s));
+    MOE_CUDA(launch_zero_empty_groups(counts, M, 1ll * D * Ha, g->dw2, s));
+    MOE_CUDA(launch_zero_empty_groups(counts, M, 1ll * n1 * D, g->dw1, s));
+    MOE_CUDA(launch_dw_finish(parts, nparts, slotp, idx, dy, biases ? w->b2 : nullptr, D, M, T, k, dwp, s));
+    if (biases) {
+      MOE_CUDA(launch_colsum_bf16(dypp, D, rwp, offp, M, P, D, g->db2, s));
+      MOE_CUDA(launch_colsum_bf16(dhb, n1, nullptr, offp, M, P, Ha, g->db1, s));
+    }
+  }
+  if (Is > 0) {
+    Range r("moe.shared_expert_backward");
+    void* hsb = at<void*>(ws, L.hsb);
+    void* asb = at<void*>(ws, L.asb);
+    void* dhsb = at<void*>(ws, L.dhsb);
+    SwapLaunch sa = bwd_swap(EPI_BWD_SWIGLU_SAVE, kSwFwd, w->sh_w1, 2ll * Is, x, T, D, 1, nullptr, nullptr, T, Is,
+                             hsb, 2 * Is, status);
+    sa.w_rows_per_group = 2 * Is;
+    sa.w_tiles = (Is + 127) / 128;
+    sa.w_tile_step = 128;
+    sa.w_hi_offset = Is;
+    sa.w_cta_step = 64;
+    sa.cols_per_tile = 128;
+    sa.half_cols = Is;
+    sa.out2 = asb;
+    sa.ldo2 = Is;
+    MOE_CUDA(launch_gemm_swap(sa, s));
+    SwapLaunch sb = bwd_swap(EPI_BWD_SWIGLU_DACT, kSwDgrad, w->sh_w2, D, dy, T, D, 1, nullptr, nullptr, T, Is, dhsb,
+                             2 * Is, status);
+    sb.k_rows_per_group = D;
+    sb.aux = hsb;
+    sb.ld_aux = 2 * Is;
+    sb.half_cols = Is;
+    MOE_CUDA(launch_gemm_swap(sb, s));
+    SwapLaunch sc = bwd_swap(EPI_STORE_F32, kSwDgrad, w->sh_w1, 2ll * Is, dhsb, T, 2 * Is, 1, nullptr, nullptr, T,
+                             D, dxs, D, status);
+    sc.k_rows_per_group = 2 * Is;
+    MOE_CUDA(launch_gemm_swap(sc, s));
+    SwapLaunch sd = bwd_swap(EPI_STORE_F32, kSwWgrad, asb, T, dy, T, 0, 1, nullptr, nullptr, T, Is, g->dsh_w2, Is,
+                             status);
+    sd.b_cols = D;
+    sd.b_tiles = (D + 255) / 256;
+    MOE_CUDA(launch_gemm_swap(sd, s));
+    SwapLaunch se = bwd_swap(EPI_STORE_F32, kSwWgrad, x, T, dhsb, T, 0, 1, nullptr, nullptr, T, D, g->dsh_w1, D,
+                             status);
+    se.b_cols = 2 * Is;
+    se.b_tiles = (2 * Is + 255) / 256;
+    MOE_CUDA(launch_gemm_swap(se, s));
+  }
+  {
+    Range r("moe.router_backward");
+    MOE_CUDA(launch_bwd_router(logits, idx, dwp, T, M, k, d->gate, d->norm_topk_prob, d->routed_scaling_factor,
+                               d->eps, dl, s));
+    BwdGemmLaunch wr = bwd_gemm(x, 1, D, true, dl, 1, M, 0, false, g->dw_r, M, D, T, M);
+    wr.mode = 1;
+    MOE_CUDA(launch_bwd_gemm(wr, s));
+    BwdGemmLaunch xr = bwd_gemm(dl, M, 1, false, w->w_r, M, 1, 0, true, dxs, D, T, M, D);
+    xr.accumulate = Is > 0 ? 1 : 0;  // onto the shared expert's dx
+    MOE_CUDA(launch_bwd_gemm(xr, s));
+  }
+  {
+    Range r("moe.combine_backward");
+    MOE_CUDA(launch_combine(d->dtype, dxpp, slotp, dxs, true, nullptr, g->dx, T, D, k, s));
+  }
+  (void)row_token;
+  (void)row_w;
+  (void)pairs;
+  return MOE_OK;
+}
+
 moe_status_t backward_impl(const moe_layer_desc_t* d, const moe_weights_t* w, const void* x, const void* dy,
                            const moe_grads_t* g, void* ws, size_t ws_bytes, cudaStream_t s) {
   MOE_TRY(check_desc(d));
@@ -944,6 +1202,7 @@ moe_status_t backward_impl(const moe_layer_desc_t* d, const moe_weights_t* w, co
   const BwdWs L = backward_layout(d);
   if (ws_bytes < L.total) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_device());
+  if (d->dtype == MOE_DTYPE_BF16) return backward_tc_impl(d, w, x, dy, g, ws, s);
   const bool bf = d->dtype == MOE_DTYPE_BF16;
   const int T = d->T, D = d->D, M = d->M, k = d->k, Ha = d->I, Is = d->I_sh;
   const int n1 = swiglu ? 2 * d->I : d->I;
@@ -1068,6 +1327,17 @@ moe_status_t moe_backward(const moe_layer_desc_t* d, const moe_weights_t* w, con
 
 int moe_backward_launch_count(const moe_layer_desc_t* d) {
   if (check_desc(d) != MOE_OK || d->T == 0) return 0;
+  if (d->dtype == MOE_DTYPE_BF16) {
+    int n = 3;  // transpose + logits GEMM or split-K logits + reduction; top-k
+    n += static_cast<long long>(d->T) * d->k <= 2048 ? 1 : 3;                    // counting sort
+    n += 2 + 2 + 2;        // padded order (offsets, pairs), two gathers, two padding zero-fills
+    n += 5 + 2 + 1;        // five expert GEMMs, empty-expert zero-fills, gate-weight gradients
+    if (d->act == MOE_ACT_GELU_TANH && d->has_bias) n += 2;        // bias gradients
+    if (d->I_sh > 0) n += 5;                                         // shared expert GEMMs
+    n += 3;                                                          // router backward, dW_r, router dx
+    n += 1;                                                          // dx combine
+    return n;
+  }
   int n = d->dtype == MOE_DTYPE_BF16 ? 3 : 2;                        // router logits + top-k
   n += static_cast<long long>(d->T) * d->k <= 2048 ? 1 : 3;          // counting sort
   n += 1;                                                            // gather

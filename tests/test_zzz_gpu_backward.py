@@ -3,11 +3,20 @@ oracle, through the C ABI, on identical seeded inputs.
 
 The GPU recomputes the routing; where its top-k differs from the oracle's
 only at a near-tie, the oracle takes the GPU's choice (as in the forward
-tests).  Every gradient of the GPU is fp32 sums of the layer-dtype inputs
-with fp32 intermediates, so against the fp64 oracle the parameter
-gradients agree to a few fp32 ulps times the length of the sums; the bound
-below leaves two orders of magnitude of room.  dx of a bf16 layer is
-rounded to bf16 once and is held to the forward's output tolerance.
+tests).
+
+Tolerances.  An fp32 layer's backward runs on the CUDA cores: fp32 sums of
+fp32 values, so against the fp64 oracle its gradients agree to a few fp32
+ulps times the length of the sums; the bound below leaves two orders of
+magnitude of room.  A bf16 layer's backward runs on the tensor cores with
+the forward's arithmetic: bf16 operands (the given x, dy and weights, and
+the recomputed h, a = act(h), w a and dh rounded to bf16 before they feed
+the next GEMM) and fp32 accumulation.  Each such rounding is a relative
+error below 2^-9 per element, of random sign, so a sum over many terms is
+off by about 1e-3 of its rms; the bf16 gradients are held to the bound the
+problem statement gives for outputs of exactly this arithmetic: max error
+<= 2e-2 rms and mean relative error <= 5e-3.  dx of a bf16 layer is rounded
+to bf16 once and is held to the forward's output tolerance.
 
 Collected after every forward suite (test_zzz_*), so that a run stopping at
 the first failure has already checked the forward path."""
@@ -21,8 +30,10 @@ from gpu_common import check_routing, check_y, gpu_inputs, np64, oracle_route
 
 pytestmark = pytest.mark.gpu
 
-GRAD_MAX_OVER_RMS = 1e-3   # max |g - g_ref| <= 1e-3 * rms(g_ref)
-GRAD_MEAN_REL = 1e-4       # sum |g - g_ref| / sum |g_ref| <= 1e-4
+GRAD_MAX_OVER_RMS = 1e-3   # fp32 layers: max |g - g_ref| <= 1e-3 * rms(g_ref)
+GRAD_MEAN_REL = 1e-4       # fp32 layers: sum |g - g_ref| / sum |g_ref| <= 1e-4
+BF16_GRAD_MAX_OVER_RMS = 2e-2  # bf16 layers (tensor cores): the forward's output bound
+BF16_GRAD_MEAN_REL = 5e-3
 PARAM_GRADS = ("dw_r", "dw1", "dw2", "db1", "db2", "dsh_w1", "dsh_w2")
 
 
@@ -89,12 +100,18 @@ def check_one_expert(cfg, inp, dy, idx, w_ref, g, e):
         w_ref[tt, jj][:, None] * dyh)
     for name in ("dw1", "dw2", "db1", "db2"):
         if ref[name] is not None:
-            check_grad(name, np64(g[name][e]), ref[name])
+            check_grad(name, np64(g[name][e]), ref[name], cfg["dtype"])
 
 
-def check_grad(name, got, ref):
+def check_grad(name, got, ref, dtype="f32"):
     m = oracle.error_metrics(got, ref)
-    assert m["max_over_rms"] <= GRAD_MAX_OVER_RMS and m["mean_rel"] <= GRAD_MEAN_REL, (name, m)
+    lim = (GRAD_MAX_OVER_RMS, GRAD_MEAN_REL) if dtype == "f32" else (BF16_GRAD_MAX_OVER_RMS, BF16_GRAD_MEAN_REL)
+    if not np.any(ref):
+        # an exactly zero reference (one expert with weight 1: no router gradient) must be met exactly
+        assert not np.any(got), (name, float(np.abs(got).max()))
+        return m
+    assert m["max_over_rms"] <= lim[0] and m["mean_rel"] <= lim[1], (name, m)
+    return m
 
 
 def check_dx(cfg, got, ref):
@@ -106,11 +123,13 @@ def check_dx(cfg, got, ref):
 
 def check_all(cfg, g, ref):
     check_dx(cfg, np64(g["dx"]), ref["dx"])
+    out = {}
     for name in PARAM_GRADS:
         if ref[name] is None:
             assert name not in g
             continue
-        check_grad(name, np64(g[name]), ref[name])
+        out[name] = check_grad(name, np64(g[name]), ref[name], cfg["dtype"])
+    return out
 
 
 SMALL = ["glam_tiny_f32", "glam_small_bf16", "glm_small_bf16", "glm_small_f32", "glm_grouped_bf16",
@@ -127,10 +146,15 @@ def test_backward_matches_oracle(B, name):
 
 @pytest.mark.parametrize("name,over", [("glm_small_bf16", dict(T=1)), ("glm_small_bf16", dict(T=65)),
                                        ("glm_small_bf16", dict(T=129, k=1)), ("glm_small_bf16", dict(k=16)),
-                                       ("glam_small_bf16", dict(M=1, k=1)), ("glm_small_f32", dict(T=200))])
+                                       ("glam_small_bf16", dict(M=1, k=1)), ("glm_small_f32", dict(T=200)),
+                                       ("glm_medium_bf16", dict()), ("glam_small_bf16", dict(T=700)),
+                                       ("glm_small_bf16", dict(I_sh=0)),
+                                       ("glm_medium_bf16", dict(e_bias=("zipf", 1.1, 1.0)))])
 def test_backward_edge_shapes(B, name, over):
     """A single token, ragged tiles, k = 1, k = M, one expert (softmax: its
-    weight is exactly 1, so the router gradient is exactly 0)."""
+    weight is exactly 1, so the router gradient is exactly 0), several
+    256-row token tiles per expert, no shared expert, and a skewed routing
+    that leaves most experts empty (their weight gradients exactly 0)."""
     cfg = ms.get_config(name, **over)
     inp, dy, _, g, idx, _ = run(B, cfg)
     ref = oracle.moe_backward.moe_backward(cfg, host(inp), np64(dy), idx=idx)
@@ -150,8 +174,8 @@ def test_backward_decode_full_size_sampled(B):
     check_one_expert(cfg, inp, dy, idx, w_ref, g, int(idx[0, 0]))
     sh = oracle.moe_backward.expert_ffn_backward(np64(inp["x"]), "swiglu", np64(inp["sh_w1"]),
                                                  np64(inp["sh_w2"]), None, None, np64(dy))
-    check_grad("dsh_w1", np64(g["dsh_w1"]), sh["dw1"])
-    check_grad("dsh_w2", np64(g["dsh_w2"]), sh["dw2"])
+    check_grad("dsh_w1", np64(g["dsh_w1"]), sh["dw1"], cfg["dtype"])
+    check_grad("dsh_w2", np64(g["dsh_w2"]), sh["dw2"], cfg["dtype"])
 
 
 def test_backward_glam_full_size_sampled(B):

@@ -73,7 +73,12 @@ def expert_ffn_backward(xe, act, w1e, w2e, b1e, b2e, dout):
     [GLM5-SE]) on rows xe [n, D] with upstream gradient dout [n, D].
 
     Returns out (the forward value), dx [n, D], dw1 (shape of w1e), dw2
-    (shape of w2e), db1, db2 (None when the bias is absent)."""
+    (shape of w2e), db1, db2 (None when the bias is absent), and for the
+    weight gradients the sums of the absolute values of their terms,
+    dw1_abs = |dpre|^T |x|, dw2_abs = |dout|^T |a|, db1_abs = sum |dpre|:
+    the scale of the rounding error of a sum whose terms carry a relative
+    error (|fl(sum p_i) - sum p_i| <= u sum |p_i| when each p_i is off by
+    at most u of itself)."""
     xe, w1e, w2e, dout = _f64(xe), _f64(w1e), _f64(w2e), _f64(dout)
     pre = xe @ w1e.T                                   # W1 x  [n, H] or [n, 2I]
     if act == "gelu_tanh":
@@ -99,7 +104,9 @@ def expert_ffn_backward(xe, act, w1e, w2e, b1e, b2e, dout):
     db1 = dpre.sum(axis=0) if (act == "gelu_tanh" and b1e is not None) else None
     dw1 = dpre.T @ xe
     dx = dpre @ w1e
-    return {"out": out, "dx": dx, "dw1": dw1, "dw2": dw2, "db1": db1, "db2": db2}
+    return {"out": out, "dx": dx, "dw1": dw1, "dw2": dw2, "db1": db1, "db2": db2,
+            "dw1_abs": np.abs(dpre).T @ np.abs(xe), "dw2_abs": np.abs(dout).T @ np.abs(a),
+            "db1_abs": None if db1 is None else np.abs(dpre).sum(axis=0)}
 
 
 def router_backward(idx, dw, logits, g, gate, norm_topk_prob, alpha, eps):
@@ -163,9 +170,11 @@ def moe_backward(cfg, inp, dy, idx=None):
     ``moe_oracle.moe_forward`` (no addend: an added term only passes dy on).
 
     Returns dx [T, D], dw_r [D, M], dw1 / dw2 (stacked like w1 / w2),
-    db1 / db2 (or None), dsh_w1 / dsh_w2 (or None), and the intermediate
+    db1 / db2 (or None), dsh_w1 / dsh_w2 (or None), the intermediate
     dw [T, k] (gradient of each chosen weight) and dl [T, M] (of the
-    logits), with the forward's routing."""
+    logits), with the forward's routing, and the absolute-term sums
+    (*_abs) of the expert and shared weight gradients (see
+    expert_ffn_backward)."""
     r = F.route(inp["x"], inp["w_r"], inp.get("e_bias"), cfg["k"], cfg["gate"],
                 cfg["norm_topk_prob"], cfg["alpha"], cfg["eps"], cfg.get("n_group", 1),
                 cfg.get("topk_group", 1))
@@ -182,7 +191,9 @@ def moe_backward(cfg, inp, dy, idx=None):
     b2 = None if inp.get("b2") is None else _f64(inp["b2"])
     dx = np.zeros((T, D))
     dw1, dw2 = np.zeros_like(w1), np.zeros_like(w2)
+    dw1_abs, dw2_abs = np.zeros_like(w1), np.zeros_like(w2)
     db1 = None if b1 is None else np.zeros_like(b1)
+    db1_abs = None if b1 is None else np.zeros_like(b1)
     db2 = None if b2 is None else np.zeros_like(b2)
     dw = np.zeros((T, k))
     for e in range(M):
@@ -197,22 +208,28 @@ def moe_backward(cfg, inp, dy, idx=None):
         np.add.at(dx, tt, g["dx"])
         dw1[e] += g["dw1"]
         dw2[e] += g["dw2"]
+        dw1_abs[e] += g["dw1_abs"]
+        dw2_abs[e] += g["dw2_abs"]
         if db1 is not None:
             db1[e] += g["db1"]
+            db1_abs[e] += g["db1_abs"]
         if db2 is not None:
             db2[e] += g["db2"]
-    dsh_w1 = dsh_w2 = None
+    dsh_w1 = dsh_w2 = dsh_w1_abs = dsh_w2_abs = None
     if cfg.get("I_sh"):
         gs = expert_ffn_backward(x, "swiglu", inp["sh_w1"], inp["sh_w2"], None, None, dy)
         dx += gs["dx"]
         dsh_w1, dsh_w2 = gs["dw1"], gs["dw2"]
+        dsh_w1_abs, dsh_w2_abs = gs["dw1_abs"], gs["dw2_abs"]
     dl = router_backward(r["idx"], dw, r["logits"], r["g"], cfg["gate"], cfg["norm_topk_prob"],
                          cfg["alpha"], cfg["eps"])
     w_r = _f64(inp["w_r"])
     dx += dl @ w_r.T                                   # logits = x W_r
     dw_r = x.T @ dl
     return {"dx": dx, "dw_r": dw_r, "dw1": dw1, "dw2": dw2, "db1": db1, "db2": db2,
-            "dsh_w1": dsh_w1, "dsh_w2": dsh_w2, "dw": dw, "dl": dl, "idx": r["idx"], "w": r["w"]}
+            "dsh_w1": dsh_w1, "dsh_w2": dsh_w2, "dw": dw, "dl": dl, "idx": r["idx"], "w": r["w"],
+            "dw1_abs": dw1_abs, "dw2_abs": dw2_abs, "db1_abs": db1_abs, "dsh_w1_abs": dsh_w1_abs,
+            "dsh_w2_abs": dsh_w2_abs}
 
 
 def dense_layer_backward(x, act, w1, w2, b1, b2, dy):

@@ -100,16 +100,21 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 // Waits for the phase of parity `parity` of mbarrier `bar` to complete.
 // Gives up (returns false) when *abort becomes non-zero or after limit_ns
 // (kWaitTimeoutNs unless given), in which case it records the timeout and
-// raises *abort.
+// raises *abort.  The clock is first read only after 32 unsuccessful polls:
+// a %globaltimer read costs hundreds of cycles, and a wait that ends soon
+// (the common case inside a pipeline) must not pay for it.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           int* status, uint64_t limit_ns = kWaitTimeoutNs) {
   if (mbar_test_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  uint64_t t0 = 0;
   for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((n & 31u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > limit_ns) {
         *abort = 1;
         set_status(status, MOE_DEVERR_TIMEOUT);
         return false;

@@ -122,7 +122,7 @@ cudaError_t launch_gemm_swap(const SwapLaunch& L, cudaStream_t s) {
   a.out2 = static_cast<__nv_bfloat16*>(L.out2);
   a.out3 = static_cast<__nv_bfloat16*>(L.out3);
   a.ldo2 = L.ldo2;
-  a.aux = static_cast<const __nv_bfloat16*>(L.aux);
+  a.aux = static_cast<const float*>(L.aux);
   a.ld_aux = L.ld_aux;
   a.parts = L.parts;
   a.ld_parts = L.ld_parts;

@@ -92,14 +92,15 @@ struct SwapArgs {
   int b_tiles;
   int b_cols;
   long long out_gstride;
-  // backward epilogues: second and third bf16 outputs [rows, ldo2] (SAVE),
-  // the saved pre-activations aux [rows, ld_aux] and the per-32-column partial
-  // dot products parts [rows, ld_parts] (DACT), and I, the offset of the up
-  // half in the SwiGLU outputs.
+  // backward epilogues: the saved fp32 pre-activations (out of SAVE, aux
+  // [rows, ld_aux] of DACT), the second and third bf16 outputs [rows, ldo2]
+  // (SAVE: a and w a), the per-32-column partial dot products parts
+  // [rows, ld_parts] (DACT), and I, the offset of the up half in the SwiGLU
+  // outputs.
   __nv_bfloat16* out2;
   __nv_bfloat16* out3;
   int ldo2;
-  const __nv_bfloat16* aux;
+  const float* aux;
   int ld_aux;
   float* parts;
   int ld_parts;
@@ -485,7 +486,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
               for (int i = 0; i < 32; ++i) u[i] = xs[lane * kSwXPitch + i];
               mbar_arrive(smem_addr(&s_xempty[pair]));
-              __nv_bfloat16* hp = static_cast<__nv_bfloat16*>(args.out);
+              float* hp = static_cast<float*>(args.out);
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
                 const float g = __uint_as_float(r[i]);
@@ -493,8 +494,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const float w = __shfl_sync(0xffffffffu, rs, i);
                 if (col_ok && i < nv) {
                   const size_t row = row0 + c + i;
-                  hp[row * args.ldo + col] = __float2bfloat16_rn(g);
-                  hp[row * args.ldo + args.half_cols + col] = __float2bfloat16_rn(u[i]);
+                  hp[row * args.ldo + col] = g;
+                  hp[row * args.ldo + args.half_cols + col] = u[i];
                   args.out2[row * args.ldo2 + col] = __float2bfloat16_rn(a);
                   if (args.out3 != nullptr) args.out3[row * args.ldo2 + col] = __float2bfloat16_rn(w * a);
                 }
@@ -515,12 +516,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (col_ok && i < nv) {
               const size_t row = row0 + c + i;
               if constexpr (EPI == EPI_BWD_GELU_DACT) {
-                const float h = __bfloat162float(args.aux[row * args.ld_aux + col]);
+                const float h = args.aux[row * args.ld_aux + col];
                 dh[row * args.ldo + col] = __float2bfloat16_rn(w * G * gelu_tanh_grad_fast(h));
                 prod[i] = G * gelu_tanh_fast(h);
               } else {
-                const float g = __bfloat162float(args.aux[row * args.ld_aux + col]);
-                const float u = __bfloat162float(args.aux[row * args.ld_aux + args.half_cols + col]);
+                const float g = args.aux[row * args.ld_aux + col];
+                const float u = args.aux[row * args.ld_aux + args.half_cols + col];
                 const float sg = __fdividef(1.0f, 1.0f + __expf(-g));
                 const float si = g * sg;
                 const float da = w * G;
@@ -549,7 +550,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               const float w = __shfl_sync(0xffffffffu, rs, i);
               if (col_ok && i < nv) {
                 const size_t row = row0 + c + i;
-                static_cast<__nv_bfloat16*>(args.out)[row * args.ldo + col] = __float2bfloat16_rn(v);
+                static_cast<float*>(args.out)[row * args.ldo + col] = v;
                 args.out2[row * args.ldo2 + col] = __float2bfloat16_rn(a);
                 if (args.out3 != nullptr) args.out3[row * args.ldo2 + col] = __float2bfloat16_rn(w * a);
               }

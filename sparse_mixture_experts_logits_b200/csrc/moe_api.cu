@@ -897,7 +897,7 @@ BwdWs backward_layout_tc(const moe_layer_desc_t* d) {
   L.rwp = c.take(P * 4);
   L.xpp = c.take(P * D * 2);
   L.dypp = c.take(P * D * 2);
-  L.hpb = c.take(P * n1 * 2);
+  L.hpb = c.take(P * n1 * 4);  // fp32 pre-activations: they feed act' and <G, a> unrounded
   L.ab = c.take(P * Ha * 2);
   L.awb = c.take(P * Ha * 2);
   L.dhb = c.take(P * n1 * 2);
@@ -905,7 +905,7 @@ BwdWs backward_layout_tc(const moe_layer_desc_t* d) {
   L.parts = c.take(P * ((Ha + 31) / 32) * 4);
   L.dwp = c.take(pairs * 4);
   L.dl = c.take(T * d->M * 4);
-  L.hsb = c.take(T * 2 * Is * 2);
+  L.hsb = c.take(T * 2 * Is * 4);
   L.asb = c.take(T * Is * 2);
   L.dhsb = c.take(T * 2 * Is * 2);
   L.dxs = c.take(T * D * 4);
@@ -1001,7 +1001,7 @@ SwapLaunch bwd_swap(int epi, int layout, const void* A, long long a_rows, const 
 
 // The backward of a bf16 layer on the tensor cores.  Per expert segment
 // (rows r of the padded dispatch order, token t(r), gate weight w_r):
-//   recompute  h = x W1^T (+ b1), a = act(h), aw = w a         (save epilogue)
+//   recompute  h = x W1^T (+ b1) (fp32), a = act(h), aw = w a   (save epilogue)
 //   dgrad      G = dy W2;  dh = w G act'(h);  parts = <G, a>   (fused epilogue)
 //              dx_rows = dh W1                                  (fp32)
 //   wgrad      dW2 = dy^T aw,  dW1 = dh^T x  over the segment   (grouped-K GEMMs)
@@ -1064,7 +1064,7 @@ moe_status_t backward_tc_impl(const moe_layer_desc_t* d, const moe_weights_t* w,
   }
   {
     Range r("moe.experts_backward");
-    // recompute: h (bf16), a = act(h), aw = w a
+    // recompute: h (fp32), a = act(h) and aw = w a (bf16 operands of the weight gradients)
     SwapLaunch ga{};
     if (swiglu) {
       ga = bwd_swap(EPI_BWD_SWIGLU_SAVE, kSwFwd, w->w1, 1ll * M * n1, xpp, P, D, M, offp, counts, P, Ha, hpb, n1,

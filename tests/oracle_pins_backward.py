@@ -176,8 +176,55 @@ def pin_single_choice_sigmoid_router(B):
     assert np.abs(g["dw"]).max() > 1e-3
 
 
+def pin_absolute_term_sums(B):
+    """The absolute-term sums of the weight gradients (the scale of their
+    rounding error), by a brute-force loop over the rows of each expert:
+    dw1_abs[n, d] = sum_r |dpre[r, n]| |x[r, d]|, dw2_abs[d, i] =
+    sum_r |dout[r, d]| |a[r, i]|, db1_abs[n] = sum_r |dpre[r, n]|, with
+    dpre = dL/d(pre-activation) and dout the expert's upstream gradient,
+    both from the finite-difference-pinned gradients above; and each sum
+    bounds its gradient: |dw| <= dw_abs elementwise (triangle inequality)."""
+    for cfg in (BWD_TINY[0], BWD_TINY[1]):
+        inp = tiny_inputs(cfg, 140)
+        dy = np.random.default_rng(141).standard_normal((cfg["T"], cfg["D"]))
+        g = B.moe_backward(cfg, inp, dy)
+        for name in ("dw1", "dw2", "db1", "dsh_w1", "dsh_w2"):
+            if g[name] is not None:
+                assert np.all(np.abs(g[name]) <= g[name + "_abs"] + 1e-12), name
+        # brute force of one expert's sums from its own rows
+        e = int(g["idx"][0, 0])
+        tt, jj = np.nonzero(g["idx"] == e)
+        x = np.asarray(inp["x"], np.float64)[tt]
+        w1, w2 = np.asarray(inp["w1"][e], np.float64), np.asarray(inp["w2"][e], np.float64)
+        dout = g["w"][tt, jj][:, None] * dy[tt]
+        pre = x @ w1.T
+        if cfg["act"] == "gelu_tanh":
+            pre = pre + np.asarray(inp["b1"][e], np.float64)
+            a = FWD.gelu_tanh(pre)
+            dpre = (dout @ w2) * B.gelu_tanh_grad(pre)
+        else:
+            I = w1.shape[0] // 2
+            a = FWD.silu(pre[:, :I]) * pre[:, I:]
+            da = dout @ w2
+            dpre = np.concatenate([da * pre[:, I:] * B.silu_grad(pre[:, :I]), da * FWD.silu(pre[:, :I])], axis=1)
+        n1, D = w1.shape
+        bf1 = np.zeros((n1, D))
+        bf2 = np.zeros(w2.shape)
+        for r in range(len(tt)):
+            for n in range(n1):
+                for d in range(D):
+                    bf1[n, d] += abs(dpre[r, n]) * abs(x[r, d])
+            for d in range(w2.shape[0]):
+                for i in range(w2.shape[1]):
+                    bf2[d, i] += abs(dout[r, d]) * abs(a[r, i])
+        assert np.allclose(g["dw1_abs"][e], bf1, rtol=1e-12, atol=1e-14)
+        assert np.allclose(g["dw2_abs"][e], bf2, rtol=1e-12, atol=1e-14)
+        if g["db1_abs"] is not None:
+            assert np.allclose(g["db1_abs"][e], np.abs(dpre).sum(axis=0), rtol=1e-12, atol=1e-14)
+
+
 BWD_PINS = [
     pin_fd_glam, pin_fd_glm_shared, pin_fd_softmax_unnormalised, pin_fd_sigmoid_unnormalised,
     pin_fd_grouped, pin_softmax_shift_invariance, pin_activation_derivatives, pin_expert_load,
-    pin_dense_backward, pin_single_choice_sigmoid_router,
+    pin_dense_backward, pin_single_choice_sigmoid_router, pin_absolute_term_sums,
 ]

@@ -24,6 +24,8 @@ struct BwdArgs {
   int N;
   int accumulate;
   long long m_tiles;  // tiles along the output rows (mode 0: upper bound)
+  int ksplit;         // mode 1 without groups: contraction split into ksplit chunks of kchunk,
+  long long kchunk;   // chunk z written to C + z * c_gstride (partial sums)
 };
 
 __device__ __forceinline__ long long lmin(long long a, long long b) { return a < b ? a : b; }
@@ -70,6 +72,12 @@ __global__ void __launch_bounds__(kBThreads) bwd_gemm_kernel(const BwdArgs p) {
             t -= tiles;
           }
         }
+      } else if (p.ksplit > 1) {
+        g = blockIdx.z;  // the chunk: its partial sums go to C + g * c_gstride
+        row0 = mt * kBM;
+        nrows = static_cast<int>(lmin(kBM, p.rows - row0));
+        kb = lmin(static_cast<long long>(g) * p.kchunk, p.K);
+        ke = lmin(kb + p.kchunk, p.K);
       } else {
         g = blockIdx.z;
         row0 = mt * kBM;
@@ -87,7 +95,7 @@ __global__ void __launch_bounds__(kBThreads) bwd_gemm_kernel(const BwdArgs p) {
     if (g < 0) continue;  // uniform across the block
     const long long row0 = s_row0, kb = s_kb, ke = s_ke;
     const int nrows = s_nrows;
-    const long long b_base = static_cast<long long>(g) * p.b_gstride;
+    const long long b_base = p.ksplit > 1 ? 0 : static_cast<long long>(g) * p.b_gstride;
     float acc[4][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -132,9 +140,20 @@ __global__ void __launch_bounds__(kBThreads) bwd_gemm_kernel(const BwdArgs p) {
         float v = acc[i][j];
         if (bias != nullptr) v += ld(bias, static_cast<long long>(g) * p.bias_gstride + n);
         float* dst = p.C + c_base + (row0 + r) * p.ldc + n;
-        *dst = p.accumulate ? *dst + v : v;
+        *dst = (p.accumulate && p.ksplit <= 1) ? *dst + v : v;
       }
     }
+  }
+}
+
+// C[i] (+)= sum over z of partial[z * n + i], z in order (split-K reduction).
+__global__ void splitk_reduce_kernel(const float* __restrict__ partial, int splits, long long n, float* C,
+                                     int accumulate) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float v = accumulate ? C[i] : 0.f;
+    for (int z = 0; z < splits; ++z) v += partial[z * n + i];
+    C[i] = v;
   }
 }
 
@@ -331,7 +350,31 @@ cudaError_t launch_bwd_gemm(const BwdGemmLaunch& L, cudaStream_t s) {
   a.C = L.C; a.ldc = L.ldc; a.c_gstride = L.c_gstride;
   a.mode = L.mode; a.offsets = L.offsets; a.G = L.offsets ? L.G : 1;
   a.rows = L.rows; a.K = L.K; a.N = L.N; a.accumulate = L.accumulate;
+  a.ksplit = 1; a.kchunk = L.K;
   if (a.rows <= 0 || a.N <= 0) return cudaSuccess;
+  if (L.mode == 1 && L.offsets == nullptr && L.ksplit > 1 && L.partial != nullptr && L.ldc == L.N) {
+    // one contraction cut into chunks whose partial sums are added in order
+    a.ksplit = L.ksplit;
+    a.kchunk = (L.K + L.ksplit - 1) / L.ksplit;
+    a.kchunk = (a.kchunk + kBK - 1) / kBK * kBK;
+    a.C = L.partial;
+    a.c_gstride = a.rows * L.ldc;
+    a.G = L.ksplit;
+    a.accumulate = 0;
+    a.m_tiles = (a.rows + kBM - 1) / kBM;
+    dim3 grid((a.N + kBN - 1) / kBN, static_cast<unsigned>(std::min<long long>(a.m_tiles, 65535)), a.ksplit);
+    if (L.a_bf16 && !L.b_bf16)
+      bwd_gemm_kernel<__nv_bfloat16, float><<<grid, kBThreads, 0, s>>>(a);
+    else if (L.a_bf16)
+      bwd_gemm_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, kBThreads, 0, s>>>(a);
+    else if (L.b_bf16)
+      bwd_gemm_kernel<float, __nv_bfloat16><<<grid, kBThreads, 0, s>>>(a);
+    else
+      bwd_gemm_kernel<float, float><<<grid, kBThreads, 0, s>>>(a);
+    const long long n = a.rows * L.N;
+    splitk_reduce_kernel<<<grid_1d(n, 256), 256, 0, s>>>(L.partial, L.ksplit, n, L.C, L.accumulate);
+    return cudaGetLastError();
+  }
   if (L.mode == 0 && L.offsets != nullptr)
     a.m_tiles = a.rows / kBM + std::min<long long>(a.G, a.rows) + 1;
   else

@@ -84,6 +84,30 @@ cudaError_t launch_swap_epi(const CUtensorMap& tw, const CUtensorMap& tx, const 
   return cudaLaunchKernelEx(&cfg, kernel, tw, tx, args);
 }
 
+// Row-grouped layouts: the forward and the input gradients.
+cudaError_t launch_swap_rows(int layout, int epi, const CUtensorMap& tw, const CUtensorMap& tx, const SwapArgs& a,
+                             long long tiles_ub, cudaStream_t s) {
+  if (layout == kSwDgrad) {
+    switch (epi) {
+      case EPI_STORE_F32: return launch_swap_epi<EPI_STORE_F32, kSwDgrad>(tw, tx, a, tiles_ub, s);
+      case EPI_BWD_GELU_DACT: return launch_swap_epi<EPI_BWD_GELU_DACT, kSwDgrad>(tw, tx, a, tiles_ub, s);
+      case EPI_BWD_SWIGLU_DACT: return launch_swap_epi<EPI_BWD_SWIGLU_DACT, kSwDgrad>(tw, tx, a, tiles_ub, s);
+    }
+    return cudaErrorInvalidValue;
+  }
+  switch (epi) {
+    case EPI_BWD_GELU_SAVE: return launch_swap_epi<EPI_BWD_GELU_SAVE>(tw, tx, a, tiles_ub, s);
+    case EPI_BWD_SWIGLU_SAVE: return launch_swap_epi<EPI_BWD_SWIGLU_SAVE>(tw, tx, a, tiles_ub, s);
+    case EPI_GELU_BIAS: return launch_swap_epi<EPI_GELU_BIAS>(tw, tx, a, tiles_ub, s);
+    case EPI_SWIGLU: return launch_swap_epi<EPI_SWIGLU>(tw, tx, a, tiles_ub, s);
+    case EPI_SCALE_BIAS: return launch_swap_epi<EPI_SCALE_BIAS>(tw, tx, a, tiles_ub, s);
+    case EPI_STORE_F32: return launch_swap_epi<EPI_STORE_F32>(tw, tx, a, tiles_ub, s);
+    case EPI_STORE_BF16: return launch_swap_epi<EPI_STORE_BF16>(tw, tx, a, tiles_ub, s);
+    case EPI_BIAS_ADD: return launch_swap_epi<EPI_BIAS_ADD>(tw, tx, a, tiles_ub, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
 }  // namespace
 
 cudaError_t launch_gemm_swap(const SwapLaunch& L, cudaStream_t s) {
@@ -137,25 +161,7 @@ cudaError_t launch_gemm_swap(const SwapLaunch& L, cudaStream_t s) {
   const long long tt_ub = L.offsets ? L.rows / kSwMaxTile + std::min<long long>(L.num_groups, L.rows)
                                     : (L.rows + kSwMaxTile - 1) / kSwMaxTile;
   const long long tiles_ub = tt_ub * L.w_tiles;
-  if (L.layout == kSwDgrad) {
-    switch (L.epi) {
-      case EPI_STORE_F32: return launch_swap_epi<EPI_STORE_F32, kSwDgrad>(tw, tx, a, tiles_ub, s);
-      case EPI_BWD_GELU_DACT: return launch_swap_epi<EPI_BWD_GELU_DACT, kSwDgrad>(tw, tx, a, tiles_ub, s);
-      case EPI_BWD_SWIGLU_DACT: return launch_swap_epi<EPI_BWD_SWIGLU_DACT, kSwDgrad>(tw, tx, a, tiles_ub, s);
-    }
-    return cudaErrorInvalidValue;
-  }
-  switch (L.epi) {
-    case EPI_BWD_GELU_SAVE: return launch_swap_epi<EPI_BWD_GELU_SAVE>(tw, tx, a, tiles_ub, s);
-    case EPI_BWD_SWIGLU_SAVE: return launch_swap_epi<EPI_BWD_SWIGLU_SAVE>(tw, tx, a, tiles_ub, s);
-    case EPI_GELU_BIAS: return launch_swap_epi<EPI_GELU_BIAS>(tw, tx, a, tiles_ub, s);
-    case EPI_SWIGLU: return launch_swap_epi<EPI_SWIGLU>(tw, tx, a, tiles_ub, s);
-    case EPI_SCALE_BIAS: return launch_swap_epi<EPI_SCALE_BIAS>(tw, tx, a, tiles_ub, s);
-    case EPI_STORE_F32: return launch_swap_epi<EPI_STORE_F32>(tw, tx, a, tiles_ub, s);
-    case EPI_STORE_BF16: return launch_swap_epi<EPI_STORE_BF16>(tw, tx, a, tiles_ub, s);
-    case EPI_BIAS_ADD: return launch_swap_epi<EPI_BIAS_ADD>(tw, tx, a, tiles_ub, s);
-  }
-  return cudaErrorInvalidValue;
+  return launch_swap_rows(L.layout, L.epi, tw, tx, a, tiles_ub, s);
 }
 
 }  // namespace moe

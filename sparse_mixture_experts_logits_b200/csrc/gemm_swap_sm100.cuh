@@ -189,14 +189,15 @@ __device__ __forceinline__ void swap_store(const SwapArgs& a, size_t base, int c
     static_cast<__nv_bfloat16*>(a.out)[base + row * a.ldo + col] = __float2bfloat16_rn(v);
 }
 
-// d/dv of the GELU tanh form 0.5 v (1 + tanh(u)), u = c (v + 0.044715 v^3):
-// 0.5 (1 + tanh u) + 0.5 v (1 - tanh^2 u) c (1 + 3 * 0.044715 v^2), with
-// tanh u = 1 - 2 / (1 + e^{2u}).
-__device__ __forceinline__ float gelu_tanh_grad_fast(float v) {
+// GELU (tanh form) and its derivative from one exponential: with
+// s = 0.5 (1 + tanh u) = 1 / (1 + e^{-2u}), GELU(v) = v s and GELU'(v) =
+// s + v 2 s (1 - s) c (1 + 3 * 0.044715 v^2), since 1 - tanh^2 u = 4 s (1 - s).
+__device__ __forceinline__ void gelu_tanh_and_grad_fast(float v, float& g, float& dg) {
   const float c = 0.7978845608028654f;
   const float u = c * fmaf(0.044715f * v, v * v, v);
-  const float th = 1.0f - __fdividef(2.0f, 1.0f + __expf(2.0f * u));
-  return 0.5f * (1.0f + th) + 0.5f * v * (1.0f - th * th) * c * fmaf(3.0f * 0.044715f, v * v, 1.0f);
+  const float sg = __fdividef(1.0f, 1.0f + __expf(-2.0f * u));
+  g = v * sg;
+  dg = fmaf(v * 2.0f * sg * (1.0f - sg) * c, fmaf(3.0f * 0.044715f, v * v, 1.0f), sg);
 }
 
 // Sum over the warp's 32 lanes of v[i] for every i, in 31 shuffles: after
@@ -267,8 +268,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int carry = 0;
     for (int base = 0; base < G; base += 32) {
       const int g = base + lane;
-      int v = 0;
-      if (g < G) v = swap_group_tiles<LAYOUT>(s_cnt[g], args);
+      const int v = g < G ? swap_group_tiles<LAYOUT>(s_cnt[g], args) : 0;
       int incl = v;
 #pragma unroll
       for (int d = 1; d < 32; d <<= 1) {
@@ -425,8 +425,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int m = q * 32 + lane;      // accumulator lane = weight row inside this CTA
     const uint32_t tempty0 = mapa_shared(smem_addr(&s_tempty[0]), 0);
     const uint32_t tempty1 = mapa_shared(smem_addr(&s_tempty[1]), 0);
-    const int pair = part * 2 + (q & 1);          // SwiGLU hand-off pair (gate q, up q + 2)
-    float* xs = xbuf + pair * 32 * kSwXPitch;
+    const int xpair = part * 2 + (q & 1);         // SwiGLU hand-off pair (gate q, up q + 2)
+    float* xs = xbuf + xpair * 32 * kSwXPitch;
     const bool up_warp = kSwiglu && q >= 2;
     uint32_t it = 0, xc = 0;
     bool ok = true;
@@ -454,7 +454,44 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       constexpr bool kScaled = EPI == EPI_SCALE_BIAS || EPI == EPI_BWD_GELU_SAVE ||
                                EPI == EPI_BWD_SWIGLU_SAVE || EPI == EPI_BWD_GELU_DACT ||
                                EPI == EPI_BWD_SWIGLU_DACT;
+      constexpr bool kDact = EPI == EPI_BWD_GELU_DACT || EPI == EPI_BWD_SWIGLU_DACT;
+      if constexpr (LAYOUT == kSwWgrad) {
+        // Weight gradients: short contractions, so the epilogue (fp32 stores
+        // of a 256 x 256 tile) is the critical path.  The warp's four chunks
+        // (N = 256) are read from TMEM two at a time, one wait per pair.
+#pragma unroll 1
+        for (int j0 = 0; j0 < 4; j0 += 2) {
+          uint32_t r2[2][32];
+          MOE_TMEM_LD32(tacc + 32 * part + 64 * j0, r2[0]);
+          MOE_TMEM_LD32(tacc + 32 * part + 64 * (j0 + 1), r2[1]);
+          tmem_ld_wait();
+          if (col_ok) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int c = 32 * part + 64 * (j0 + j);
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (c + i < t.nrows) swap_store<EPI>(args, gofs, col, __uint_as_float(r2[j][i]), row0 + c + i);
+            }
+          }
+        }
+      } else
       for (int c = 32 * part; c < t.n; c += 64) {
+        // input-gradient epilogues: the chunk's saved pre-activations are
+        // requested first, so that their memory latency overlaps the TMEM read
+        // and each other's
+        float hv[32], uv[32];
+        if constexpr (kDact) {
+          const int nvd = min(32, t.nrows - c);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const bool live = col_ok && i < nvd;
+            const size_t row = row0 + c + i;
+            hv[i] = live ? args.aux[row * args.ld_aux + col] : 0.f;
+            if constexpr (EPI == EPI_BWD_SWIGLU_DACT)
+              uv[i] = live ? args.aux[row * args.ld_aux + args.half_cols + col] : 0.f;
+          }
+        }
         uint32_t r[32];
         MOE_TMEM_LD32(tacc + c, r);
         tmem_ld_wait();
@@ -465,17 +502,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if constexpr (kSwiglu) {
           if (up_warp) {
-            if (!mbar_wait(smem_addr(&s_xempty[pair]), (xc & 1u) ^ 1u, abort_flag, args.status)) { ok = false; break; }
+            if (!mbar_wait(smem_addr(&s_xempty[xpair]), (xc & 1u) ^ 1u, abort_flag, args.status)) { ok = false; break; }
 #pragma unroll
             for (int i = 0; i < 32; ++i) xs[lane * kSwXPitch + i] = __uint_as_float(r[i]);
-            mbar_arrive(smem_addr(&s_xfull[pair]));
+            mbar_arrive(smem_addr(&s_xfull[xpair]));
           } else {
-            if (!mbar_wait(smem_addr(&s_xfull[pair]), xc & 1u, abort_flag, args.status)) { ok = false; break; }
+            if (!mbar_wait(smem_addr(&s_xfull[xpair]), xc & 1u, abort_flag, args.status)) { ok = false; break; }
             if constexpr (EPI == EPI_SWIGLU) {
               float v[32];
 #pragma unroll
               for (int i = 0; i < 32; ++i) v[i] = silu_fast(__uint_as_float(r[i])) * xs[lane * kSwXPitch + i];
-              mbar_arrive(smem_addr(&s_xempty[pair]));
+              mbar_arrive(smem_addr(&s_xempty[xpair]));
               if (col_ok) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
@@ -485,7 +522,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               float u[32];
 #pragma unroll
               for (int i = 0; i < 32; ++i) u[i] = xs[lane * kSwXPitch + i];
-              mbar_arrive(smem_addr(&s_xempty[pair]));
+              mbar_arrive(smem_addr(&s_xempty[xpair]));
               float* hp = static_cast<float*>(args.out);
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
@@ -516,12 +553,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (col_ok && i < nv) {
               const size_t row = row0 + c + i;
               if constexpr (EPI == EPI_BWD_GELU_DACT) {
-                const float h = args.aux[row * args.ld_aux + col];
-                dh[row * args.ldo + col] = __float2bfloat16_rn(w * G * gelu_tanh_grad_fast(h));
-                prod[i] = G * gelu_tanh_fast(h);
+                float a, da_dh;
+                gelu_tanh_and_grad_fast(hv[i], a, da_dh);
+                dh[row * args.ldo + col] = __float2bfloat16_rn(w * G * da_dh);
+                prod[i] = G * a;
               } else {
-                const float g = args.aux[row * args.ld_aux + col];
-                const float u = args.aux[row * args.ld_aux + args.half_cols + col];
+                const float g = hv[i], u = uv[i];
                 const float sg = __fdividef(1.0f, 1.0f + __expf(-g));
                 const float si = g * sg;
                 const float da = w * G;

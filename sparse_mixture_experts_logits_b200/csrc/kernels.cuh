@@ -154,6 +154,10 @@ struct BwdGemmLaunch {
   long long rows, K;
   int N;
   int accumulate;
+  // mode 1 without groups: split the contraction into ksplit chunks whose
+  // partial sums ([ksplit, rows, N] in `partial`) are added in order (ldc == N)
+  int ksplit;
+  float* partial;
 };
 cudaError_t launch_bwd_gemm(const BwdGemmLaunch& L, cudaStream_t s);
 // a = GELU(h) or SiLU(gate) * up for rows < min(rows, *n_rows) (n_rows may be null).

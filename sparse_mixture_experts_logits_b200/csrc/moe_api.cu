@@ -872,8 +872,12 @@ struct BwdWs {
   size_t xp, hpre, act, dO, da, dxp, dwp, dl, hs, as, das, dxs, total;
   // tensor-core path (bf16): the padded dispatch order and its bf16 tensors
   long long rows_pad;
-  size_t offp, slotp, rtp, rwp, xpp, dypp, hpb, ab, awb, dhb, dxpp, parts, hsb, asb, dhsb;
+  size_t offp, slotp, rtp, rwp, xpp, dypp, hpb, ab, awb, dhb, dxpp, parts, hsb, asb, dhsb, rpart;
 };
+
+// Chunks of the token sum in the router's weight gradient dW_r = x^T dlogits
+// (partial sums added in order): enough blocks to fill the GPU.
+int router_ksplit(int T) { return std::max(1, std::min(16, T / 1024)); }
 
 // Rows of the backward's padded dispatch order: every expert's segment is
 // rounded up to 64 rows, so at most T k + 63 M rows.
@@ -909,6 +913,7 @@ BwdWs backward_layout_tc(const moe_layer_desc_t* d) {
   L.asb = c.take(T * Is * 2);
   L.dhsb = c.take(T * 2 * Is * 2);
   L.dxs = c.take(T * D * 4);
+  L.rpart = c.take(static_cast<size_t>(router_ksplit(d->T)) * D * d->M * 4);
   L.total = c.off;
   return L;
 }
@@ -1169,6 +1174,8 @@ moe_status_t backward_tc_impl(const moe_layer_desc_t* d, const moe_weights_t* w,
                                d->eps, dl, s));
     BwdGemmLaunch wr = bwd_gemm(x, 1, D, true, dl, 1, M, 0, false, g->dw_r, M, D, T, M);
     wr.mode = 1;
+    wr.ksplit = router_ksplit(T);
+    wr.partial = at<float*>(ws, L.rpart);
     MOE_CUDA(launch_bwd_gemm(wr, s));
     BwdGemmLaunch xr = bwd_gemm(dl, M, 1, false, w->w_r, M, 1, 0, true, dxs, D, T, M, D);
     xr.accumulate = Is > 0 ? 1 : 0;  // onto the shared expert's dx
@@ -1335,6 +1342,7 @@ int moe_backward_launch_count(const moe_layer_desc_t* d) {
     if (d->act == MOE_ACT_GELU_TANH && d->has_bias) n += 2;        // bias gradients
     if (d->I_sh > 0) n += 5;                                         // shared expert GEMMs
     n += 3;                                                          // router backward, dW_r, router dx
+    if (router_ksplit(d->T) > 1) n += 1;                             // dW_r chunk sums
     n += 1;                                                          // dx combine
     return n;
   }

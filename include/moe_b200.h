@@ -32,6 +32,11 @@
  *  - dtype MOE_DTYPE_BF16: x, W_r, expert/shared weights, biases, y are
  *    bf16; all accumulation is fp32.  MOE_DTYPE_F32: all of them are fp32.
  *    e_bias, topk_w and row_w are always fp32; indices are int32.
+ *  - MOE_DTYPE_BF16 tensors that the tensor-core kernels move with TMA start
+ *    on a 16-byte boundary: x, W_r, the routed and shared weight stacks, and
+ *    in moe_backward also dy and the fp32 weight gradients dw1, dw2, dsh_w1,
+ *    dsh_w2 (cudaMalloc and PyTorch allocations are).  A misaligned one is
+ *    MOE_ERR_INVALID_ARG, found before anything is launched.
  *  - Errors: every call validates its arguments on the host and returns a
  *    status without launching anything when they are invalid.  Device-side
  *    faults are never raised: kernels that find an out-of-range expert index

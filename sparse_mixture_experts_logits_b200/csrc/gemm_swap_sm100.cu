@@ -39,9 +39,24 @@ bool tmap_bf16(CUtensorMap* map, const void* base, long long rows, int cols, int
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 [groups][rows][cols] with row pitch `ld` and group pitch `gstride`
+// elements, 32 x 32 x 1 boxes, no swizzle: the weight-gradient output.
+bool tmap_f32_out(CUtensorMap* map, void* base, int cols, long long rows, int groups, long long ld,
+                  long long gstride) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(groups)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld) * 4, static_cast<cuuint64_t>(gstride) * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int EPI, int LAYOUT = kSwFwd>
-cudaError_t launch_swap_epi(const CUtensorMap& tw, const CUtensorMap& tx, const SwapArgs& args,
-                            long long tiles_ub, cudaStream_t s) {
+cudaError_t launch_swap_epi(const SwapMaps& maps, const SwapArgs& args, long long tiles_ub, cudaStream_t s) {
   static std::atomic<unsigned> configured{0};
   static std::atomic<int> max_clusters[32];
   int dev = 0;
@@ -81,29 +96,29 @@ cudaError_t launch_swap_epi(const CUtensorMap& tw, const CUtensorMap& tx, const 
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, tw, tx, args);
+  return cudaLaunchKernelEx(&cfg, kernel, maps, args);
 }
 
 // Row-grouped layouts: the forward and the input gradients.
-cudaError_t launch_swap_rows(int layout, int epi, const CUtensorMap& tw, const CUtensorMap& tx, const SwapArgs& a,
-                             long long tiles_ub, cudaStream_t s) {
+cudaError_t launch_swap_rows(int layout, int epi, const SwapMaps& m, const SwapArgs& a, long long tiles_ub,
+                             cudaStream_t s) {
   if (layout == kSwDgrad) {
     switch (epi) {
-      case EPI_STORE_F32: return launch_swap_epi<EPI_STORE_F32, kSwDgrad>(tw, tx, a, tiles_ub, s);
-      case EPI_BWD_GELU_DACT: return launch_swap_epi<EPI_BWD_GELU_DACT, kSwDgrad>(tw, tx, a, tiles_ub, s);
-      case EPI_BWD_SWIGLU_DACT: return launch_swap_epi<EPI_BWD_SWIGLU_DACT, kSwDgrad>(tw, tx, a, tiles_ub, s);
+      case EPI_STORE_F32: return launch_swap_epi<EPI_STORE_F32, kSwDgrad>(m, a, tiles_ub, s);
+      case EPI_BWD_GELU_DACT: return launch_swap_epi<EPI_BWD_GELU_DACT, kSwDgrad>(m, a, tiles_ub, s);
+      case EPI_BWD_SWIGLU_DACT: return launch_swap_epi<EPI_BWD_SWIGLU_DACT, kSwDgrad>(m, a, tiles_ub, s);
     }
     return cudaErrorInvalidValue;
   }
   switch (epi) {
-    case EPI_BWD_GELU_SAVE: return launch_swap_epi<EPI_BWD_GELU_SAVE>(tw, tx, a, tiles_ub, s);
-    case EPI_BWD_SWIGLU_SAVE: return launch_swap_epi<EPI_BWD_SWIGLU_SAVE>(tw, tx, a, tiles_ub, s);
-    case EPI_GELU_BIAS: return launch_swap_epi<EPI_GELU_BIAS>(tw, tx, a, tiles_ub, s);
-    case EPI_SWIGLU: return launch_swap_epi<EPI_SWIGLU>(tw, tx, a, tiles_ub, s);
-    case EPI_SCALE_BIAS: return launch_swap_epi<EPI_SCALE_BIAS>(tw, tx, a, tiles_ub, s);
-    case EPI_STORE_F32: return launch_swap_epi<EPI_STORE_F32>(tw, tx, a, tiles_ub, s);
-    case EPI_STORE_BF16: return launch_swap_epi<EPI_STORE_BF16>(tw, tx, a, tiles_ub, s);
-    case EPI_BIAS_ADD: return launch_swap_epi<EPI_BIAS_ADD>(tw, tx, a, tiles_ub, s);
+    case EPI_BWD_GELU_SAVE: return launch_swap_epi<EPI_BWD_GELU_SAVE>(m, a, tiles_ub, s);
+    case EPI_BWD_SWIGLU_SAVE: return launch_swap_epi<EPI_BWD_SWIGLU_SAVE>(m, a, tiles_ub, s);
+    case EPI_GELU_BIAS: return launch_swap_epi<EPI_GELU_BIAS>(m, a, tiles_ub, s);
+    case EPI_SWIGLU: return launch_swap_epi<EPI_SWIGLU>(m, a, tiles_ub, s);
+    case EPI_SCALE_BIAS: return launch_swap_epi<EPI_SCALE_BIAS>(m, a, tiles_ub, s);
+    case EPI_STORE_F32: return launch_swap_epi<EPI_STORE_F32>(m, a, tiles_ub, s);
+    case EPI_STORE_BF16: return launch_swap_epi<EPI_STORE_BF16>(m, a, tiles_ub, s);
+    case EPI_BIAS_ADD: return launch_swap_epi<EPI_BIAS_ADD>(m, a, tiles_ub, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -111,14 +126,18 @@ cudaError_t launch_swap_rows(int layout, int epi, const CUtensorMap& tw, const C
 }  // namespace
 
 cudaError_t launch_gemm_swap(const SwapLaunch& L, cudaStream_t s) {
-  CUtensorMap tw, tx;
+  SwapMaps m = {};
   // A: K-major weight rows, or (backward) an MN-major [rows, a_cols] matrix;
   // B: K-major token rows (128-row boxes), or (weight gradients) MN-major.
   const int a_inner = L.layout == kSwFwd ? L.K : L.a_cols;
-  if (!tmap_bf16(&tw, L.W, L.w_rows, a_inner, 64)) return cudaErrorInvalidValue;
+  if (!tmap_bf16(&m.w, L.W, L.w_rows, a_inner, 64)) return cudaErrorInvalidValue;
   if (L.layout == kSwWgrad) {
-    if (!tmap_bf16(&tx, L.X, L.x_rows, L.b_cols, 64)) return cudaErrorInvalidValue;
-  } else if (!tmap_bf16(&tx, L.X, L.x_rows, L.K, 128)) {
+    if (!tmap_bf16(&m.x, L.X, L.x_rows, L.b_cols, 64)) return cudaErrorInvalidValue;
+    if (L.num_groups > 1 && L.out_gstride < static_cast<long long>(L.b_cols) * L.ldo) return cudaErrorInvalidValue;
+    if (!tmap_f32_out(&m.out, L.out, L.out_cols, L.b_cols, L.num_groups, L.ldo,
+                      L.num_groups > 1 ? L.out_gstride : static_cast<long long>(L.b_cols) * L.ldo))
+      return cudaErrorInvalidValue;
+  } else if (!tmap_bf16(&m.x, L.X, L.x_rows, L.K, 128)) {
     return cudaErrorInvalidValue;
   }
   SwapArgs a = {};
@@ -155,13 +174,13 @@ cudaError_t launch_gemm_swap(const SwapLaunch& L, cudaStream_t s) {
   if (L.layout == kSwWgrad) {
     const long long tiles_ub = static_cast<long long>(L.num_groups) * L.w_tiles * L.b_tiles;
     if (L.epi != EPI_STORE_F32) return cudaErrorInvalidValue;
-    return launch_swap_epi<EPI_STORE_F32, kSwWgrad>(tw, tx, a, tiles_ub, s);
+    return launch_swap_epi<EPI_STORE_F32, kSwWgrad>(m, a, tiles_ub, s);
   }
   // token tiles of a segment: ceil(rows_g / 256) at most, so the total is at most rows/256 + #groups
   const long long tt_ub = L.offsets ? L.rows / kSwMaxTile + std::min<long long>(L.num_groups, L.rows)
                                     : (L.rows + kSwMaxTile - 1) / kSwMaxTile;
   const long long tiles_ub = tt_ub * L.w_tiles;
-  return launch_swap_rows(L.layout, L.epi, tw, tx, a, tiles_ub, s);
+  return launch_swap_rows(L.layout, L.epi, m, a, tiles_ub, s);
 }
 
 }  // namespace moe

@@ -68,6 +68,27 @@ constexpr int kSwDynSmem = kSwStages * kSwStageBytes + kSwXBytes + 1024;
 constexpr int kSwMaxTile = 256;               // tokens per tile
 static_assert(kBK == 64, "the MMA loop issues four K = 16 slices per stage");
 
+// Tensor maps of one launch.  The token operand always moves 128 rows per
+// CTA and k-block, whatever the tile's N: a copy per exact N / 2 rows
+// (boxes of 64, 32, 16 and 8 rows) costs more in TMA instructions than the
+// rows it saves.
+struct SwapMaps {
+  CUtensorMap w;    // A operand
+  CUtensorMap x;    // B operand
+  CUtensorMap out;  // kSwWgrad: fp32 [G][b_cols][out_cols] output, 32 x 32 boxes
+};
+
+// The weight-gradient layout contracts over an expert's rows only (a few
+// k-blocks per tile), so its epilogue, not the MMA, sets the pace.  It runs
+// a 2-stage pipeline and gives the third stage's 64 KB to its eight epilogue
+// warps as two 4 KB store-staging buffers each: every 32 x 32 fp32 chunk
+// leaves through one TMA store instead of 32 warp-wide scalar stores.
+constexpr int kSwWgStages = 2;
+constexpr int kSwWgStageBufBytes = 32 * 32 * 4;
+static_assert(kSwStages > kSwWgStages &&
+                  kGemmThreads / 32 - 2 == 8 && 8 * 2 * kSwWgStageBufBytes <= kSwStageBytes,
+              "the store staging buffers fill the weight-gradient pipeline's unused stage");
+
 struct SwapArgs {
   int num_groups;
   const int* offsets;      // [G + 1] or nullptr: one group [0, rows)
@@ -219,9 +240,8 @@ __device__ __forceinline__ float warp_transpose_sum(float (&v)[32], int lane) {
 
 template <int EPI, int LAYOUT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    moe_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmap_w,
-                         const __grid_constant__ CUtensorMap tmap_x, const SwapArgs args) {
-  constexpr int S = kSwStages;
+    moe_gemm_swap_kernel(const __grid_constant__ SwapMaps maps, const SwapArgs args) {
+  constexpr int S = LAYOUT == kSwWgrad ? kSwWgStages : kSwStages;
   constexpr bool kSwiglu = EPI == EPI_SWIGLU || EPI == EPI_BWD_SWIGLU_SAVE;
   constexpr bool kAMn = LAYOUT != kSwFwd;
   constexpr bool kBMn = LAYOUT == kSwWgrad;
@@ -248,7 +268,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int unit = static_cast<int>(blockIdx.x >> 1);
   const int units = static_cast<int>(gridDim.x >> 1);
   const uint32_t smem_base = (smem_addr(dyn_smem) + 1023u) & ~1023u;
-  float* xbuf = reinterpret_cast<float*>(dyn_smem + (smem_base - smem_addr(dyn_smem)) + S * kSwStageBytes);
+  float* xbuf = reinterpret_cast<float*>(dyn_smem + (smem_base - smem_addr(dyn_smem)) + kSwStages * kSwStageBytes);
   const int G = args.num_groups;
 
   // Segment bounds clamped to [0, rows], so that offsets that are not a
@@ -296,8 +316,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       mbar_init(smem_addr(&s_drain), 1);
       fence_mbar_init();
-      tma_prefetch_desc(&tmap_w);
-      tma_prefetch_desc(&tmap_x);
+      tma_prefetch_desc(&maps.w);
+      tma_prefetch_desc(&maps.x);
+      if constexpr (LAYOUT == kSwWgrad) tma_prefetch_desc(&maps.out);
     }
   } else if (warp == 1) {
     tmem_alloc_pair(smem_addr(&s_tmem_base), 512);
@@ -321,8 +342,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // -------------------------------------------------------- TMA producer
     uint32_t s = 0, ph = 0;
     bool ok = true;
-    // both CTAs' bytes of one k-block: weight rows + 128 token rows each
-    constexpr uint32_t kb_bytes = 2u * (kSwATileBytes + kSwBTileBytes);
     for (int tile = unit; ok && tile < total; tile += units) {
       const SwapTile t = swap_decode<LAYOUT>(tile, G, s_tstart, s_cnt, args, num_kb);
       // kSwFwd / kSwDgrad: B = this CTA's half of the token tile, K-major rows.
@@ -333,6 +352,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int w_base = (LAYOUT == kSwFwd ? t.g * args.w_rows_per_group : 0) + t.wt * args.w_tile_step +
                          static_cast<int>(rank) * args.w_cta_step;
       const int k_row0 = LAYOUT == kSwDgrad ? t.g * args.k_rows_per_group : s_off[t.g];
+      // both CTAs' bytes of one k-block: 128 weight rows + 128 B rows each
+      constexpr uint32_t kb_bytes = 2u * (kSwATileBytes + kSwBTileBytes);
       for (int kb0 = 0; kb0 < t.nkb; kb0 += kSwKB) {
         const int nk = min(kSwKB, t.nkb - kb0);
         if (!mbar_wait_all(smem_addr(&s_empty[s]), ph ^ 1u, abort_flag, args.status)) { ok = false; break; }
@@ -346,18 +367,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t ai = sa + i * kSwATileBytes;
             const uint32_t bi = sb + i * kSwBTileBytes;
             if constexpr (!kAMn) {
-              tma_load_2d_pair(ai, &tmap_w, full_leader, kc, w_base);
-              tma_load_2d_pair(ai + 64 * kBK * 2, &tmap_w, full_leader, kc, w_base + args.w_hi_offset);
+              tma_load_2d_pair(ai, &maps.w, full_leader, kc, w_base);
+              tma_load_2d_pair(ai + 64 * kBK * 2, &maps.w, full_leader, kc, w_base + args.w_hi_offset);
             } else {
               // two boxes of 64 A columns x 64 K rows (8 KB each, 8 KB apart)
-              tma_load_2d_pair(ai, &tmap_w, full_leader, w_base, k_row0 + kc);
-              tma_load_2d_pair(ai + 64 * kBK * 2, &tmap_w, full_leader, w_base + args.w_hi_offset, k_row0 + kc);
+              tma_load_2d_pair(ai, &maps.w, full_leader, w_base, k_row0 + kc);
+              tma_load_2d_pair(ai + 64 * kBK * 2, &maps.w, full_leader, w_base + args.w_hi_offset, k_row0 + kc);
             }
             if constexpr (!kBMn) {
-              tma_load_2d_pair(bi, &tmap_x, full_leader, kc, x_row);
+              tma_load_2d_pair(bi, &maps.x, full_leader, kc, x_row);
             } else {
-              tma_load_2d_pair(bi, &tmap_x, full_leader, b_col, k_row0 + kc);
-              tma_load_2d_pair(bi + 64 * kBK * 2, &tmap_x, full_leader, b_col + 64, k_row0 + kc);
+              tma_load_2d_pair(bi, &maps.x, full_leader, b_col, k_row0 + kc);
+              tma_load_2d_pair(bi + 64 * kBK * 2, &maps.x, full_leader, b_col + 64, k_row0 + kc);
             }
           }
         }
@@ -429,6 +450,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     float* xs = xbuf + xpair * 32 * kSwXPitch;
     const bool up_warp = kSwiglu && q >= 2;
     uint32_t it = 0, xc = 0;
+    uint32_t sc = 0;  // kSwWgrad: chunks this warp has stored (staging buffer sc & 1)
+    const uint32_t stg = smem_base + kSwWgStages * kSwStageBytes + (warp - 2) * 2 * kSwWgStageBufBytes;
+    float* stgp = reinterpret_cast<float*>(dyn_smem + (stg - smem_addr(dyn_smem)));
     bool ok = true;
     for (int tile = unit; ok && tile < total; tile += units, ++it) {
       const SwapTile t = swap_decode<LAYOUT>(tile, G, s_tstart, s_cnt, args, num_kb);
@@ -456,22 +480,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                EPI == EPI_BWD_SWIGLU_DACT;
       constexpr bool kDact = EPI == EPI_BWD_GELU_DACT || EPI == EPI_BWD_SWIGLU_DACT;
       if constexpr (LAYOUT == kSwWgrad) {
-        // Weight gradients: short contractions, so the epilogue (fp32 stores
-        // of a 256 x 256 tile) is the critical path.  The warp's four chunks
-        // (N = 256) are read from TMEM two at a time, one wait per pair.
+        // Weight gradients: the warp's four 32 x 32 chunks (N = 256) are read
+        // from TMEM two at a time, one wait per pair, written to a staging
+        // buffer in the output's own row-major layout (lane = column, so each
+        // row of 32 floats is one conflict-free store) and sent out by one
+        // TMA store per chunk.  The tensor map's extents clip the rows past
+        // b_cols and the columns past out_cols.
+        (void)gofs;
+        (void)row0;
+        const int col0 = col - lane;  // the warp's first output column (a multiple of 32)
 #pragma unroll 1
         for (int j0 = 0; j0 < 4; j0 += 2) {
           uint32_t r2[2][32];
           MOE_TMEM_LD32(tacc + 32 * part + 64 * j0, r2[0]);
           MOE_TMEM_LD32(tacc + 32 * part + 64 * (j0 + 1), r2[1]);
           tmem_ld_wait();
-          if (col_ok) {
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const int c = 32 * part + 64 * (j0 + j);
+          for (int j = 0; j < 2; ++j) {
+            const int c = 32 * part + 64 * (j0 + j);
+            if (col0 < args.out_cols && c < t.nrows) {
+              const uint32_t b = sc & 1u;
+              if (lane == 0) bulk_wait_group_read<1>();  // the store that last used buffer b has read it
+              __syncwarp();
+              float* st = stgp + b * (kSwWgStageBufBytes / 4);
 #pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (c + i < t.nrows) swap_store<EPI>(args, gofs, col, __uint_as_float(r2[j][i]), row0 + c + i);
+              for (int i = 0; i < 32; ++i) st[i * 32 + lane] = __uint_as_float(r2[j][i]);
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_3d(&maps.out, stg + b * kSwWgStageBufBytes, col0, t.tok0 + c, t.g);
+                bulk_commit_group();
+              }
+              ++sc;
             }
           }
         }
@@ -600,6 +640,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!ok) break;
       tc_fence_before();
       mbar_arrive_remote(buf ? tempty1 : tempty0);
+    }
+    if constexpr (LAYOUT == kSwWgrad) {
+      // the staged chunks are read and written before shared memory is released
+      if (lane == 0) bulk_wait_group<0>();
+      __syncwarp();
     }
   }
 

@@ -60,6 +60,9 @@ inline moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_O
 #define MOE_CUDA(expr) MOE_TRY(cuda_status(expr))
 
 bool aligned_ws(const void* ws) { return (reinterpret_cast<uintptr_t>(ws) % kAlign) == 0; }
+// bf16 tensors that the tensor-core kernels move with TMA, and the fp32
+// weight gradients they store with it, start on a 16-byte boundary.
+bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 moe_status_t check_router_args(int T, int D, int M, int k, int dtype, int gate) {
   if (T < 0 || D < 1 || M < 1 || k < 1) return MOE_ERR_INVALID_ARG;
@@ -106,6 +109,10 @@ moe_status_t check_weights(const moe_layer_desc_t* d, const moe_weights_t* w, bo
       return MOE_ERR_INVALID_ARG;
   }
   if (shared && d->I_sh > 0 && (w->sh_w1 == nullptr || w->sh_w2 == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (d->dtype == MOE_DTYPE_BF16) {
+    if (routed && (!al16(w->w1) || !al16(w->w2))) return MOE_ERR_INVALID_ARG;
+    if (shared && d->I_sh > 0 && (!al16(w->sh_w1) || !al16(w->sh_w2))) return MOE_ERR_INVALID_ARG;
+  }
   return MOE_OK;
 }
 
@@ -468,6 +475,7 @@ moe_status_t moe_route_topk(const void* x, const void* w_r, const float* e_bias,
   if (!(eps >= 0.0f)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   if (!x || !w_r || !topk_idx || !topk_w || !ws || !aligned_ws(ws)) return MOE_ERR_INVALID_ARG;
+  if (dtype == MOE_DTYPE_BF16 && (!al16(x) || !al16(w_r))) return MOE_ERR_INVALID_ARG;
   const RouteWs L = route_layout(T, D, M, dtype);
   if (ws_bytes < L.total) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_device());
@@ -548,6 +556,7 @@ moe_status_t moe_expert_ffn(const moe_layer_desc_t* d, const moe_weights_t* w, c
   if (d->T == 0) return MOE_OK;
   if (!x || !offsets || !row_token || !row_w || !out_perm || !ws || !aligned_ws(ws))
     return MOE_ERR_INVALID_ARG;
+  if (d->dtype == MOE_DTYPE_BF16 && !al16(x)) return MOE_ERR_INVALID_ARG;
   const FfnWs L = ffn_layout(d);
   if (ws_bytes < L.total) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_device());
@@ -570,6 +579,7 @@ moe_status_t moe_shared_expert(const moe_layer_desc_t* d, const moe_weights_t* w
   MOE_TRY(check_weights(d, w, false, true));
   if (d->T == 0) return MOE_OK;
   if (!x || !y_sh || !ws || !aligned_ws(ws)) return MOE_ERR_INVALID_ARG;
+  if (d->dtype == MOE_DTYPE_BF16 && !al16(x)) return MOE_ERR_INVALID_ARG;
   const SharedWs L = shared_layout(d);
   if (ws_bytes < L.total) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_device());
@@ -627,6 +637,7 @@ moe_status_t dense_impl(const moe_dense_desc_t* d, const void* w1, const void* b
   const bool bias = !swiglu && d->has_bias;
   if (!w1 || !w2 || !x || !y || !ws || !aligned_ws(ws)) return MOE_ERR_INVALID_ARG;
   if (bias && (!b1 || !b2)) return MOE_ERR_INVALID_ARG;
+  if (d->dtype == MOE_DTYPE_BF16 && (!al16(x) || !al16(w1) || !al16(w2))) return MOE_ERR_INVALID_ARG;
   const DenseWs L = dense_layout(d);
   if (ws_bytes < L.total) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_device());
@@ -746,6 +757,7 @@ static moe_status_t forward_impl(const moe_layer_desc_t* d, const moe_weights_t*
   if (w->w_r == nullptr) return MOE_ERR_INVALID_ARG;
   if (d->T == 0) return MOE_OK;
   if (!x || !y || !ws || !aligned_ws(ws)) return MOE_ERR_INVALID_ARG;
+  if (d->dtype == MOE_DTYPE_BF16 && (!al16(x) || !al16(w->w_r))) return MOE_ERR_INVALID_ARG;
   const FwdWs L = forward_layout(d);
   if (ws_bytes < L.pub.total) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_device());
@@ -1206,6 +1218,10 @@ moe_status_t backward_impl(const moe_layer_desc_t* d, const moe_weights_t* w, co
     return zero_param_grads(d, g, s);
   }
   if (!x || !dy || !g->dx || !ws || !aligned_ws(ws)) return MOE_ERR_INVALID_ARG;
+  if (d->dtype == MOE_DTYPE_BF16) {
+    if (!al16(x) || !al16(dy) || !al16(w->w_r) || !al16(g->dw1) || !al16(g->dw2)) return MOE_ERR_INVALID_ARG;
+    if (d->I_sh > 0 && (!al16(g->dsh_w1) || !al16(g->dsh_w2))) return MOE_ERR_INVALID_ARG;
+  }
   const BwdWs L = backward_layout(d);
   if (ws_bytes < L.total) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_device());

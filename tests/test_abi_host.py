@@ -207,6 +207,38 @@ def test_backward_host_checks(B):
     assert B.moe_backward_workspace_size(bad) == 0 and B.moe_backward_launch_count(bad) == 0
 
 
+def test_bf16_tma_operands_must_be_16_byte_aligned(B):
+    """bf16 tensors the TMA kernels read, and the fp32 weight gradients they
+    write, are checked for 16-byte alignment before any launch."""
+    d = _desc(B, "glm_small_bf16")
+    need = B.moe_backward_workspace_size(d)
+    full = dict(dx=256, dw_r=256, dw1=256, dw2=256, dsh_w1=256, dsh_w2=256)
+    for field in ("w_r", "w1", "w2", "sh_w1", "sh_w2"):
+        w = B.Weights()
+        w.w_r, w.w1, w.w2, w.sh_w1, w.sh_w2 = 256, 256, 256, 256, 256
+        setattr(w, field, 264)
+        with pytest.raises(B.MoEError) as e:
+            B.moe_forward(d, w, 256, 256, 256, B.moe_workspace_size(d))
+        assert e.value.status == 1, field
+        with pytest.raises(B.MoEError) as e:
+            B.moe_backward(d, w, 256, 256, B.Grads(**full), 256, need)
+        assert e.value.status == 1, field
+    w = B.Weights()
+    w.w_r, w.w1, w.w2, w.sh_w1, w.sh_w2 = 256, 256, 256, 256, 256
+    for x, dy in ((258, 256), (256, 260)):
+        with pytest.raises(B.MoEError) as e:
+            B.moe_backward(d, w, x, dy, B.Grads(**full), 256, need)
+        assert e.value.status == 1
+    with pytest.raises(B.MoEError) as e:
+        B.moe_forward(d, w, 258, 256, 256, B.moe_workspace_size(d))
+    assert e.value.status == 1
+    for field in ("dw1", "dw2", "dsh_w1", "dsh_w2"):
+        g = B.Grads(**dict(full, **{field: 260}))
+        with pytest.raises(B.MoEError) as e:
+            B.moe_backward(d, w, 256, 256, g, 256, need)
+        assert e.value.status == 1, field
+
+
 def test_gather_rows_host_checks(B):
     with pytest.raises(B.MoEError) as e:
         B.moe_gather_rows(256, 256, None, 256, -1, 4, 8, 1)

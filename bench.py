@@ -62,6 +62,8 @@ def parse_args():
                     help="backward: time moe_backward (all gradients of the layer) instead of the forward")
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism: each of the N ranks owns M/N experts, rows exchanged by all-to-all")
+    ap.add_argument("--capacity-factor", type=float, default=2.0,
+                    help="--ep: each expert takes at most ceil(f T k / M) rows from each rank (fixed splits)")
     return ap.parse_args()
 
 
@@ -915,7 +917,7 @@ def run_ep(args):
     del full
     r0, r1 = token_rows(rank, T)
     x = ms.normal_rows(torch.arange(r0, r1, device=dev), D, 1.0, ms._key(cfg, "x"), ms.act_dtype(cfg))
-    layer = ep.ExpertParallelMoE(cfg, mine, rank, world)
+    layer = ep.ExpertParallelMoE(cfg, mine, rank, world, capacity_factor=args.capacity_factor)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     for _ in range(max(3, args.warmup)):
@@ -930,23 +932,23 @@ def run_ep(args):
     torch.cuda.synchronize()
     if sampler:
         sampler.start()
-    recv, launches = [], 0
     for i in range(K):
         flush.zero_()
         starts[i].record(stream)
         layer.forward(x)
         ends[i].record(stream)
-        recv.append(layer.last_plan.rows_received)
-        launches += layer.launch_count(T, recv[-1])
     torch.cuda.synchronize()
+    launches = K * layer.launch_count(T)
+    bufs = layer.buffers(T, x.dtype)
+    kept_sent = int(bufs["kept"].sum().item())          # after the timed steps: the same every step
+    kept_recv = int(bufs["recv_kept"].sum().item())
     clocks = sampler.stop() if sampler else None
     if dist is not None:
         dist.barrier()
     ms_step = max_over_ranks(dist, sum(starts[i].elapsed_time(ends[i]) for i in range(K)) / K, dev)
-    if int(layer.status.item()) != 0:
+    if any(layer.status.tolist()):
         raise RuntimeError("device status flag set during the timed steps")
     if rank == 0:
-        rows_out = (world - 1) / max(1, world) * T * cfg["k"]  # rows that leave the rank, on average
         out = {
             "metric": "MoE layer forward throughput, expert-parallel (routed experts split over the ranks)",
             "value": world * T / (ms_step / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": K,
@@ -956,10 +958,12 @@ def run_ep(args):
             "config": {"workload": args.config, "T_per_gpu": T, "D": D, "M": cfg["M"], "k": cfg["k"],
                        "I": cfg["I"], "I_sh": cfg.get("I_sh", 0), "parallelism": f"ep{world}",
                        "l2": "flushed between steps (256 MiB write outside the timed events)"},
-            "exchange": {"rows_received_rank0_mean": float(np.mean(recv)),
-                         "rows_leaving_each_rank_expected": rows_out,
-                         "bytes_out_per_rank_expected": rows_out * D * (2 if cfg["dtype"] == "bf16" else 4)
-                         + rows_out * 4 + rows_out * D * 4},
+            "exchange": {"capacity_factor": args.capacity_factor, "cap_rows_per_expert_per_rank": bufs["cap"],
+                         "rows_per_rank_pair": bufs["R"] // world,
+                         "pairs_kept_rank0": kept_sent, "pairs_dropped_rank0": T * cfg["k"] - kept_sent,
+                         "rows_received_rank0": kept_recv,
+                         "bytes_out_per_rank": (world - 1) * (bufs["R"] // world) * (
+                             D * (2 if cfg["dtype"] == "bf16" else 4) + 4 + D * 4)},
             "e2e": None, "gpu_launches": launches, "gpu_launches_note": "rank 0's own kernels; NCCL's not counted",
             "clocks": clocks,
         }

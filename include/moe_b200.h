@@ -77,6 +77,7 @@ typedef enum { MOE_ACT_GELU_TANH = 0, MOE_ACT_SWIGLU = 1 } moe_act_t;
 #define MOE_DEVERR_BAD_EXPERT_INDEX 1 /* topk_idx entry outside [0, M] (M: the sentinel) */
 #define MOE_DEVERR_TIMEOUT 2          /* a bounded wait inside a kernel gave up */
 #define MOE_DEVERR_BAD_ROW_TOKEN 3    /* row_token entry outside [0, T) (row zero-filled) */
+#define MOE_DEVERR_BAD_COUNT 4        /* an exchanged row count outside [0, cap] (clamped) */
 
 /* One MoE layer's shape and options (HF config names in brackets). */
 typedef struct {
@@ -235,6 +236,47 @@ int moe_expert_capacity(double factor, int T, int k, int M);
 moe_status_t moe_gather_rows(const void* x, const int32_t* row_token, const int32_t* n_rows,
                              void* x_perm, int rows, int T, int D, int dtype,
                              int32_t* device_status, void* stream);
+
+/* ---- expert parallelism: fixed-split exchange (GLaM industry article,
+ *      first route: cross-node communication between experts) ------------
+ * The routed experts split over `world` ranks, rank q owning experts
+ * [q E, (q + 1) E), E = M / world.  Every split of the exchange is E * cap
+ * rows, whatever the routing, so the all-to-alls between these calls need
+ * no row counts on the host and a step runs without a device-to-host read.
+ * An expert keeps the first `cap` of its pairs in dispatch order (the rule
+ * of moe_capacity_drop); later pairs are dropped (they add nothing to y). */
+
+/* Sender: pack the dispatch order of moe_permute (offsets [M+1],
+ * row_token, row_w, slot_of [T, k]) into M blocks of cap rows, block e
+ * holding expert e's first min(counts[e], cap) rows and zeros after them:
+ *   x_pad [M * cap, D] (dtype), w_pad [M * cap] fp32 (0 on padding rows),
+ *   kept [M] int32 = min(counts[e], cap),
+ *   slot_pad [T, k] int32 = e * cap + i for the pair at position i of
+ *     expert e's segment when i < cap, else -1 (dropped or sentinel).
+ * Owner q's rows are x_pad[q E cap, (q + 1) E cap): one piece per rank.
+ * x and x_pad in dtype.  A row_token outside [0, T) gives a zero row with
+ * weight 0 and sets MOE_DEVERR_BAD_ROW_TOKEN in *device_status (a device
+ * int32 cleared by the call, may be NULL).  cap >= 0, M <= 1024. */
+moe_status_t moe_ep_pack(const void* x, const int32_t* offsets, const int32_t* row_token,
+                         const float* row_w, const int32_t* slot_of, int T, int k, int M, int D,
+                         int dtype, int cap, void* x_pad, float* w_pad, int32_t* slot_pad,
+                         int32_t* kept, int32_t* device_status, void* stream);
+
+/* Receiver: the blocks arrive as [world][E][cap] (source rank q, local
+ * expert e, row i) with recv_kept [world, E] = the senders' kept counts and
+ * w_recv [world * E * cap] their w_pad.  Builds the expert-major dispatch
+ * order over the arrival rows, for moe_expert_ffn with M = E and k = 1:
+ *   offsets [E+1]: expert e's rows from rank 0, then rank 1, ...;
+ *   row_token[p], row_w[p] for p < offsets[E]: the arrival row at dispatch
+ *     position p and its gate weight;
+ *   slot_of [world * E * cap]: the dispatch position of each arrival row,
+ *     -1 for padding (moe_combine with k = 1 puts the expert outputs back
+ *     into arrival order, padding rows zero).
+ * A recv_kept entry outside [0, cap] is clamped and sets
+ * MOE_DEVERR_BAD_COUNT.  world * E <= 1024. */
+moe_status_t moe_ep_unpack(const int32_t* recv_kept, const float* w_recv, int world, int E, int cap,
+                           int32_t* offsets, int32_t* row_token, float* row_w, int32_t* slot_of,
+                           int32_t* device_status, void* stream);
 
 /* ---- experts: "GLaM" eq. FFN; GLM-5 GlmMoeDsaExperts.forward ----------- */
 

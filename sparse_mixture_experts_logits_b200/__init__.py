@@ -19,8 +19,8 @@ from .abi import (  # noqa: F401
     moe_algorithmic_work, EXPORTED_SYMBOLS, moe_forward_add,
     DenseDesc, moe_dense_ffn_workspace_size, moe_dense_ffn, moe_dense_ffn_profiled, NUM_DENSE_EVENTS,
     Grads, moe_backward_workspace_size, moe_backward, moe_backward_launch_count, moe_gather_rows,
-    moe_capacity_drop, moe_expert_capacity, moe_selftest_wait_timeout,
+    moe_capacity_drop, moe_expert_capacity, moe_selftest_wait_timeout, moe_ep_pack, moe_ep_unpack,
     DTYPE_F32, DTYPE_BF16, GATE_SOFTMAX, GATE_SIGMOID_BIAS, ACT_GELU_TANH, ACT_SWIGLU,
-    DEVERR_NONE, DEVERR_BAD_EXPERT_INDEX, DEVERR_TIMEOUT, DEVERR_BAD_ROW_TOKEN,
+    DEVERR_NONE, DEVERR_BAD_EXPERT_INDEX, DEVERR_TIMEOUT, DEVERR_BAD_ROW_TOKEN, DEVERR_BAD_COUNT,
 )
 from .layer import DenseLayer, MoELayer, dense_desc_from_config, desc_from_config, weights_from_tensors  # noqa: F401,E501

@@ -16,7 +16,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_DEVICE =
 DTYPE_F32, DTYPE_BF16 = 0, 1
 GATE_SOFTMAX, GATE_SIGMOID_BIAS = 0, 1
 ACT_GELU_TANH, ACT_SWIGLU = 0, 1
-DEVERR_NONE, DEVERR_BAD_EXPERT_INDEX, DEVERR_TIMEOUT, DEVERR_BAD_ROW_TOKEN = 0, 1, 2, 3
+DEVERR_NONE, DEVERR_BAD_EXPERT_INDEX, DEVERR_TIMEOUT, DEVERR_BAD_ROW_TOKEN, DEVERR_BAD_COUNT = 0, 1, 2, 3, 4
 
 EXPORTED_SYMBOLS = [
     "moe_status_string", "moe_version", "moe_device_status",
@@ -28,7 +28,7 @@ EXPORTED_SYMBOLS = [
     "moe_forward_profiled", "moe_forward_launch_count", "moe_algorithmic_work",
     "moe_forward_add", "moe_dense_ffn_workspace_size", "moe_dense_ffn", "moe_dense_ffn_profiled",
     "moe_backward_workspace_size", "moe_backward", "moe_backward_launch_count", "moe_gather_rows",
-    "moe_capacity_drop", "moe_expert_capacity", "moe_selftest_wait_timeout",
+    "moe_capacity_drop", "moe_expert_capacity", "moe_selftest_wait_timeout", "moe_ep_pack", "moe_ep_unpack",
 ]
 NUM_STAGE_EVENTS = 9
 NUM_DENSE_EVENTS = 3
@@ -120,6 +120,8 @@ _decl("moe_dense_ffn_profiled", _i, [_P(DenseDesc), _vp, _vp, _vp, _vp, _vp, _vp
                                      _P(_vp), _i])
 _decl("moe_gather_rows", _i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp])
 _decl("moe_capacity_drop", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp])
+_decl("moe_ep_pack", _i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp])
+_decl("moe_ep_unpack", _i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp])
 _decl("moe_expert_capacity", _i, [ctypes.c_double, _i, _i, _i])
 _decl("moe_selftest_wait_timeout", _i, [ctypes.c_uint64, _vp, _vp, _vp])
 _decl("moe_backward_workspace_size", _sz, [_P(LayerDesc)])
@@ -281,6 +283,18 @@ def moe_gather_rows(x, row_token, n_rows, x_perm, rows, T, D, dtype, device_stat
 
 def moe_capacity_drop(topk_idx, slot_of, offsets, T, k, M, capacity, stream=None):
     _check("moe_capacity_drop", lib.moe_capacity_drop(topk_idx, slot_of, offsets, T, k, M, capacity, stream))
+
+
+def moe_ep_pack(x, offsets, row_token, row_w, slot_of, T, k, M, D, dtype, cap, x_pad, w_pad, slot_pad, kept,
+                device_status=None, stream=None):
+    _check("moe_ep_pack", lib.moe_ep_pack(x, offsets, row_token, row_w, slot_of, T, k, M, D, dtype, cap, x_pad,
+                                          w_pad, slot_pad, kept, device_status, stream))
+
+
+def moe_ep_unpack(recv_kept, w_recv, world, E, cap, offsets, row_token, row_w, slot_of, device_status=None,
+                  stream=None):
+    _check("moe_ep_unpack", lib.moe_ep_unpack(recv_kept, w_recv, world, E, cap, offsets, row_token, row_w,
+                                              slot_of, device_status, stream))
 
 
 def moe_expert_capacity(factor, T, k, M) -> int:

@@ -174,7 +174,10 @@ def moe_backward(cfg, inp, dy, idx=None):
     dw [T, k] (gradient of each chosen weight) and dl [T, M] (of the
     logits), with the forward's routing, and the absolute-term sums
     (*_abs) of the expert and shared weight gradients (see
-    expert_ffn_backward)."""
+    expert_ffn_backward) and of the router's, dw_r_abs = |x|^T |dl|: the
+    scale of the rounding error of a sum whose terms carry one bf16
+    rounding of an operand (dl, when the router's backward GEMMs run on
+    bf16 operands)."""
     r = F.route(inp["x"], inp["w_r"], inp.get("e_bias"), cfg["k"], cfg["gate"],
                 cfg["norm_topk_prob"], cfg["alpha"], cfg["eps"], cfg.get("n_group", 1),
                 cfg.get("topk_group", 1))
@@ -229,7 +232,7 @@ def moe_backward(cfg, inp, dy, idx=None):
     return {"dx": dx, "dw_r": dw_r, "dw1": dw1, "dw2": dw2, "db1": db1, "db2": db2,
             "dsh_w1": dsh_w1, "dsh_w2": dsh_w2, "dw": dw, "dl": dl, "idx": r["idx"], "w": r["w"],
             "dw1_abs": dw1_abs, "dw2_abs": dw2_abs, "db1_abs": db1_abs, "dsh_w1_abs": dsh_w1_abs,
-            "dsh_w2_abs": dsh_w2_abs}
+            "dsh_w2_abs": dsh_w2_abs, "dw_r_abs": np.abs(x).T @ np.abs(dl)}
 
 
 def dense_layer_backward(x, act, w1, w2, b1, b2, dy):

@@ -188,9 +188,16 @@ def pin_absolute_term_sums(B):
         inp = tiny_inputs(cfg, 140)
         dy = np.random.default_rng(141).standard_normal((cfg["T"], cfg["D"]))
         g = B.moe_backward(cfg, inp, dy)
-        for name in ("dw1", "dw2", "db1", "dsh_w1", "dsh_w2"):
+        for name in ("dw1", "dw2", "db1", "dsh_w1", "dsh_w2", "dw_r"):
             if g[name] is not None:
                 assert np.all(np.abs(g[name]) <= g[name + "_abs"] + 1e-12), name
+        # the router's: dw_r_abs[d, m] = sum_t |x[t, d]| |dl[t, m]| by a scalar loop
+        xa = np.abs(np.asarray(inp["x"], np.float64))
+        for d, m in ((0, 0), (cfg["D"] - 1, cfg["M"] - 1), (1, 2)):
+            s = 0.0
+            for t in range(cfg["T"]):
+                s += xa[t, d] * abs(g["dl"][t, m])
+            assert abs(s - g["dw_r_abs"][d, m]) <= 1e-12 * max(1.0, s), (d, m)
         # brute force of one expert's sums from its own rows
         e = int(g["idx"][0, 0])
         tt, jj = np.nonzero(g["idx"] == e)

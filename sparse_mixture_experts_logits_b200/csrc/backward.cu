@@ -271,7 +271,8 @@ __device__ __forceinline__ float warp_max(float v) {
 // the weight formula of the router (lane j < k holds chosen slot j).
 __global__ void bwd_router_kernel(const float* __restrict__ logits, const int32_t* __restrict__ idx,
                                   const float* __restrict__ dw, int T, int M, int k, int gate, int norm,
-                                  float alpha, float eps, float* __restrict__ dl) {
+                                  float alpha, float eps, float* __restrict__ dl,
+                                  __nv_bfloat16* __restrict__ dl_bf) {
   const int lane = threadIdx.x & 31;
   const int warps = gridDim.x * (blockDim.x >> 5);
   for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
@@ -303,6 +304,8 @@ __global__ void bwd_router_kernel(const float* __restrict__ logits, const int32_
       __syncwarp();
       if (e >= 0) dlt[e] += alpha * pj * g;
       __syncwarp();
+      if (dl_bf != nullptr)
+        for (int i = lane; i < M; i += 32) dl_bf[static_cast<long long>(t) * M + i] = __float2bfloat16_rn(dlt[i]);
       continue;
     }
     for (int i = lane; i < M; i += 32) dlt[i] = 0.f;
@@ -332,6 +335,8 @@ __global__ void bwd_router_kernel(const float* __restrict__ logits, const int32_
       if (e >= 0) dlt[e] = dg * gj * (1.0f - gj);
     }
     __syncwarp();
+    if (dl_bf != nullptr)
+      for (int i = lane; i < M; i += 32) dl_bf[static_cast<long long>(t) * M + i] = __float2bfloat16_rn(dlt[i]);
   }
 }
 
@@ -432,10 +437,11 @@ cudaError_t launch_bwd_colsum(const float* Y, long long ldy, const int32_t* offs
 }
 
 cudaError_t launch_bwd_router(const float* logits, const int32_t* idx, const float* dw, int T, int M, int k,
-                              int gate, int norm, float alpha, float eps, float* dl, cudaStream_t s) {
+                              int gate, int norm, float alpha, float eps, float* dl, void* dl_bf,
+                              cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  bwd_router_kernel<<<grid_1d(static_cast<long long>(T) * 32, 256), 256, 0, s>>>(logits, idx, dw, T, M, k, gate,
-                                                                                 norm, alpha, eps, dl);
+  bwd_router_kernel<<<grid_1d(static_cast<long long>(T) * 32, 256), 256, 0, s>>>(
+      logits, idx, dw, T, M, k, gate, norm, alpha, eps, dl, static_cast<__nv_bfloat16*>(dl_bf));
   return cudaGetLastError();
 }
 

@@ -51,6 +51,7 @@ enum GemmEpilogue : int {
   EPI_BWD_GELU_DACT = 9,    // G = acc, h = aux[r, n]: out = w G GELU'(h); parts += G GELU(h)
   EPI_BWD_SWIGLU_DACT = 10, // G = acc, g = aux[r, n], u = aux[r, I + n], a = SiLU(g) u, da = w G:
                             //   out[., n] = da u SiLU'(g), out[., I + n] = da SiLU(g); parts += G a
+  EPI_ACCUM_F32 = 11,       // out fp32 += acc   (the router's dx onto the shared expert's)
 };
 
 // Operand layouts of the tokens-on-N GEMM (gemm_swap_sm100.cuh): the forward

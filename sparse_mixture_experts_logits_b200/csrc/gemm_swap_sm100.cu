@@ -119,6 +119,7 @@ cudaError_t launch_swap_rows(int layout, int epi, const SwapMaps& m, const SwapA
     case EPI_STORE_F32: return launch_swap_epi<EPI_STORE_F32>(m, a, tiles_ub, s);
     case EPI_STORE_BF16: return launch_swap_epi<EPI_STORE_BF16>(m, a, tiles_ub, s);
     case EPI_BIAS_ADD: return launch_swap_epi<EPI_BIAS_ADD>(m, a, tiles_ub, s);
+    case EPI_ACCUM_F32: return launch_swap_epi<EPI_ACCUM_F32>(m, a, tiles_ub, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -196,7 +196,7 @@ __device__ __forceinline__ SwapTile swap_decode(int tile, int G, const int* s_ts
 // lanes cover 32 consecutive columns, i.e. one contiguous row segment.
 template <int EPI>
 __device__ __forceinline__ void swap_store(const SwapArgs& a, size_t row, int col, float v) {
-  if constexpr (EPI == EPI_SCALE_BIAS || EPI == EPI_STORE_F32)
+  if constexpr (EPI == EPI_SCALE_BIAS || EPI == EPI_STORE_F32 || EPI == EPI_ACCUM_F32)
     static_cast<float*>(a.out)[row * a.ldo + col] = v;
   else
     static_cast<__nv_bfloat16*>(a.out)[row * a.ldo + col] = __float2bfloat16_rn(v);
@@ -204,7 +204,7 @@ __device__ __forceinline__ void swap_store(const SwapArgs& a, size_t row, int co
 // Same at an element offset `base` (a group's own output block).
 template <int EPI>
 __device__ __forceinline__ void swap_store(const SwapArgs& a, size_t base, int col, float v, size_t row) {
-  if constexpr (EPI == EPI_SCALE_BIAS || EPI == EPI_STORE_F32)
+  if constexpr (EPI == EPI_SCALE_BIAS || EPI == EPI_STORE_F32 || EPI == EPI_ACCUM_F32)
     static_cast<float*>(a.out)[base + row * a.ldo + col] = v;
   else
     static_cast<__nv_bfloat16*>(a.out)[base + row * a.ldo + col] = __float2bfloat16_rn(v);
@@ -517,20 +517,44 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       } else
       for (int c = 32 * part; c < t.n; c += 64) {
-        // input-gradient epilogues: the chunk's saved pre-activations are
-        // requested first, so that their memory latency overlaps the TMEM read
-        // and each other's
+        // Every value this chunk reads from memory (the input-gradient
+        // epilogues' saved pre-activations, the addend, the fp32 sum added
+        // onto) is requested first, all 32 rows together, so that the loads
+        // overlap the TMEM read and each other's.  Read inside the store loop
+        // they would wait one memory round trip per row: the compiler cannot
+        // move a load above the store to `out` before it.
         float hv[32], uv[32];
-        if constexpr (kDact) {
+        if constexpr (kDact || EPI == EPI_BIAS_ADD) {
           const int nvd = min(32, t.nrows - c);
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const bool live = col_ok && i < nvd;
             const size_t row = row0 + c + i;
-            hv[i] = live ? args.aux[row * args.ld_aux + col] : 0.f;
-            if constexpr (EPI == EPI_BWD_SWIGLU_DACT)
-              uv[i] = live ? args.aux[row * args.ld_aux + args.half_cols + col] : 0.f;
+            if constexpr (kDact) {
+              hv[i] = live ? args.aux[row * args.ld_aux + col] : 0.f;
+              if constexpr (EPI == EPI_BWD_SWIGLU_DACT)
+                uv[i] = live ? args.aux[row * args.ld_aux + args.half_cols + col] : 0.f;
+            } else {
+              hv[i] = live && args.addend != nullptr ? __bfloat162float(args.addend[row * args.ldo + col]) : 0.f;
+            }
           }
+        }
+        if constexpr (EPI == EPI_ACCUM_F32) {
+          // out += acc in place: the chunk's 32 rows read first, then the TMEM read
+          const int nva = col_ok ? min(32, t.nrows - c) : 0;
+          float* op = static_cast<float*>(args.out) + (row0 + c) * args.ldo + col;
+          const size_t ld = args.ldo;
+          const float* lp = op;
+#pragma unroll
+          for (int i = 0; i < 32; ++i, lp += ld) hv[i] = i < nva ? *lp : 0.f;
+          uint32_t ra[32];
+          MOE_TMEM_LD32(tacc + c, ra);
+          tmem_ld_wait();
+          float* sp = op;
+#pragma unroll
+          for (int i = 0; i < 32; ++i, sp += ld)
+            if (i < nva) *sp = __uint_as_float(ra[i]) + hv[i];
+          continue;
         }
         uint32_t r[32];
         MOE_TMEM_LD32(tacc + c, r);
@@ -618,10 +642,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             float v = __uint_as_float(r[i]) + bias;
             if constexpr (EPI == EPI_GELU_BIAS) v = gelu_tanh_fast(v);
             if constexpr (EPI == EPI_SCALE_BIAS) v *= __shfl_sync(0xffffffffu, rs, i);
-            if constexpr (EPI == EPI_BIAS_ADD) {
-              if (args.addend != nullptr && col_ok && i < nv)
-                v += __bfloat162float(args.addend[(row0 + c + i) * args.ldo + col]);
-            }
+            if constexpr (EPI == EPI_BIAS_ADD || EPI == EPI_ACCUM_F32) v += hv[i];
             if constexpr (EPI == EPI_BWD_GELU_SAVE) {
               const float a = gelu_tanh_fast(v);
               const float w = __shfl_sync(0xffffffffu, rs, i);

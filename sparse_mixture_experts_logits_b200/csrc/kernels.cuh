@@ -173,8 +173,10 @@ cudaError_t launch_bwd_pairs(int dtype, const void* dy, const float* o, const in
 // out[g, :] = column sums of Y over the rows of group g.
 cudaError_t launch_bwd_colsum(const float* Y, long long ldy, const int32_t* offsets, int G, long long rows_cap,
                               int N, float* out, cudaStream_t s);
-// dL/dlogits [T, M] from dL/dw [T, k].
+// dL/dlogits [T, M] from dL/dw [T, k] (fp32), and a bf16 copy when dl_bf is
+// not null (the operand of the router's tensor-core backward GEMMs).
 cudaError_t launch_bwd_router(const float* logits, const int32_t* idx, const float* dw, int T, int M, int k,
-                              int gate, int norm, float alpha, float eps, float* dl, cudaStream_t s);
+                              int gate, int norm, float alpha, float eps, float* dl, void* dl_bf,
+                              cudaStream_t s);
 
 }  // namespace moe

@@ -884,12 +884,21 @@ struct BwdWs {
   size_t xp, hpre, act, dO, da, dxp, dwp, dl, hs, as, das, dxs, total;
   // tensor-core path (bf16): the padded dispatch order and its bf16 tensors
   long long rows_pad;
-  size_t offp, slotp, rtp, rwp, xpp, dypp, hpb, ab, awb, dhb, dxpp, parts, hsb, asb, dhsb, rpart;
+  size_t offp, slotp, rtp, rwp, xpp, dypp, hpb, ab, awb, dhb, dxpp, parts, hsb, asb, dhsb, rpart, dlb;
 };
 
 // Chunks of the token sum in the router's weight gradient dW_r = x^T dlogits
 // (partial sums added in order): enough blocks to fill the GPU.
 int router_ksplit(int T) { return std::max(1, std::min(16, T / 1024)); }
+
+// A bf16 layer runs the router's two backward GEMMs (dW_r = x^T dlogits and
+// dx += dlogits W_r^T) on the tensor cores, with dlogits rounded to bf16 as
+// their operand, when every TMA box of them has whole rows: M a multiple of
+// 8 and at least one 64-column box wide.  Otherwise (small test layers) on
+// the CUDA cores in fp32.
+bool router_bwd_tc(const moe_layer_desc_t* d) {
+  return d->dtype == MOE_DTYPE_BF16 && d->M % 8 == 0 && d->M >= 64;
+}
 
 // Rows of the backward's padded dispatch order: every expert's segment is
 // rounded up to 64 rows, so at most T k + 63 M rows.
@@ -925,7 +934,8 @@ BwdWs backward_layout_tc(const moe_layer_desc_t* d) {
   L.asb = c.take(T * Is * 2);
   L.dhsb = c.take(T * 2 * Is * 2);
   L.dxs = c.take(T * D * 4);
-  L.rpart = c.take(static_cast<size_t>(router_ksplit(d->T)) * D * d->M * 4);
+  L.rpart = router_bwd_tc(d) ? 0 : c.take(static_cast<size_t>(router_ksplit(d->T)) * D * d->M * 4);
+  L.dlb = router_bwd_tc(d) ? c.take(T * d->M * 2) : 0;
   L.total = c.off;
   return L;
 }
@@ -1182,16 +1192,34 @@ moe_status_t backward_tc_impl(const moe_layer_desc_t* d, const moe_weights_t* w,
   }
   {
     Range r("moe.router_backward");
+    const bool tc = router_bwd_tc(d);
+    void* dlb = tc ? at<void*>(ws, L.dlb) : nullptr;
     MOE_CUDA(launch_bwd_router(logits, idx, dwp, T, M, k, d->gate, d->norm_topk_prob, d->routed_scaling_factor,
-                               d->eps, dl, s));
-    BwdGemmLaunch wr = bwd_gemm(x, 1, D, true, dl, 1, M, 0, false, g->dw_r, M, D, T, M);
-    wr.mode = 1;
-    wr.ksplit = router_ksplit(T);
-    wr.partial = at<float*>(ws, L.rpart);
-    MOE_CUDA(launch_bwd_gemm(wr, s));
-    BwdGemmLaunch xr = bwd_gemm(dl, M, 1, false, w->w_r, M, 1, 0, true, dxs, D, T, M, D);
-    xr.accumulate = Is > 0 ? 1 : 0;  // onto the shared expert's dx
-    MOE_CUDA(launch_bwd_gemm(xr, s));
+                               d->eps, dl, dlb, s));
+    if (tc) {
+      // dW_r [D, M] = x^T dlogits: the weight-gradient layout over one group of T rows,
+      // dlogits (bf16) on the A side so that its M columns are the output's contiguous ones
+      SwapLaunch gw = bwd_swap(EPI_STORE_F32, kSwWgrad, dlb, T, x, T, 0, 1, nullptr, nullptr, T, M, g->dw_r, M,
+                               status);
+      gw.b_cols = D;
+      gw.b_tiles = (D + 255) / 256;
+      gw.out_gstride = 1ll * D * M;
+      MOE_CUDA(launch_gemm_swap(gw, s));
+      // dx += dlogits W_r^T: the forward layout, W_r [D, M] as K-major weight rows (K = M),
+      // added onto the shared expert's dx when there is one
+      SwapLaunch gx = bwd_swap(Is > 0 ? EPI_ACCUM_F32 : EPI_STORE_F32, kSwFwd, w->w_r, D, dlb, T, M, 1, nullptr,
+                               nullptr, T, D, dxs, D, status);
+      MOE_CUDA(launch_gemm_swap(gx, s));
+    } else {
+      BwdGemmLaunch wr = bwd_gemm(x, 1, D, true, dl, 1, M, 0, false, g->dw_r, M, D, T, M);
+      wr.mode = 1;
+      wr.ksplit = router_ksplit(T);
+      wr.partial = at<float*>(ws, L.rpart);
+      MOE_CUDA(launch_bwd_gemm(wr, s));
+      BwdGemmLaunch xr = bwd_gemm(dl, M, 1, false, w->w_r, M, 1, 0, true, dxs, D, T, M, D);
+      xr.accumulate = Is > 0 ? 1 : 0;  // onto the shared expert's dx
+      MOE_CUDA(launch_bwd_gemm(xr, s));
+    }
   }
   {
     Range r("moe.combine_backward");
@@ -1319,7 +1347,7 @@ moe_status_t backward_impl(const moe_layer_desc_t* d, const moe_weights_t* w, co
   {
     Range r("moe.router_backward");
     MOE_CUDA(launch_bwd_router(logits, idx, dwp, T, M, k, d->gate, d->norm_topk_prob, d->routed_scaling_factor,
-                               d->eps, dl, s));
+                               d->eps, dl, nullptr, s));
     BwdGemmLaunch wr = bwd_gemm(x, 1, D, bf, dl, 1, M, 0, false, g->dw_r, M, D, T, M);
     wr.mode = 1;
     MOE_CUDA(launch_bwd_gemm(wr, s));
@@ -1358,7 +1386,7 @@ int moe_backward_launch_count(const moe_layer_desc_t* d) {
     if (d->act == MOE_ACT_GELU_TANH && d->has_bias) n += 2;        // bias gradients
     if (d->I_sh > 0) n += 5;                                         // shared expert GEMMs
     n += 3;                                                          // router backward, dW_r, router dx
-    if (router_ksplit(d->T) > 1) n += 1;                             // dW_r chunk sums
+    if (!router_bwd_tc(d) && router_ksplit(d->T) > 1) n += 1;        // dW_r chunk sums
     n += 1;                                                          // dx combine
     return n;
   }

@@ -170,12 +170,18 @@ def test_backward_matches_oracle(B, name):
                                        ("glam_small_bf16", dict(M=1, k=1)), ("glm_small_f32", dict(T=200)),
                                        ("glm_medium_bf16", dict()), ("glam_small_bf16", dict(T=700)),
                                        ("glm_small_bf16", dict(I_sh=0)),
-                                       ("glm_medium_bf16", dict(e_bias=("zipf", 1.1, 1.0)))])
+                                       ("glm_medium_bf16", dict(e_bias=("zipf", 1.1, 1.0))),
+                                       ("glm_medium_bf16", dict(M=160)), ("glm_small_bf16", dict(M=64, D=320)),
+                                       ("glm_small_bf16", dict(M=72, I_sh=0))])
 def test_backward_edge_shapes(B, name, over):
     """A single token, ragged tiles, k = 1, k = M, one expert (softmax: its
     weight is exactly 1, so the router gradient is exactly 0), several
     256-row token tiles per expert, no shared expert, and a skewed routing
-    that leaves most experts empty (their weight gradients exactly 0)."""
+    that leaves most experts empty (their weight gradients exactly 0).  The
+    last three take the router's backward onto the tensor cores (M a multiple
+    of 8, at least 64): a partial k-block of dlogits (M = 160, 72), a partial
+    256-column output tile (D = 320), and dx stored rather than added onto
+    the shared expert's (no shared expert)."""
     cfg = ms.get_config(name, **over)
     inp, dy, _, g, idx, _ = run(B, cfg)
     ref = oracle.moe_backward.moe_backward(cfg, host(inp), np64(dy), idx=idx)

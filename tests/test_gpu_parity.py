@@ -81,7 +81,10 @@ def test_group_limited_full_size(B):
 
 @pytest.mark.parametrize("name,over", [
     ("glm_small_bf16", dict(T=1)),
+    ("glm_small_bf16", dict(T=128)),
     ("glm_small_bf16", dict(T=129)),
+    ("glm_small_bf16", dict(T=64, I_sh=208)),            # a shared gate/up width not a multiple of 32
+    ("glm_medium_bf16", dict(T=40)),                     # few tokens, I_sh = 320, D = 512
     ("glm_small_bf16", dict(k=1)),
     ("glm_small_bf16", dict(M=4, k=4)),
     ("glam_small_bf16", dict(M=1, k=1)),

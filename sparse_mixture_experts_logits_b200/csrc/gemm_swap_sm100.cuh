@@ -53,10 +53,9 @@
 
 namespace moe {
 
-// A pipeline stage holds kSwKB consecutive k-blocks of 64: the MMA thread waits
-// once and commits once per stage.  Each barrier wait and commit costs the
-// single issuing thread as much as an N = 256 MMA takes to run, so fewer of
-// them per MMA keeps the tensor pipe fed.
+// A pipeline stage holds kSwKB consecutive k-blocks of 64: the MMA thread
+// waits once and commits once per stage.  Two k-blocks per stage (3 stages
+// of 64 KB) measured faster than one (6 stages of 32 KB) and than three.
 constexpr int kSwKB = 2;
 constexpr int kSwStages = 3;
 constexpr int kSwATileBytes = 128 * kBK * 2;  // 128 weight rows per CTA, one k-block

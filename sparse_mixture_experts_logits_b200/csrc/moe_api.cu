@@ -267,8 +267,8 @@ moe_status_t run_experts(const moe_layer_desc_t* d, const moe_weights_t* w, cons
   const void* b1 = (!swiglu && d->has_bias) ? w->b1 : nullptr;
   const void* b2 = (!swiglu && d->has_bias) ? w->b2 : nullptr;
   // A handful of rows per expert (decode): tokens on M with single-CTA MMAs. The 128-row token
-  // tile is mostly padding, but a single-CTA MMA issues far faster than a pair's, and the
-  // weights still stream once (measured: GLM-4.5 decode expert GEMMs 0.837 -> 0.810 ms).
+  // tile is mostly padding, but each CTA streams its own slice of the touched experts'
+  // weights once (measured: GLM-4.5 decode expert GEMMs 0.837 -> 0.810 ms).
   const bool few_rows = static_cast<long long>(d->T) * d->k < 4ll * d->M;
   if (d->dtype == MOE_DTYPE_BF16 && few_rows) {
     MOE_CUDA(launch_gather_rows(x, row_token, offsets + d->M, x_perm, pairs, d->T, d->D, 2, status, s));

@@ -68,7 +68,7 @@ cudaError_t launch_swap_epi(const SwapMaps& maps, const SwapArgs& args, long lon
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t q = {};
     q.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
-    q.blockDim = dim3(kGemmThreads, 1, 1);
+    q.blockDim = dim3(swap_threads<EPI>(), 1, 1);
     q.dynamicSmemBytes = kSwDynSmem;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;
@@ -86,7 +86,7 @@ cudaError_t launch_swap_epi(const SwapMaps& maps, const SwapArgs& args, long lon
   const long long units = std::min<long long>(max_clusters[dev & 31].load(), std::max<long long>(1, tiles_ub));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(2 * units), 1, 1);
-  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.blockDim = dim3(swap_threads<EPI>(), 1, 1);
   cfg.dynamicSmemBytes = kSwDynSmem;
   cfg.stream = s;
   cudaLaunchAttribute at[1];

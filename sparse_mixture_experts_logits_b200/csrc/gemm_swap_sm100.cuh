@@ -82,10 +82,21 @@ struct SwapMaps {
 // a 2-stage pipeline and gives the third stage's 64 KB to its eight epilogue
 // warps as two 4 KB store-staging buffers each: every 32 x 32 fp32 chunk
 // leaves through one TMA store instead of 32 warp-wide scalar stores.
+// Epilogue warps (a multiple of 4: one per TMEM lane quarter, then more
+// chunk parts).  The fused SwiGLU epilogue is light next to its long
+// contraction, and with 4 warps the producer and MMA warps share their
+// schedulers with fewer epilogue warps: the gate/up GEMMs ran 2-6% faster
+// (GLM-5, GLM-4.5).  The heavier epilogues (GELU, fp32 rows, the backward's)
+// keep 8: with 4 they were 20-50% slower.
+template <int EPI>
+constexpr int swap_epi_warps() { return EPI == EPI_SWIGLU ? 4 : 8; }
+template <int EPI>
+constexpr int swap_threads() { return 64 + 32 * swap_epi_warps<EPI>(); }
+
 constexpr int kSwWgStages = 2;
 constexpr int kSwWgStageBufBytes = 32 * 32 * 4;
 static_assert(kSwStages > kSwWgStages &&
-                  kGemmThreads / 32 - 2 == 8 && 8 * 2 * kSwWgStageBufBytes <= kSwStageBytes,
+                  swap_epi_warps<EPI_STORE_F32>() * 2 * kSwWgStageBufBytes <= kSwStageBytes,
               "the store staging buffers fill the weight-gradient pipeline's unused stage");
 
 struct SwapArgs {
@@ -238,7 +249,7 @@ __device__ __forceinline__ float warp_transpose_sum(float (&v)[32], int lane) {
 }
 
 template <int EPI, int LAYOUT>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(swap_threads<EPI>(), 1)
     moe_gemm_swap_kernel(const __grid_constant__ SwapMaps maps, const SwapArgs args) {
   constexpr int S = LAYOUT == kSwWgrad ? kSwWgStages : kSwStages;
   constexpr bool kSwiglu = EPI == EPI_SWIGLU || EPI == EPI_BWD_SWIGLU_SAVE;
@@ -307,7 +318,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       for (int b = 0; b < 2; ++b) {
         mbar_init(smem_addr(&s_tfull[b]), 1);
-        mbar_init(smem_addr(&s_tempty[b]), kEpiWarps * 32 * 2);
+        mbar_init(smem_addr(&s_tempty[b]), swap_epi_warps<EPI>() * 32 * 2);
       }
       for (int x = 0; x < 4; ++x) {
         mbar_init(smem_addr(&s_xfull[x]), 32);
@@ -441,7 +452,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;           // TMEM lane quarter
-    const int part = (warp - 2) >> 2; // token chunks part, part + 2, ...
+    constexpr int kParts = swap_epi_warps<EPI>() / 4;  // epilogue warps per TMEM lane quarter
+    const int part = (warp - 2) >> 2; // token chunks part, part + kParts, ...
     const int m = q * 32 + lane;      // accumulator lane = weight row inside this CTA
     const uint32_t tempty0 = mapa_shared(smem_addr(&s_tempty[0]), 0);
     const uint32_t tempty1 = mapa_shared(smem_addr(&s_tempty[1]), 0);
@@ -489,14 +501,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         (void)row0;
         const int col0 = col - lane;  // the warp's first output column (a multiple of 32)
 #pragma unroll 1
-        for (int j0 = 0; j0 < 4; j0 += 2) {
+        for (int j0 = 0; j0 < 8 / kParts; j0 += 2) {
           uint32_t r2[2][32];
-          MOE_TMEM_LD32(tacc + 32 * part + 64 * j0, r2[0]);
-          MOE_TMEM_LD32(tacc + 32 * part + 64 * (j0 + 1), r2[1]);
+          MOE_TMEM_LD32(tacc + 32 * (part + kParts * j0), r2[0]);
+          MOE_TMEM_LD32(tacc + 32 * (part + kParts * (j0 + 1)), r2[1]);
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
-            const int c = 32 * part + 64 * (j0 + j);
+            const int c = 32 * (part + kParts * (j0 + j));
             if (col0 < args.out_cols && c < t.nrows) {
               const uint32_t b = sc & 1u;
               if (lane == 0) bulk_wait_group_read<1>();  // the store that last used buffer b has read it
@@ -515,7 +527,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       } else
-      for (int c = 32 * part; c < t.n; c += 64) {
+      for (int c = 32 * part; c < t.n; c += 32 * kParts) {
         // Every value this chunk reads from memory (the input-gradient
         // epilogues' saved pre-activations, the addend, the fp32 sum added
         // onto) is requested first, all 32 rows together, so that the loads

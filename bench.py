@@ -171,18 +171,60 @@ E2E_NOTE = ("each step copies its own inputs in from pinned host memory and its 
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    """SM clocks, power and clock-event reasons sampled DURING the timed region.
+
+    NVML is read from a background thread every few milliseconds between
+    start() and stop(), so even a timed region of a few tens of milliseconds
+    (decode) gets samples; without NVML, nvidia-smi's own -lms loop is the
+    fallback.  Only reads: no clock or other setting is touched."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4}
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.out = None
+        self.thread = None
+        self.rows = []
+        self.stopping = False
+        self.nvml = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            handle = None
+            try:  # the CUDA device's own NVML handle, whatever CUDA_VISIBLE_DEVICES says
+                props = torch.cuda.get_device_properties(gpu_index)
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(gpu_index)
+            self.nvml = (pynvml, handle)
+        except Exception:
+            self.nvml = None
+
+    def _poll(self):
+        pynvml, h = self.nvml
+        smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        while not self.stopping:
+            try:
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                reasons = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                power = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                self.rows.append((float(sm), float(smax), power, int(reasons)))
+            except Exception:
+                pass
+            time.sleep(0.005)
 
     def start(self):
+        if self.nvml is not None:
+            import threading
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -192,6 +234,16 @@ class ClockSampler:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self.stopping = True
+            self.thread.join(timeout=5)
+            rows = self.rows
+            if not rows:
+                return None
+            reasons = sorted(n for n, bit in self.REASONS.items() if any(r[3] & bit for r in rows))
+            return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                    "reasons": reasons, "samples": len(rows), "power_w_max": max(r[2] for r in rows),
+                    "source": "nvml, every 5 ms during the timed region"}
         if self.proc is None:
             return None
         time.sleep(0.25)
@@ -204,12 +256,8 @@ class ClockSampler:
         rows = []
         for line in out.strip().splitlines():
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
+            if len(parts) >= 9:
                 rows.append(parts)
-            except ValueError:
-                pass
         if not rows:
             return None
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
@@ -220,7 +268,7 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
                 "reasons": reasons, "samples": len(rows),
-                "power_w_max": max(power) if power else None}
+                "power_w_max": max(power) if power else None, "source": "nvidia-smi -lms 200"}
 
 
 def source_hash(paths):

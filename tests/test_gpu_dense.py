@@ -54,11 +54,13 @@ def test_dense_edge_cases(B, over):
 
 def test_dense_full_size_sampled(B):
     """The GLaM dense layer between its MoE layers (T=8192, D=2048, H=8192,
-    GELU with biases) in the launch configuration the benchmark times."""
+    GELU with biases) in the launch configuration the benchmark times: the
+    first and last token of every 256-token tile (every tile of both GEMMs
+    holds one), plus random tokens."""
     cfg = ms.get_config("glam_dense_bf16")
     inp, _, y = run_dense(B, cfg, True)
-    rows = np.array(sorted({0, 1, 255, 256, 4095, 4096, 8190, 8191} |
-                           set(np.random.default_rng(0).integers(0, cfg["T"], 24).tolist())))
+    tiles = {r for t0 in range(0, cfg["T"], 256) for r in (t0, min(t0 + 255, cfg["T"] - 1))}
+    rows = np.array(sorted(tiles | set(np.random.default_rng(0).integers(0, cfg["T"], 24).tolist())))
     got = np64(y[torch.as_tensor(rows, device=y.device)])
     check_y(dict(cfg, named=False), got, dense_reference(cfg, inp, rows, True))
 

@@ -220,15 +220,16 @@ __device__ __forceinline__ void swap_store(const SwapArgs& a, size_t base, int c
     static_cast<__nv_bfloat16*>(a.out)[base + row * a.ldo + col] = __float2bfloat16_rn(v);
 }
 
-// GELU (tanh form) and its derivative from one exponential: with
-// s = 0.5 (1 + tanh u) = 1 / (1 + e^{-2u}), GELU(v) = v s and GELU'(v) =
-// s + v 2 s (1 - s) c (1 + 3 * 0.044715 v^2), since 1 - tanh^2 u = 4 s (1 - s).
+// GELU (tanh form) and its derivative from one tanh: with t = tanh u,
+// u = c (v + 0.044715 v^3) and s = 0.5 (1 + t), GELU(v) = v s and
+// GELU'(v) = s + 0.5 v (1 - t^2) c (1 + 3 * 0.044715 v^2).
 __device__ __forceinline__ void gelu_tanh_and_grad_fast(float v, float& g, float& dg) {
   const float c = 0.7978845608028654f;
   const float u = c * fmaf(0.044715f * v, v * v, v);
-  const float sg = __fdividef(1.0f, 1.0f + __expf(-2.0f * u));
-  g = v * sg;
-  dg = fmaf(v * 2.0f * sg * (1.0f - sg) * c, fmaf(3.0f * 0.044715f, v * v, 1.0f), sg);
+  const float t = tanh_hw(u);
+  const float s = fmaf(0.5f, t, 0.5f);  // 0.5 (1 + tanh u)
+  g = v * s;
+  dg = fmaf(0.5f * v * fmaf(-t, t, 1.0f) * c, fmaf(3.0f * 0.044715f, v * v, 1.0f), s);
 }
 
 // Sum over the warp's 32 lanes of v[i] for every i, in 31 shuffles: after

@@ -93,6 +93,7 @@ def test_group_limited_full_size(B):
     ("glm_small_bf16", dict(e_bias=("const", 0.0), alpha=1.0)),
     ("glm_medium_bf16", dict(e_bias=("zipf", 1.1, 1.0))),  # literal beta = 1: most experts empty
     ("glam_tiny_f32", dict(T=1)),
+    ("glam_small_bf16", dict(T=5)),                      # GELU experts on the few-rows (tokens-on-M) path
     ("glm_small_bf16", dict(n_group=16, topk_group=4)),  # one expert per group
     ("glm_small_bf16", dict(n_group=4, topk_group=4)),   # every group kept
     ("glm_small_bf16", dict(n_group=4, topk_group=1)),   # k = the whole kept group

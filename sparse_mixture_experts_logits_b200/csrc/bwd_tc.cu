@@ -85,14 +85,16 @@ __global__ void gather_pad_kernel(const uint4* __restrict__ src, const int32_t* 
 }
 
 // Zero the padding rows [offsets_pad[e] + counts[e], offsets_pad[e + 1]) of a
-// [rows, vecs x 16 B] buffer; block per expert.
+// [rows, vecs x 16 B] buffer; blockIdx.x is the expert, blockIdx.y a share of its rows.
 __global__ void zero_pad_rows_kernel(const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets_pad,
                                      uint4* __restrict__ buf, long long rows_cap, int vecs) {
   const int e = blockIdx.x;
   const long long r0 = min(rows_cap, static_cast<long long>(offsets_pad[e]) + max(counts[e], 0));
   const long long r1 = min(rows_cap, static_cast<long long>(offsets_pad[e + 1]));
   const long long n = (r1 - r0) * vecs;
-  for (long long i = threadIdx.x; i < n; i += blockDim.x) buf[r0 * vecs + i] = make_uint4(0u, 0u, 0u, 0u);
+  for (long long i = static_cast<long long>(blockIdx.y) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.y) * blockDim.x)
+    buf[r0 * vecs + i] = make_uint4(0u, 0u, 0u, 0u);
 }
 
 // dw[t, j] = sum_p parts[q, p] (+ <dy_t, b2_e>) with q = slot_pad[t, j], in a
@@ -142,6 +144,53 @@ __global__ void colsum_bf16_kernel(const __nv_bfloat16* __restrict__ Y, long lon
   out[static_cast<long long>(g) * N + n] = s;
 }
 
+// The same sums, two columns per thread (N and ldy even, Y 4-byte aligned):
+// each warp reads 128 contiguous bytes of a row, and the loads of 16 rows are
+// issued before any of them is added, so that a thread keeps 16 requests in
+// flight instead of one.  Each column still adds its rows one by one in row
+// order, so the sums are the scalar kernel's bit for bit.
+__global__ void colsum_bf16x2_kernel(const __nv_bfloat162* __restrict__ Y, long long ldy2,
+                                     const float* __restrict__ scale, const int32_t* __restrict__ offsets,
+                                     long long rows_cap, int N2, float2* __restrict__ out) {
+  constexpr int kRows = 16;
+  const int g = blockIdx.y;
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N2) return;
+  const long long b = min(rows_cap, static_cast<long long>(max(offsets[g], 0)));
+  const long long e = min(rows_cap, static_cast<long long>(max(offsets[g + 1], 0)));
+  float s0 = 0.f, s1 = 0.f;
+  long long r = b;
+  for (; r + kRows <= e; r += kRows) {
+    __nv_bfloat162 v[kRows];
+#pragma unroll
+    for (int i = 0; i < kRows; ++i) v[i] = Y[(r + i) * ldy2 + n];
+#pragma unroll
+    for (int i = 0; i < kRows; ++i) {
+      const float2 f = __bfloat1622float2(v[i]);
+      if (scale != nullptr) {
+        const float c = scale[r + i];
+        s0 = fmaf(c, f.x, s0);
+        s1 = fmaf(c, f.y, s1);
+      } else {
+        s0 += f.x;
+        s1 += f.y;
+      }
+    }
+  }
+  for (; r < e; ++r) {
+    const float2 f = __bfloat1622float2(Y[r * ldy2 + n]);
+    if (scale != nullptr) {
+      const float c = scale[r];
+      s0 = fmaf(c, f.x, s0);
+      s1 = fmaf(c, f.y, s1);
+    } else {
+      s0 += f.x;
+      s1 += f.y;
+    }
+  }
+  out[static_cast<long long>(g) * N2 + n] = make_float2(s0, s1);
+}
+
 // out[g, :] = 0 (per_group floats) for every g with counts[g] == 0.
 __global__ void zero_empty_groups_kernel(const int32_t* __restrict__ counts, long long per_group,
                                          float* __restrict__ out) {
@@ -185,7 +234,11 @@ cudaError_t launch_zero_pad_rows(const int32_t* counts, const int32_t* offsets_p
                                  long long rows_cap, int cols_bf16, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
   if (cols_bf16 % 8 != 0) return cudaErrorInvalidValue;
-  zero_pad_rows_kernel<<<M, 256, 0, s>>>(counts, offsets_pad, static_cast<uint4*>(buf), rows_cap, cols_bf16 / 8);
+  // A group pads at most 63 rows: 16 blocks per group cover them in a few
+  // rounds of 16-byte stores (one block per group left the stores waiting
+  // one after another).
+  zero_pad_rows_kernel<<<dim3(M, 16), 256, 0, s>>>(counts, offsets_pad, static_cast<uint4*>(buf), rows_cap,
+                                                   cols_bf16 / 8);
   return cudaGetLastError();
 }
 
@@ -203,6 +256,13 @@ cudaError_t launch_colsum_bf16(const void* Y, long long ldy, const float* scale,
                                long long rows_cap, int N, float* out, cudaStream_t s) {
   if (G <= 0 || N <= 0) return cudaSuccess;
   if (G > 65535) return cudaErrorInvalidValue;
+  if (N % 2 == 0 && ldy % 2 == 0 && reinterpret_cast<uintptr_t>(Y) % 4 == 0 &&
+      reinterpret_cast<uintptr_t>(out) % 8 == 0) {
+    dim3 grid((N / 2 + 255) / 256, G);
+    colsum_bf16x2_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat162*>(Y), ldy / 2, scale, offsets,
+                                              rows_cap, N / 2, reinterpret_cast<float2*>(out));
+    return cudaGetLastError();
+  }
   dim3 grid((N + 255) / 256, G);
   colsum_bf16_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(Y), ldy, scale, offsets, rows_cap, N,
                                           out);

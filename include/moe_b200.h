@@ -23,9 +23,12 @@
  *  - Every pointer argument is a DEVICE pointer to caller-owned memory on
  *    the current device, except the descriptor and weight structs, which are
  *    host structs (the pointers inside them are device pointers).  The
- *    library never allocates, frees or synchronises; every call only
+ *    library never allocates memory, frees or synchronises; every call only
  *    enqueues kernels on `stream` (a cudaStream_t; NULL = legacy default
- *    stream) and returns.
+ *    stream) and returns.  The one exception to "only on `stream`" is
+ *    moe_forward's decode-size shared expert (below): it may run on an
+ *    internal stream that waits for `stream` and that `stream` waits for
+ *    before the combine, so the call's ordering is the same.
  *  - Scratch memory ("workspace") is caller-provided; each entry point has a
  *    *_workspace_size query.  Workspaces must be 256-byte aligned.  Calls
  *    that share a workspace must be ordered on one stream.
@@ -326,7 +329,16 @@ moe_status_t moe_workspace_layout(const moe_layer_desc_t* d, moe_ws_layout_t* ou
  * I_sh > 0, its output kept in fp32) and the combine, which adds each
  * token's k weighted expert rows and its shared-expert row in fp32 and
  * rounds once.  All stages run back to back on `stream` with no host
- * synchronisation. */
+ * synchronisation, with one exception: in bf16 with a shared expert and
+ * T * k < 4 M (the decode sizes, where each expert gets a handful of rows)
+ * the shared expert's two GEMMs read only x, so they run on an internal
+ * stream beside the routing stage.  That stream (one per device and CUDA
+ * context, with two events, made on the first such call that is not
+ * inside a stream capture) waits for `stream` before them, and `stream`
+ * waits for it before the combine; a call that returns early still joins
+ * it.  Inside a capture the fork and join are captured as graph branches;
+ * without the stream (not yet made, or a creation that failed) everything
+ * runs on `stream`.  The result is the same either way. */
 moe_status_t moe_forward(const moe_layer_desc_t* d, const moe_weights_t* w,
                          const void* x, void* y, void* ws, size_t ws_bytes, void* stream);
 
@@ -350,7 +362,11 @@ moe_status_t moe_forward_add(const moe_layer_desc_t* d, const moe_weights_t* w,
  * done; 5: routed experts' second GEMM done; 6: shared expert's first GEMM
  * done; 7: shared expert's second GEMM done; 8: combine (the k routed rows
  * of every token plus its shared-expert row) done.  Stages a
- * layer does not have record their event right after the previous one. */
+ * layer does not have record their event right after the previous one.
+ * When the shared expert runs beside the routing stage (moe_forward),
+ * events 6 and 7 are recorded on `stream` after it joins: stage 6 then
+ * holds only the part of the shared expert that the routed stages did not
+ * cover, and stage 7 is empty. */
 
 /* moe_forward, recording `events[i]` (cudaEvent_t handles created by the
  * caller, n_events == MOE_NUM_STAGE_EVENTS) on `stream` at each boundary. */

@@ -4,6 +4,7 @@
 #include <cmath>
 #include <atomic>
 #include <cstring>
+#include <mutex>
 
 #include "gemm_sm100.cuh"
 #include <nvtx3/nvToolsExt.h>
@@ -50,6 +51,12 @@ struct Carve {
 };
 
 inline size_t esize(int dtype) { return dtype == MOE_DTYPE_BF16 ? 2 : 4; }
+
+// A handful of rows per expert (decode): the routed GEMMs take the
+// tokens-on-M path of run_experts.
+inline bool few_rows(const moe_layer_desc_t* d) {
+  return static_cast<long long>(d->T) * d->k < 4ll * d->M;
+}
 
 inline moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 #define MOE_TRY(expr)                          \
@@ -269,8 +276,7 @@ moe_status_t run_experts(const moe_layer_desc_t* d, const moe_weights_t* w, cons
   // A handful of rows per expert (decode): tokens on M with single-CTA MMAs. The 128-row token
   // tile is mostly padding, but each CTA streams its own slice of the touched experts'
   // weights once (measured: GLM-4.5 decode expert GEMMs 0.837 -> 0.810 ms).
-  const bool few_rows = static_cast<long long>(d->T) * d->k < 4ll * d->M;
-  if (d->dtype == MOE_DTYPE_BF16 && few_rows) {
+  if (d->dtype == MOE_DTYPE_BF16 && few_rows(d)) {
     MOE_CUDA(launch_gather_rows(x, row_token, offsets + d->M, x_perm, pairs, d->T, d->D, 2, status, s));
     MOE_TRY(mk.at(3));
     GemmLaunch g1{};
@@ -431,6 +437,108 @@ moe_status_t run_shared(const moe_layer_desc_t* d, const moe_weights_t* w, const
   MOE_TRY(mk.at(7));
   return MOE_OK;
 }
+
+// One internal stream and two events per device and CUDA context, made on
+// the first call that is not inside a stream capture.  At decode sizes the
+// forward runs the shared expert there, beside the routing stage, and joins
+// it back before the combine.  Lookups are serialised by `mu`, and a caller
+// holds `mu` from the fork to the join, so that concurrent callers never
+// interleave their records of the two events.
+struct SideStream {
+  cudaStream_t st = nullptr;
+  cudaEvent_t fork = nullptr;
+  cudaEvent_t join = nullptr;
+  CUcontext ctx = nullptr;
+  std::mutex mu;
+};
+
+CUcontext current_ctx() {
+  using Fn = CUresult (*)(CUcontext*);
+  static std::once_flag once;
+  static Fn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<Fn>(p);
+  });
+  CUcontext c = nullptr;
+  if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// The device's side stream, or nullptr (the caller then runs everything on
+// its own stream): an unknown context, a capture in progress when the
+// stream does not exist yet, or a failed creation.
+SideStream* side_stream(cudaStream_t s) {
+  constexpr int kDevices = 64;
+  static SideStream sides[kDevices];
+  static std::mutex make_mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevices) return nullptr;
+  const CUcontext ctx = current_ctx();
+  if (ctx == nullptr) return nullptr;
+  SideStream& x = sides[dev];
+  std::lock_guard<std::mutex> lock(make_mu);
+  if (x.st != nullptr && x.ctx == ctx) return &x;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return nullptr;
+  // a context made anew invalidated the old handles: they are dropped, not destroyed
+  x.st = nullptr;
+  x.fork = x.join = nullptr;
+  cudaStream_t st = nullptr;
+  cudaEvent_t f = nullptr, j = nullptr;
+  if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+  if (cudaEventCreateWithFlags(&f, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&j, cudaEventDisableTiming) != cudaSuccess) {
+    if (f != nullptr) cudaEventDestroy(f);
+    cudaStreamDestroy(st);
+    return nullptr;
+  }
+  x.fork = f;
+  x.join = j;
+  x.ctx = ctx;
+  x.st = st;
+  return &x;
+}
+
+// Holds a side stream from the fork to the join.  The destructor joins it
+// back if the caller returns early, so that no work the caller launched on
+// the side stream can outlive the call's view of its workspace.
+class SideFork {
+ public:
+  SideFork() = default;
+  SideFork(const SideFork&) = delete;
+  SideFork& operator=(const SideFork&) = delete;
+  ~SideFork() { (void)join(); }
+  // Makes the side stream wait for everything enqueued on s so far.
+  moe_status_t fork(SideStream* side, cudaStream_t s) {
+    lock_ = std::unique_lock<std::mutex>(side->mu);
+    side_ = side;
+    s_ = s;
+    forked_ = true;
+    if (cudaEventRecord(side->fork, s) != cudaSuccess) return MOE_ERR_CUDA;
+    return cudaStreamWaitEvent(side->st, side->fork, 0) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  }
+  // Makes s wait for everything enqueued on the side stream so far.
+  moe_status_t join() {
+    if (!forked_) return MOE_OK;
+    forked_ = false;
+    moe_status_t st = MOE_OK;
+    if (cudaEventRecord(side_->join, side_->st) != cudaSuccess ||
+        cudaStreamWaitEvent(s_, side_->join, 0) != cudaSuccess)
+      st = MOE_ERR_CUDA;
+    lock_.unlock();
+    return st;
+  }
+
+ private:
+  std::unique_lock<std::mutex> lock_;
+  SideStream* side_ = nullptr;
+  cudaStream_t s_ = nullptr;
+  bool forked_ = false;
+};
 
 }  // namespace
 
@@ -775,6 +883,23 @@ static moe_status_t forward_impl(const moe_layer_desc_t* d, const moe_weights_t*
   void* out_perm = at<void*>(ws, L.pub.out_perm);
   Range whole("moe_forward");
   MOE_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
+  // At decode sizes the shared expert's two GEMMs stream their weights
+  // through a few CTA pairs, each waiting on its whole K in turn, while the
+  // routing stage's small kernels leave most SMs idle.  The shared expert
+  // reads only x, so it runs on the side stream under the routing stage and
+  // joins before the combine.  Its outputs go to their own workspace
+  // regions, which no other stage touches.
+  void* y_sh = d->I_sh > 0 ? at<void*>(ws, L.y_sh) : nullptr;
+  SideFork shared_fork;
+  bool shared_done = false;
+  if (d->I_sh > 0 && d->dtype == MOE_DTYPE_BF16 && few_rows(d)) {
+    if (SideStream* side = side_stream(s)) {
+      Range r("moe.shared_expert");
+      MOE_TRY(shared_fork.fork(side, s));
+      MOE_TRY(run_shared(d, w, x, y_sh, at<void*>(ws, L.h_sh), true, status, side->st));
+      shared_done = true;
+    }
+  }
   MOE_TRY(mk.at(0));
   {
     Range r("moe.route");
@@ -798,10 +923,12 @@ static moe_status_t forward_impl(const moe_layer_desc_t* d, const moe_weights_t*
     MOE_TRY(run_experts(d, w, x, offsets, row_token, row_w, out_perm, at<void*>(ws, L.x_perm),
                         at<void*>(ws, L.h), status, s, mk, by_token ? slot_of : nullptr));
   }
-  void* y_sh = nullptr;
-  if (d->I_sh > 0) {
+  if (shared_done) {
+    MOE_TRY(shared_fork.join());
+    MOE_TRY(mk.at(6));
+    MOE_TRY(mk.at(7));
+  } else if (d->I_sh > 0) {
     Range r("moe.shared_expert");
-    y_sh = at<void*>(ws, L.y_sh);
     MOE_TRY(run_shared(d, w, x, y_sh, at<void*>(ws, L.h_sh), true, status, s, mk));
   } else {
     MOE_TRY(mk.at(6));

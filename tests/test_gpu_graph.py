@@ -1,6 +1,11 @@
 """The forward pass makes no host synchronisation and no allocation, so it
 can be captured once into a CUDA graph and replayed (the decode loop's way
-of removing launch overhead), and it runs on any stream."""
+of removing launch overhead), and it runs on any stream.  At decode sizes
+the shared expert runs on the library's internal side stream: several host
+threads driving layers on their own streams at once must still get the
+results of one-at-a-time calls."""
+import threading
+
 import pytest
 import torch
 
@@ -73,3 +78,42 @@ def test_forward_on_a_side_stream(B):
         layer.forward(inp["x"], y=y1, stream=s)
     s.synchronize()
     assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))
+
+
+def test_concurrent_decode_forwards_on_own_streams(B):
+    """Two host threads, each with its own decode-size layer (shared expert,
+    T * k < 4 M), workspace and stream, run forwards at the same time; the
+    ctypes calls release the GIL, so the two fork to the side stream and
+    join back concurrently.  Every y equals the one-at-a-time y bit for
+    bit."""
+    cfg = ms.get_config("glm45_decode_bf16")
+    assert cfg["T"] * cfg["k"] < 4 * cfg["M"] and cfg["I_sh"] > 0
+    inp = ms.layer_inputs(cfg, "cuda")
+    layers = [B.MoELayer(cfg, inp), B.MoELayer(cfg, inp)]
+    xs = [inp["x"], ms.normal((cfg["T"], cfg["D"]), 1.0, ms._key(cfg, "x2"), "cuda", ms.act_dtype(cfg))]
+    ref = [layers[i].forward(xs[i]) for i in range(2)]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = [[torch.empty_like(xs[i]) for _ in range(6)] for i in range(2)]
+    for i in range(2):
+        streams[i].wait_stream(torch.cuda.current_stream())
+    errors = []
+
+    def run(i):
+        try:
+            for y in outs[i]:
+                layers[i].forward(xs[i], y=y, stream=streams[i])
+        except Exception as e:  # reported below, on the main thread
+            errors.append(e)
+
+    threads = [threading.Thread(target=run, args=(i,)) for i in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    torch.cuda.synchronize()
+    assert not errors
+    for i in range(2):
+        assert layers[i].device_status() == 0
+        for y in outs[i]:
+            assert torch.equal(y.view(torch.int16), ref[i].view(torch.int16))

@@ -81,6 +81,7 @@ def test_group_limited_full_size(B):
 
 @pytest.mark.parametrize("name,over", [
     ("glm_small_bf16", dict(T=1)),
+    ("glm_small_bf16", dict(T=15)),                      # few rows: the shared expert on the side stream
     ("glm_small_bf16", dict(T=128)),
     ("glm_small_bf16", dict(T=129)),
     ("glm_small_bf16", dict(T=64, I_sh=208)),            # a shared gate/up width not a multiple of 32

@@ -46,7 +46,8 @@ enum GemmEpilogue : int {
   EPI_BIAS_ADD = 6,    // out (layer dtype) = acc + b[n] + addend[r, n]   (dense FFN down projection;
                        //            bias and addend optional)
   // Backward (tokens-on-N kernel only):
-  EPI_BWD_GELU_SAVE = 7,    // v = acc + b1: out = v (fp32), out2 = GELU(v), out3 = row_scale[r] GELU(v) (bf16)
+  EPI_BWD_GELU_SAVE = 7,    // v = acc + b1: out = v (fp32), out2 = GELU(v), out3 = row_scale[r] GELU(v) (bf16;
+                            // out2, out3 optional)
   EPI_BWD_SWIGLU_SAVE = 8,  // g, u: out[., n] = g, out[., I + n] = u (fp32), out2 = SiLU(g) u, out3 = w out2
   EPI_BWD_GELU_DACT = 9,    // G = acc, h = aux[r, n]: out = w G GELU'(h); parts += G GELU(h)
   EPI_BWD_SWIGLU_DACT = 10, // G = acc, g = aux[r, n], u = aux[r, I + n], a = SiLU(g) u, da = w G:

@@ -609,7 +609,7 @@ __global__ void __launch_bounds__(swap_threads<EPI>(), 1)
                   const size_t row = row0 + c + i;
                   hp[row * args.ldo + col] = g;
                   hp[row * args.ldo + args.half_cols + col] = u[i];
-                  args.out2[row * args.ldo2 + col] = __float2bfloat16_rn(a);
+                  if (args.out2 != nullptr) args.out2[row * args.ldo2 + col] = __float2bfloat16_rn(a);
                   if (args.out3 != nullptr) args.out3[row * args.ldo2 + col] = __float2bfloat16_rn(w * a);
                 }
               }
@@ -661,7 +661,7 @@ __global__ void __launch_bounds__(swap_threads<EPI>(), 1)
               if (col_ok && i < nv) {
                 const size_t row = row0 + c + i;
                 static_cast<float*>(args.out)[row * args.ldo + col] = v;
-                args.out2[row * args.ldo2 + col] = __float2bfloat16_rn(a);
+                if (args.out2 != nullptr) args.out2[row * args.ldo2 + col] = __float2bfloat16_rn(a);
                 if (args.out3 != nullptr) args.out3[row * args.ldo2 + col] = __float2bfloat16_rn(w * a);
               }
             } else {

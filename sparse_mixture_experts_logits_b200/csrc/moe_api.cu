@@ -1011,7 +1011,7 @@ struct BwdWs {
   size_t xp, hpre, act, dO, da, dxp, dwp, dl, hs, as, das, dxs, total;
   // tensor-core path (bf16): the padded dispatch order and its bf16 tensors
   long long rows_pad;
-  size_t offp, slotp, rtp, rwp, xpp, dypp, hpb, ab, awb, dhb, dxpp, parts, hsb, asb, dhsb, rpart, dlb;
+  size_t offp, slotp, rtp, rwp, xpp, dypp, hpb, awb, dhb, dxpp, parts, hsb, asb, dhsb, rpart, dlb;
 };
 
 // Chunks of the token sum in the router's weight gradient dW_r = x^T dlogits
@@ -1050,7 +1050,6 @@ BwdWs backward_layout_tc(const moe_layer_desc_t* d) {
   L.xpp = c.take(P * D * 2);
   L.dypp = c.take(P * D * 2);
   L.hpb = c.take(P * n1 * 4);  // fp32 pre-activations: they feed act' and <G, a> unrounded
-  L.ab = c.take(P * Ha * 2);
   L.awb = c.take(P * Ha * 2);
   L.dhb = c.take(P * n1 * 2);
   L.dxpp = c.take(P * D * 4);
@@ -1188,7 +1187,6 @@ moe_status_t backward_tc_impl(const moe_layer_desc_t* d, const moe_weights_t* w,
   void* xpp = at<void*>(ws, L.xpp);
   void* dypp = at<void*>(ws, L.dypp);
   void* hpb = at<void*>(ws, L.hpb);
-  void* ab = at<void*>(ws, L.ab);
   void* awb = at<void*>(ws, L.awb);
   void* dhb = at<void*>(ws, L.dhb);
   float* dxpp = at<float*>(ws, L.dxpp);
@@ -1218,7 +1216,8 @@ moe_status_t backward_tc_impl(const moe_layer_desc_t* d, const moe_weights_t* w,
   }
   {
     Range r("moe.experts_backward");
-    // recompute: h (fp32), a = act(h) and aw = w a (bf16 operands of the weight gradients)
+    // recompute: h (fp32) and aw = w a (bf16, the operand of dW2).  The unscaled a is not kept:
+    // the input-gradient epilogue forms <G, a> from h itself.
     SwapLaunch ga{};
     if (swiglu) {
       ga = bwd_swap(EPI_BWD_SWIGLU_SAVE, kSwFwd, w->w1, 1ll * M * n1, xpp, P, D, M, offp, counts, P, Ha, hpb, n1,
@@ -1236,7 +1235,7 @@ moe_status_t backward_tc_impl(const moe_layer_desc_t* d, const moe_weights_t* w,
       ga.w_rows_per_group = Ha;
       ga.bias = biases ? w->b1 : nullptr;
     }
-    ga.out2 = ab;
+    ga.out2 = nullptr;
     ga.out3 = awb;
     ga.ldo2 = Ha;
     ga.row_scale = rwp;

@@ -150,6 +150,16 @@ __device__ __forceinline__ void token_tiling(int cnt, int& width, int& ntiles) {
   ntiles = (cnt + width - 1) / width;
 }
 
+// Tile of round rd for CTA pair `unit`: rounds of `units` consecutive tiles,
+// dealt in alternating directions, so that the pair that takes the last
+// tile of one round takes the first of the next.  Tile costs vary with the
+// width of each expert's token tiles; dealing every round in the same
+// direction gave the low-numbered pairs the larger share (same-box A/B:
+// GLaM layer 1.32 -> 1.29 ms, GLM-4.5 prefill 7.27-7.36 -> 7.19-7.25 ms).
+__device__ __forceinline__ int swap_tile_at(int rd, int unit, int units) {
+  return rd * units + ((rd & 1) ? units - 1 - unit : unit);
+}
+
 struct SwapTile {
   int g, wt, tok0, nrows, n;  // group, weight tile, first token, rows, MMA N
   int nkb;                    // k-blocks of this tile (kSwWgrad: the group's rows / 64)
@@ -353,7 +363,7 @@ __global__ void __launch_bounds__(swap_threads<EPI>(), 1)
     // -------------------------------------------------------- TMA producer
     uint32_t s = 0, ph = 0;
     bool ok = true;
-    for (int tile = unit; ok && tile < total; tile += units) {
+    for (int rd = 0, tile = unit; ok && tile < total; ++rd, tile = swap_tile_at(rd, unit, units)) {
       const SwapTile t = swap_decode<LAYOUT>(tile, G, s_tstart, s_cnt, args, num_kb);
       // kSwFwd / kSwDgrad: B = this CTA's half of the token tile, K-major rows.
       // kSwWgrad: B = this CTA's 128 of the tile's 256 B columns, rows of the segment.
@@ -411,7 +421,7 @@ __global__ void __launch_bounds__(swap_threads<EPI>(), 1)
       const uint64_t da0 = kAMn ? sw128_mnmajor_desc(smem_base, 64 * kBK * 2) : sw128_kmajor_desc(smem_base);
       const uint64_t db0 = kBMn ? sw128_mnmajor_desc(smem_base + kSwKB * kSwATileBytes, 64 * kBK * 2)
                                 : sw128_kmajor_desc(smem_base + kSwKB * kSwATileBytes);
-      for (int tile = unit; ok && tile < total; tile += units, ++it) {
+      for (int rd = 0, tile = unit; ok && tile < total; ++rd, tile = swap_tile_at(rd, unit, units), ++it) {
         const SwapTile t = swap_decode<LAYOUT>(tile, G, s_tstart, s_cnt, args, num_kb);
         const uint32_t idesc = umma_idesc_bf16_major(256, t.n, kAMn ? 1 : 0, kBMn ? 1 : 0);
         const uint32_t buf = it & 1u;
@@ -466,7 +476,7 @@ __global__ void __launch_bounds__(swap_threads<EPI>(), 1)
     const uint32_t stg = smem_base + kSwWgStages * kSwStageBytes + (warp - 2) * 2 * kSwWgStageBufBytes;
     float* stgp = reinterpret_cast<float*>(dyn_smem + (stg - smem_addr(dyn_smem)));
     bool ok = true;
-    for (int tile = unit; ok && tile < total; tile += units, ++it) {
+    for (int rd = 0, tile = unit; ok && tile < total; ++rd, tile = swap_tile_at(rd, unit, units), ++it) {
       const SwapTile t = swap_decode<LAYOUT>(tile, G, s_tstart, s_cnt, args, num_kb);
       const uint32_t buf = it & 1u;
       const uint32_t tph = (it >> 1) & 1u;

@@ -170,6 +170,14 @@ E2E_NOTE = ("each step copies its own inputs in from pinned host memory and its 
             "alternate so that the copies run on the copy engines under the neighbouring steps' compute")
 
 
+def wait_on_last(events):
+    """Blocks until the last of `events` completes by polling it with short
+    sleeps: the host thread holds no lock while it waits, so the clock
+    sampler keeps reading NVML through the timed region."""
+    while events and not events[-1].query():
+        time.sleep(0.0005)
+
+
 class ClockSampler:
     """SM clocks, power and clock-event reasons sampled DURING the timed region.
 
@@ -393,6 +401,7 @@ def run_ours(args):
         B.moe_forward_profiled(layer.desc, layer.weights, x.data_ptr(), y.data_ptr(), layer.ws_ptr,
                                layer.ws_bytes, sh, [e.cuda_event for e in stage_ev[i]])
         ends[i].record(stream)
+    wait_on_last(ends)  # sleeps, so that the clock sampler thread gets the GIL
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
     if dist is not None:
@@ -619,6 +628,7 @@ def run_dense(args):
         B.moe_dense_ffn_profiled(layer.desc, *wargs, x.data_ptr(), a.data_ptr(), y.data_ptr(), layer.ws_ptr,
                                  layer.ws_bytes, sh, [e.cuda_event for e in ev[i]])
         ends[i].record(stream)
+    wait_on_last(ends)  # sleeps, so that the clock sampler thread gets the GIL
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
     if dist is not None:
@@ -942,6 +952,7 @@ def run_backward(args):
         starts[i].record(stream)
         layer.backward(inp["x"], dy, grads=grads)
         ends[i].record(stream)
+    wait_on_last(ends)  # sleeps, so that the clock sampler thread gets the GIL
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
     if dist is not None:
@@ -1031,6 +1042,7 @@ def run_ep(args):
         starts[i].record(stream)
         layer.forward(x)
         ends[i].record(stream)
+    wait_on_last(ends)  # sleeps, so that the clock sampler thread gets the GIL
     torch.cuda.synchronize()
     launches = K * layer.launch_count(T)
     bufs = layer.buffers(T, x.dtype)

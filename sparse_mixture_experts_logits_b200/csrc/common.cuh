@@ -91,6 +91,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with acquire at cluster scope: for a phase completed by another
+// CTA's release arrive, after which this thread reads data that CTA wrote
+// into this CTA's shared memory.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Non-blocking test of the same phase (the cheap first look: a completed
 // phase returns without the suspend/wake-up of try_wait).
 __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
@@ -138,6 +153,35 @@ __device__ __forceinline__ bool mbar_wait_all(uint32_t bar, uint32_t parity, vol
                                               int* status, uint64_t limit_ns = kWaitTimeoutNs) {
   const bool ok = mbar_wait(bar, parity, abort, status, limit_ns);
   return __all_sync(0xffffffffu, ok);
+}
+
+// mbar_wait_all with cluster-scope acquire (see mbar_try_wait_cluster).
+__device__ __forceinline__ bool mbar_wait_all_cluster(uint32_t bar, uint32_t parity, volatile int* abort,
+                                                      int* status) {
+  bool ok = true;
+  uint64_t t0 = 0;
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait_cluster(bar, parity)) break;
+    if ((n & 31u) == 0) {
+      if (*abort) { ok = false; break; }
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitTimeoutNs) {
+        *abort = 1;
+        set_status(status, MOE_DEVERR_TIMEOUT);
+        ok = false;
+        break;
+      }
+    }
+  }
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Stores a 32-bit value at a shared::cluster address (another CTA's shared
+// memory, from mapa_shared).
+__device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, int v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 
 // Same, bounded by time only (used while draining after an abort).

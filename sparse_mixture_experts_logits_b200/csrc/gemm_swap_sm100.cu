@@ -172,6 +172,7 @@ cudaError_t launch_gemm_swap(const SwapLaunch& L, cudaStream_t s) {
   a.ld_parts = L.ld_parts;
   a.half_cols = L.half_cols;
   a.counts = L.counts;
+  a.tile_ctr = L.tile_ctr;
   if (L.layout == kSwWgrad) {
     const long long tiles_ub = static_cast<long long>(L.num_groups) * L.w_tiles * L.b_tiles;
     if (L.epi != EPI_STORE_F32) return cudaErrorInvalidValue;

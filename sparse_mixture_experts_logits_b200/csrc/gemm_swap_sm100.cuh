@@ -139,6 +139,11 @@ struct SwapArgs {
   // optional [G]: rows of group g's segment to compute (the segment starts
   // at offsets[g] and may be longer: zero padding that no tile covers)
   const int* counts;
+  // optional: a counter that is 0 when the launch starts.  Given, and when
+  // at least a quarter of the groups with rows have fewer than 64 rows, the
+  // CTA pairs claim tiles from it in index order as they become free
+  // (dynamic schedule); otherwise they take fixed rounds (swap_tile_at).
+  int* tile_ctr;
 };
 
 // Token tiles of a segment of `cnt` rows: ceil(cnt / 256) tiles of equal
@@ -278,9 +283,16 @@ __global__ void __launch_bounds__(swap_threads<EPI>(), 1)
   __shared__ __align__(8) uint64_t s_xfull[4];
   __shared__ __align__(8) uint64_t s_xempty[4];
   __shared__ __align__(8) uint64_t s_drain;
+  // dynamic schedule: the leader CTA's producer publishes each claimed tile
+  // into this ring in both CTAs of the pair
+  constexpr int kTq = 8;
+  __shared__ int s_tq[kTq];
+  __shared__ __align__(8) uint64_t s_tq_full[kTq];   // one arrival: the leader's producer
+  __shared__ __align__(8) uint64_t s_tq_empty[kTq];  // leader's: every reader releases the slot
   __shared__ uint32_t s_tmem_base;
   __shared__ int s_abort;
   __shared__ int s_total;
+  __shared__ int s_dyn;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -307,9 +319,13 @@ __global__ void __launch_bounds__(swap_threads<EPI>(), 1)
   __syncthreads();
   if (warp == 0) {
     int carry = 0;
+    int busy = 0, narrow = 0;  // groups with rows; of those, groups of fewer than 64 rows
     for (int base = 0; base < G; base += 32) {
       const int g = base + lane;
-      const int v = g < G ? swap_group_tiles<LAYOUT>(s_cnt[g], args) : 0;
+      const int c = g < G ? s_cnt[g] : 0;
+      busy += __popc(__ballot_sync(0xffffffffu, c > 0));
+      narrow += __popc(__ballot_sync(0xffffffffu, c > 0 && c < 64));
+      const int v = g < G ? swap_group_tiles<LAYOUT>(c, args) : 0;
       int incl = v;
 #pragma unroll
       for (int d = 1; d < 32; d <<= 1) {
@@ -323,6 +339,14 @@ __global__ void __launch_bounds__(swap_threads<EPI>(), 1)
       s_tstart[G] = carry;
       s_total = carry;
       s_abort = 0;
+      // Claim tiles dynamically when at least a quarter of the groups with
+      // rows are narrow: their tiles stream a whole weight tile for a few
+      // rows, at a cost that depends on what runs beside them, which fixed
+      // rounds cannot balance (GLM-5 skewed prefill: 40% narrow, expert
+      // GEMM1 6.28 -> 5.77 ms).  With few narrow groups the fixed rounds
+      // were as fast or faster (GLaM: none, GEMM1 0.547 against 0.583 ms
+      // dynamic; GLM-4.5: 19%, within noise).
+      s_dyn = args.tile_ctr != nullptr && narrow > 0 && 4 * narrow >= busy;
       for (int s = 0; s < S; ++s) {
         mbar_init(smem_addr(&s_full[s]), 1);
         mbar_init(smem_addr(&s_empty[s]), 1);
@@ -336,6 +360,12 @@ __global__ void __launch_bounds__(swap_threads<EPI>(), 1)
         mbar_init(smem_addr(&s_xempty[x]), 32);
       }
       mbar_init(smem_addr(&s_drain), 1);
+      // readers of a ring slot: the leader's MMA warp and epilogue warps, the
+      // peer's producer and epilogue warps (one elected lane each)
+      for (int q = 0; q < kTq; ++q) {
+        mbar_init(smem_addr(&s_tq_full[q]), 1);
+        mbar_init(smem_addr(&s_tq_empty[q]), 2 + 2 * swap_epi_warps<EPI>());
+      }
       fence_mbar_init();
       tma_prefetch_desc(&maps.w);
       tma_prefetch_desc(&maps.x);
@@ -354,6 +384,41 @@ __global__ void __launch_bounds__(swap_threads<EPI>(), 1)
   const int total = s_total;
   const int num_kb = (args.K + kBK - 1) / kBK;
   volatile int* abort_flag = &s_abort;
+  const bool dyn = s_dyn != 0;
+
+  // Dynamic schedule.  The leader's producer posts lane 0's `tile` as round
+  // i's to ring slot i % kTq of both CTAs (warp-uniform; false when the
+  // wait for a free slot gave up).  It claims each tile from the counter
+  // one round before posting it, so the atomic's round trip overlaps a
+  // whole tile of loads.
+  auto tq_post = [&](int i, int tile) -> bool {
+    const int r = i & (kTq - 1);
+    if (!mbar_wait_all(smem_addr(&s_tq_empty[r]), ((i / kTq) & 1) ^ 1u, abort_flag, args.status)) return false;
+    if (lane == 0) {
+      s_tq[r] = tile;
+      st_shared_cluster_u32(mapa_shared(smem_addr(&s_tq[r]), 1), tile);
+      mbar_arrive(smem_addr(&s_tq_full[r]));
+      mbar_arrive_remote(mapa_shared(smem_addr(&s_tq_full[r]), 1));
+    }
+    __syncwarp();
+    return true;
+  };
+  // Every other role reads round i's tile from its own CTA's ring and
+  // releases the slot to the leader (warp-uniform; okr = false on give-up).
+  auto tq_take = [&](int i, bool& okr) -> int {
+    const int r = i & (kTq - 1);
+    if (!mbar_wait_all_cluster(smem_addr(&s_tq_full[r]), (i / kTq) & 1, abort_flag, args.status)) {
+      okr = false;
+      return 0;
+    }
+    const int tile = *reinterpret_cast<volatile int*>(&s_tq[r]);
+    __syncwarp();
+    if (lane == 0) {
+      if (leader) mbar_arrive(smem_addr(&s_tq_empty[r]));
+      else mbar_arrive_remote(mapa_shared(smem_addr(&s_tq_empty[r]), 0));
+    }
+    return tile;
+  };
 
   // The producer and MMA loops run on whole warps with warp-uniform control
   // (stage, phase, tile); only lane 0 issues the TMA copies, MMAs and
@@ -363,7 +428,34 @@ __global__ void __launch_bounds__(swap_threads<EPI>(), 1)
     // -------------------------------------------------------- TMA producer
     uint32_t s = 0, ph = 0;
     bool ok = true;
-    for (int rd = 0, tile = unit; ok && tile < total; ++rd, tile = swap_tile_at(rd, unit, units)) {
+    // dynamic schedule, leader: `cur` is this round's tile (posted); lane 0's
+    // `claimed` is the next round's, taken from the counter a round earlier
+    int cur = 0, claimed = 0;
+    if (dyn && leader) {
+      int first = 0;
+      if (lane == 0) {
+        first = atomicAdd(args.tile_ctr, 1);
+        claimed = atomicAdd(args.tile_ctr, 1);
+      }
+      ok = tq_post(0, first);
+      cur = __shfl_sync(0xffffffffu, first, 0);
+    }
+    for (int rd = 0; ok; ++rd) {
+      int tile;
+      if (!dyn) {
+        tile = swap_tile_at(rd, unit, units);
+      } else if (leader) {
+        tile = cur;
+        if (tile < total) {
+          if (!tq_post(rd + 1, claimed)) break;
+          cur = __shfl_sync(0xffffffffu, claimed, 0);
+          if (cur < total && lane == 0) claimed = atomicAdd(args.tile_ctr, 1);
+        }
+      } else {
+        tile = tq_take(rd, ok);
+        if (!ok) break;
+      }
+      if (tile >= total) break;
       const SwapTile t = swap_decode<LAYOUT>(tile, G, s_tstart, s_cnt, args, num_kb);
       // kSwFwd / kSwDgrad: B = this CTA's half of the token tile, K-major rows.
       // kSwWgrad: B = this CTA's 128 of the tile's 256 B columns, rows of the segment.
@@ -421,7 +513,15 @@ __global__ void __launch_bounds__(swap_threads<EPI>(), 1)
       const uint64_t da0 = kAMn ? sw128_mnmajor_desc(smem_base, 64 * kBK * 2) : sw128_kmajor_desc(smem_base);
       const uint64_t db0 = kBMn ? sw128_mnmajor_desc(smem_base + kSwKB * kSwATileBytes, 64 * kBK * 2)
                                 : sw128_kmajor_desc(smem_base + kSwKB * kSwATileBytes);
-      for (int rd = 0, tile = unit; ok && tile < total; ++rd, tile = swap_tile_at(rd, unit, units), ++it) {
+      for (int rd = 0; ok; ++rd, ++it) {
+        int tile;
+        if (dyn) {
+          tile = tq_take(rd, ok);
+          if (!ok) break;
+        } else {
+          tile = swap_tile_at(rd, unit, units);
+        }
+        if (tile >= total) break;
         const SwapTile t = swap_decode<LAYOUT>(tile, G, s_tstart, s_cnt, args, num_kb);
         const uint32_t idesc = umma_idesc_bf16_major(256, t.n, kAMn ? 1 : 0, kBMn ? 1 : 0);
         const uint32_t buf = it & 1u;
@@ -476,7 +576,15 @@ __global__ void __launch_bounds__(swap_threads<EPI>(), 1)
     const uint32_t stg = smem_base + kSwWgStages * kSwStageBytes + (warp - 2) * 2 * kSwWgStageBufBytes;
     float* stgp = reinterpret_cast<float*>(dyn_smem + (stg - smem_addr(dyn_smem)));
     bool ok = true;
-    for (int rd = 0, tile = unit; ok && tile < total; ++rd, tile = swap_tile_at(rd, unit, units), ++it) {
+    for (int rd = 0; ok; ++rd, ++it) {
+      int tile;
+      if (dyn) {
+        tile = tq_take(rd, ok);
+        if (!ok) break;
+      } else {
+        tile = swap_tile_at(rd, unit, units);
+      }
+      if (tile >= total) break;
       const SwapTile t = swap_decode<LAYOUT>(tile, G, s_tstart, s_cnt, args, num_kb);
       const uint32_t buf = it & 1u;
       const uint32_t tph = (it >> 1) & 1u;

@@ -98,6 +98,8 @@ struct SwapLaunch {
   float* parts; int ld_parts;
   int half_cols;
   const int* counts;         // optional [G]: rows computed per group (segments start at offsets)
+  int* tile_ctr;             // optional: 0 at launch; with many narrow groups, tiles are claimed
+                             // from it as CTA pairs free up
 };
 cudaError_t launch_gemm_swap(const SwapLaunch& L, cudaStream_t s);
 

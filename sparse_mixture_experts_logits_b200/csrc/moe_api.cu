@@ -267,7 +267,8 @@ moe_status_t run_route(const void* x, const void* w_r, const float* e_bias, int 
 moe_status_t run_experts(const moe_layer_desc_t* d, const moe_weights_t* w, const void* x,
                          const int32_t* offsets, const int32_t* row_token, const float* row_w,
                          void* out_perm, void* x_perm, void* h, int* status, cudaStream_t s,
-                         const Marks& mk = Marks(), const int32_t* slot_of = nullptr) {
+                         const Marks& mk = Marks(), const int32_t* slot_of = nullptr,
+                         int* tile_ctrs = nullptr) {
   const int pairs = d->T * d->k;
   const bool swiglu = d->act == MOE_ACT_SWIGLU;
   const int n1 = swiglu ? 2 * d->I : d->I;
@@ -343,6 +344,7 @@ moe_status_t run_experts(const moe_layer_desc_t* d, const moe_weights_t* w, cons
     g1.w_tiles = (d->I + g1.cols_per_tile - 1) / g1.cols_per_tile;
     g1.out_cols = d->I; g1.ldo = d->I; g1.out = h;
     g1.status = status;
+    g1.tile_ctr = tile_ctrs;
     MOE_CUDA(launch_gemm_swap(g1, s));
     MOE_TRY(mk.at(4));
 
@@ -357,6 +359,7 @@ moe_status_t run_experts(const moe_layer_desc_t* d, const moe_weights_t* w, cons
     g2.out_cols = d->D; g2.ldo = d->D; g2.out = out_perm;
     g2.row_scale = row_w; g2.bias = b2;
     g2.status = status;
+    g2.tile_ctr = tile_ctrs != nullptr ? tile_ctrs + 1 : nullptr;
     MOE_CUDA(launch_gemm_swap(g2, s));
     MOE_TRY(mk.at(5));
   } else {
@@ -882,7 +885,11 @@ static moe_status_t forward_impl(const moe_layer_desc_t* d, const moe_weights_t*
   float* row_w = at<float*>(ws, L.pub.row_w);
   void* out_perm = at<void*>(ws, L.pub.out_perm);
   Range whole("moe_forward");
-  MOE_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
+  // the status flag and, in the same 256-byte slot of the workspace, the
+  // tile counters of the two routed expert GEMMs (ints 2 and 3), which
+  // must be 0 when their launches start
+  int* tile_ctrs = status + 2;
+  MOE_CUDA(cudaMemsetAsync(status, 0, 4 * sizeof(int), s));
   // At decode sizes the shared expert's two GEMMs stream their weights
   // through a few CTA pairs, each waiting on its whole K in turn, while the
   // routing stage's small kernels leave most SMs idle.  The shared expert
@@ -921,7 +928,7 @@ static moe_status_t forward_impl(const moe_layer_desc_t* d, const moe_weights_t*
   {
     Range r("moe.experts");
     MOE_TRY(run_experts(d, w, x, offsets, row_token, row_w, out_perm, at<void*>(ws, L.x_perm),
-                        at<void*>(ws, L.h), status, s, mk, by_token ? slot_of : nullptr));
+                        at<void*>(ws, L.h), status, s, mk, by_token ? slot_of : nullptr, tile_ctrs));
   }
   if (shared_done) {
     MOE_TRY(shared_fork.join());

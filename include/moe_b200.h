@@ -120,7 +120,9 @@ typedef struct {
  * forward pass leaves there (valid after the stream reaches the end of a
  * moe_forward call).  Exposed so that tests can check every stage. */
 typedef struct {
-  size_t status;    /* int32 device status flag */
+  size_t status;    /* int32 device status flag; the 256-byte slot it starts
+                       also holds, as int32 words 2 and 3, the routed expert
+                       GEMMs' tile counters (zeroed by each moe_forward) */
   size_t topk_idx;  /* int32 [T, k] */
   size_t topk_w;    /* fp32  [T, k] */
   size_t counts;    /* int32 [M] */
